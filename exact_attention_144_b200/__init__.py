@@ -1,0 +1,212 @@
+"""Exact attention for NVIDIA B200 (sm_100a): thin Python binding of the C ABI.
+
+The functions here carry the C entry points' names (``fa_fwd``, ``fa_fwd_f16``,
+``fa_bwd``, ``fa_bwd_f16``, ...) and only marshal arguments: they check torch
+tensors, allocate outputs when asked, and pass raw device pointers and the
+current CUDA stream to ``libfa_b200.so``.  Every step of the computation runs
+in the library's CUDA kernels; there is no other implementation to fall back
+on: the first call fails loudly when the library has not been built.
+
+Layout: q, k, v, o, dout, dq, dk, dv are contiguous [B, N, H, d] tensors of
+bfloat16 (``fa_fwd``/``fa_bwd``) or float16 (``*_f16``); lse is a contiguous
+[B, H, N] float32 tensor (natural log).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa_b200.h")
+
+_lib = None
+
+
+def _load() -> ctypes.CDLL:
+    """Load libfa_b200.so once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m exact_attention_144_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp]
+    lib.fa_fwd_f16.argtypes = lib.fa_fwd.argtypes
+    lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, f, vp]
+    lib.fa_bwd_f16.argtypes = lib.fa_bwd.argtypes
+    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16"):
+        getattr(lib, n).restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), i]
+    lib.fa_get_device_status.restype = i
+    lib.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.fa_selftest_bounded_wait.restype = i
+    lib.fa_version.restype = i
+    _lib = lib
+    return lib
+
+
+FA_OK = 0
+FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_ALIGN = -1, -2, -3, -4
+FA_ERR_LAUNCH, FA_ERR_NOMEM, FA_ERR_DEVICE, FA_ERR_SCALE = -5, -6, -7, -8
+
+
+class FAError(RuntimeError):
+    def __init__(self, where: str, status: int):
+        super().__init__(f"{where}: {fa_status_string(status)} (status {status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (for callers that want the raw entry points)."""
+    return _load()
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/fa_b200.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)
+
+
+def fa_status_string(status: int) -> str:
+    return _load().fa_status_string(int(status)).decode()
+
+
+def fa_version() -> int:
+    return int(_load().fa_version())
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check_bnhd(name: str, t: torch.Tensor, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _fwd(entry: str, dtype, q, k, v, o, lse, scale, stream):
+    _check_bnhd("q", q, dtype)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, N, H, d]")
+    B, N, H, d = q.shape
+    _check_bnhd("k", k, dtype, q.shape)
+    _check_bnhd("v", v, dtype, q.shape)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_bnhd("o", o, dtype, q.shape)
+    _check_bnhd("lse", lse, torch.float32, (B, H, N))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                              float(scale), _stream(stream))
+    if rc != FA_OK:
+        raise FAError(entry, rc)
+    return o, lse
+
+
+def _bwd(entry: str, dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream):
+    _check_bnhd("q", q, dtype)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, N, H, d]")
+    B, N, H, d = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_bnhd(name, t, dtype, q.shape)
+    _check_bnhd("lse", lse, torch.float32, (B, H, N))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bnhd(name, t, dtype, q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                              _stream(stream))
+    if rc != FA_OK:
+        raise FAError(entry, rc)
+    return dq, dk, dv
+
+
+def fa_fwd(q, k, v, o=None, lse=None, scale=None, stream=None):
+    """bf16 forward: returns (o, lse); allocates them when not given."""
+    return _fwd("fa_fwd", torch.bfloat16, q, k, v, o, lse, scale, stream)
+
+
+def fa_fwd_f16(q, k, v, o=None, lse=None, scale=None, stream=None):
+    """fp16 forward: returns (o, lse); allocates them when not given."""
+    return _fwd("fa_fwd_f16", torch.float16, q, k, v, o, lse, scale, stream)
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, stream=None):
+    """bf16 backward by recompute: returns (dq, dk, dv) (overwritten, not accumulated)."""
+    return _bwd("fa_bwd", torch.bfloat16, q, k, v, o, dout, lse, dq, dk, dv, scale, stream)
+
+
+def fa_bwd_f16(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, stream=None):
+    """fp16 backward by recompute: returns (dq, dk, dv)."""
+    return _bwd("fa_bwd_f16", torch.float16, q, k, v, o, dout, lse, dq, dk, dv, scale, stream)
+
+
+_FWD = {torch.bfloat16: fa_fwd, torch.float16: fa_fwd_f16}
+_BWD = {torch.bfloat16: fa_bwd, torch.float16: fa_bwd_f16}
+
+
+def forward(q, k, v, scale=None, o=None, lse=None, stream=None):
+    """fa_fwd or fa_fwd_f16, chosen by q's element type."""
+    if q.dtype not in _FWD:
+        raise TypeError(f"unsupported element type {q.dtype}")
+    return _FWD[q.dtype](q, k, v, o=o, lse=lse, scale=scale, stream=stream)
+
+
+def backward(q, k, v, o, dout, lse, scale=None, dq=None, dk=None, dv=None, stream=None):
+    """fa_bwd or fa_bwd_f16, chosen by q's element type."""
+    if q.dtype not in _BWD:
+        raise TypeError(f"unsupported element type {q.dtype}")
+    return _BWD[q.dtype](q, k, v, o, dout, lse, dq=dq, dk=dk, dv=dv, scale=scale, stream=stream)
+
+
+def fa_get_device_status(clear: bool = False) -> int:
+    """The device status word (0 = no bounded wait gave up).  Synchronises."""
+    out = ctypes.c_ulonglong(0)
+    rc = _load().fa_get_device_status(ctypes.byref(out), 1 if clear else 0)
+    if rc != FA_OK:
+        raise FAError("fa_get_device_status", rc)
+    return int(out.value)
+
+
+def fa_selftest_bounded_wait(limit_us: int = 20000) -> int:
+    """Runs the bounded-wait self test; returns the status it recorded."""
+    out = ctypes.c_ulonglong(0)
+    rc = _load().fa_selftest_bounded_wait(int(limit_us), ctypes.byref(out))
+    if rc != FA_OK:
+        raise FAError("fa_selftest_bounded_wait", rc)
+    return int(out.value)

@@ -1,0 +1,260 @@
+// fa_api.cu -- the C ABI: argument validation, device checks, TMA tensor-map
+// encoding and the device status word.  No torch types cross this boundary.
+#include <math.h>
+#include <mutex>
+
+#include "fa_common.cuh"
+#include "fa_host.h"
+
+namespace fa {
+
+__device__ unsigned long long g_status = 0;
+
+unsigned long long* device_status_ptr() {
+  static std::mutex mu;
+  static unsigned long long* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status) == cudaSuccess)
+      cached[dev] = static_cast<unsigned long long*>(ptr);
+    else
+      cudaGetLastError();
+  }
+  return cached[dev];
+}
+
+// ------------------------------------------------------------ device info
+int current_device(DeviceInfo* info) {
+  static std::mutex mu;
+  static int cached_sm[64] = {0};
+  static int cached_smem[64] = {0};
+  static int cached_ok[64] = {0};  // 0 unknown, 1 sm_100, -1 other
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  if (dev < 0 || dev >= 64) return FA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached_ok[dev] == 0) {
+    int major = 0, minor = 0, sms = 0, smem = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    cached_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    cached_sm[dev] = sms;
+    cached_smem[dev] = smem;
+  }
+  if (cached_ok[dev] != 1) return FA_ERR_DEVICE;
+  info->device = dev;
+  info->sm_count = cached_sm[dev];
+  info->max_smem_optin = cached_smem[dev];
+  return FA_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d,
+                   int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_LAUNCH;
+  // dims innermost first: element within head, head, token, batch
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
+                                 (cuuint64_t)N * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int make_tmap_f32_rows(CUtensorMap* map, const void* base, size_t rows, int cols, int box_cols,
+                       int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------ validation
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_common(int B, int H, int N, int d, float scale, bool bwd) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  if (bwd ? !(d == 64) : !(d == 64 || d == 128 || d == 256)) return FA_ERR_HEADDIM;
+  if ((long long)B * N * H * d >= (1ll << 31)) return FA_ERR_SHAPE;
+  if (!isfinite(scale)) return FA_ERR_SCALE;
+  return FA_OK;
+}
+
+static int check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (p == nullptr) return FA_ERR_NULL;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+template <class T>
+static int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, float scale, cudaStream_t stream) {
+  int rc = check_ptrs({q, k, v, o, lse});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK) rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, stream);
+  return rc;
+}
+
+template <class T>
+static int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                     float scale, cudaStream_t stream) {
+  int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK)
+    rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, stream);
+  return rc;
+}
+
+// ---------------------------------------------------- bounded-wait test
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned long long* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    // expects two arrivals; only one ever comes, so the phase never completes
+    mbar_init(smem_u32(&bar), 2);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive(smem_u32(&bar));
+    const WaitCtl w{&abort_flag, limit_ns, status};
+    mbar_wait(smem_u32(&bar), 0, w, 0x7F);
+  }
+  __syncthreads();
+}
+
+}  // namespace fa
+
+// =================================================================== C ABI
+// Only these entry points are visible outside the library.
+#define FA_EXPORT __attribute__((visibility("default")))
+
+extern "C" {
+
+FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, cudaStream_t stream) {
+  return fa::fwd_entry<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, stream);
+}
+
+FA_EXPORT int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, cudaStream_t stream) {
+  return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, stream);
+}
+
+FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+           cudaStream_t stream) {
+  return fa::bwd_entry<__nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale,
+                                      stream);
+}
+
+FA_EXPORT int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+               float scale, cudaStream_t stream) {
+  return fa::bwd_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, stream);
+}
+
+FA_EXPORT const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "a required pointer is NULL";
+    case FA_ERR_SHAPE: return "B, H or N below 1, or a tensor of 2^31 or more elements";
+    case FA_ERR_HEADDIM: return "head dimension not supported by this entry point";
+    case FA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FA_ERR_LAUNCH: return "the CUDA runtime rejected a launch or call";
+    case FA_ERR_NOMEM: return "scratch allocation failed";
+    case FA_ERR_DEVICE: return "current device is not compute capability 10.0 (B200)";
+    case FA_ERR_SCALE: return "scale is NaN or infinite";
+    default: return "unknown status";
+  }
+}
+
+FA_EXPORT int fa_get_device_status(unsigned long long* status_out, int clear) {
+  if (status_out == nullptr) return FA_ERR_NULL;
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  *status_out = v;
+  if (clear) {
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(zero)) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+  }
+  return FA_OK;
+}
+
+FA_EXPORT int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long* status_out) {
+  if (status_out == nullptr) return FA_ERR_NULL;
+  if (limit_us < 1 || limit_us > 10000000u) return FA_ERR_SHAPE;
+  fa::DeviceInfo dev;
+  int rc = fa::current_device(&dev);
+  if (rc != FA_OK) return rc;
+  unsigned long long prev = 0;
+  if ((rc = fa_get_device_status(&prev, 1)) != FA_OK) return rc;
+  fa::selftest_wait_kernel<<<1, 32>>>((unsigned long long)limit_us * 1000ull,
+                                      fa::device_status_ptr());
+  if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return fa_get_device_status(status_out, 1);
+}
+
+FA_EXPORT int fa_version(void) { return 100; }
+
+}  // extern "C"

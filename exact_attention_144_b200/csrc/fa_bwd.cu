@@ -1,0 +1,563 @@
+// fa_bwd.cu -- backward pass of exact attention on sm_100a, by recompute.
+//
+// The forward keeps only O and the per-row LSE; the backward rebuilds P from
+// Q, K and the LSE instead of storing it (LLM explainer page, section 6.2,
+// recompute strategy; YOLO11 page, section 2.3).  With c = scale * log2(e):
+//   P^T  = exp2(c K Q^T - LSE * log2(e))      (no max or sum: LSE is saved)
+//   dV  += P^T dO
+//   dP^T = V dO^T,   dS^T = P^T o (dP^T - D),   D_i = sum_x dO_ix O_ix
+//   dK  += scale dS^T Q
+//   dQ  += scale dS K   (fp32, reduced into global memory across K/V tiles)
+//
+// Three kernels:
+//   fa_bwd_pre_kernel   D, base-2 LSE (padded to whole Q tiles) and a zeroed
+//                       fp32 dQ accumulator
+//   fa_bwd_kernel       one block per (K/V tile of 128 keys, head, batch); its
+//                       loop walks the Q tiles of 128 queries
+//   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to 16 bits
+//
+// fa_bwd_kernel layout (320 threads, one block per SM):
+//   warps 0-3  recompute P^T and dS^T; thread t owns key row t (TMEM lane t);
+//              epilogue for dK and dV
+//   warps 4-7  dQ drain: TMEM -> shared memory -> bulk reduce-add to global
+//   warp  8    TMA producer
+//   warp  9    TMEM allocator and tcgen05.mma issuer
+// Tensor memory (d = 64): S^T [0,128) (P^T over its first 64 columns),
+// dP^T [128,256) (dS^T over its first 64), dV [256,320), dK [320,384),
+// dQ [384,448).
+#include "fa_common.cuh"
+#include "fa_host.h"
+
+namespace fa {
+
+struct BwdTraits64 {
+  static constexpr int D = 64;
+  static constexpr int BN = 128;  // keys per block
+  static constexpr int BM = 128;  // queries per inner tile
+  static constexpr int QST = 2;   // Q / dO stages
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int QT_BYTES = BM * D * 2;
+  static constexpr int DS_BYTES = BN * BM * 2;       // dS tile, 16-bit
+  static constexpr int STAGE_BYTES = BM * D * 4;     // dQ tile, fp32
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + QST * QT_BYTES;
+  static constexpr int OFF_DS = OFF_DO + QST * QT_BYTES;
+  static constexpr int OFF_STG = OFF_DS + 2 * DS_BYTES;
+  static constexpr int OFF_L = OFF_STG + STAGE_BYTES;  // base-2 LSE per stage
+  static constexpr int OFF_DD = OFF_L + QST * BM * 4;  // D per stage
+  static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
+  static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
+                       B_S_FULL = B_Q_EMPTY + QST, B_DP_FULL = B_S_FULL + 1,
+                       B_DS_READY = B_DP_FULL + 1, B_DSBUF_FREE = B_DS_READY + 1,
+                       B_DQ_FULL = B_DSBUF_FREE + 2, B_DQ_FREE = B_DQ_FULL + 1,
+                       B_KV_DONE = B_DQ_FREE + 1, B_DRAIN = B_KV_DONE + 1,
+                       NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct BwdParams {
+  const float* lse2;  // [B, H, Npad] base-2 LSE, +inf past N
+  const float* dvec;  // [B, H, Npad] D, 0 past N
+  float* dq_acc;      // [B, H, Npad, D] fp32
+  void* dk;           // [B, N, H, D]
+  void* dv;
+  int B, H, N, Npad, n_qt;
+  float sl2;          // scale * log2(e)
+  float scale;
+  unsigned long long limit_ns;
+  unsigned long long* status;
+};
+
+enum { kBSiteQEmpty = 0x21, kBSiteKV, kBSiteQFull, kBSiteDsReady, kBSiteDqFree, kBSiteSFull,
+       kBSiteDpFull, kBSiteQFullSm, kBSiteDsBuf, kBSiteDqFull, kBSiteKvDone };
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Reduce-add of a shared-memory tile into global memory through a tensor map
+// (element type, box and swizzle come from the map).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int c0,
+                                                  int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <class T, class Tr>
+__global__ void __launch_bounds__(320, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
+                  const __grid_constant__ CUtensorMap tmacc, const BwdParams p) {
+  constexpr int D = Tr::D, BN = Tr::BN, BM = Tr::BM, QST = Tr::QST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + Tr::OFF_K, sV = base + Tr::OFF_V, sQ = base + Tr::OFF_Q,
+                 sDO = base + Tr::OFF_DO, sDS = base + Tr::OFF_DS, sSTG = base + Tr::OFF_STG;
+  const float* sL = reinterpret_cast<const float*>(gbase + Tr::OFF_L);
+  const float* sDD = reinterpret_cast<const float*>(gbase + Tr::OFF_DD);
+  uint8_t* gDS = gbase + Tr::OFF_DS;
+  uint8_t* gSTG = gbase + Tr::OFF_STG;
+  const uint32_t bars = base + Tr::OFF_BAR;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + Tr::OFF_MISC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + Tr::OFF_MISC + 4);
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtl w{abort_flag, p.limit_ns, p.status};
+  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n_qt = p.n_qt;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(Tr::B_KV_FULL), 1);
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(bar(Tr::B_Q_FULL + s), 1);
+      mbar_init(bar(Tr::B_Q_EMPTY + s), 1);
+    }
+    mbar_init(bar(Tr::B_S_FULL), 1);
+    mbar_init(bar(Tr::B_DP_FULL), 1);
+    mbar_init(bar(Tr::B_DS_READY), 128);
+    mbar_init(bar(Tr::B_DSBUF_FREE), 1);
+    mbar_init(bar(Tr::B_DSBUF_FREE + 1), 1);
+    mbar_init(bar(Tr::B_DQ_FULL), 1);
+    mbar_init(bar(Tr::B_DQ_FREE), 128);
+    mbar_init(bar(Tr::B_KV_DONE), 1);
+    mbar_init(bar(Tr::B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), Tr::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // -------------------------------------------------------- producer
+    if (lane == 0) {
+      mbar_expect_tx(bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
+      tma_load_4d(sK, &tmk, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
+      tma_load_4d(sV, &tmv, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
+      const size_t row0 = ((size_t)b * p.H + h) * p.Npad;
+      int issued = 0;
+      for (int i = 0; i < n_qt; ++i) {
+        const int qs = i % QST;
+        if (i >= QST &&
+            !mbar_wait(bar(Tr::B_Q_EMPTY + qs), ((i / QST) - 1) & 1, w, kBSiteQEmpty))
+          break;
+        const uint32_t fb = bar(Tr::B_Q_FULL + qs);
+        mbar_expect_tx(fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
+        tma_load_4d(sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, i * BM, b);
+        tma_load_4d(sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, i * BM, b);
+        bulk_load(base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
+        bulk_load(base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
+        ++issued;
+      }
+      mbar_drain(bar(Tr::B_KV_FULL), 0, p.limit_ns);
+      for (int s = 0; s < QST; ++s)
+        if (issued > s) mbar_drain(bar(Tr::B_Q_FULL + s), ((issued - 1 - s) / QST) & 1, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ----------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = Elem<T>::kFmt;
+      constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);       // K-major x K-major
+      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);        // TS, B MN-major
+      constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, D, true) | (1u << 15);  // A, B MN-major
+      bool ok = mbar_wait(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
+      tc_fence_after();
+      for (int i = 0; i < n_qt && ok; ++i) {
+        const int qs = i % QST;
+        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL + qs), (i / QST) & 1, w, kBSiteQFull))) break;
+        tc_fence_after();
+        const uint32_t q_s = sQ + qs * Tr::QT_BYTES, do_s = sDO + qs * Tr::QT_BYTES;
+        // S^T = K Q^T and dP^T = V dO^T (both K-major over d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
+          umma_ss(tmem + Tr::TM_S, sw128_desc(sK + ch * (BN * 128) + in, 16, 1024),
+                  sw128_desc(q_s + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(Tr::B_S_FULL));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
+          umma_ss(tmem + Tr::TM_DP, sw128_desc(sV + ch * (BN * 128) + in, 16, 1024),
+                  sw128_desc(do_s + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(Tr::B_DP_FULL));
+        // P^T and dS^T written by the softmax warps
+        if (!(ok = mbar_wait(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+        tc_fence_after();
+        // dV += P^T dO ; dK += dS^T Q   (A from TMEM, B MN-major: queries x d)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_S + kk * 8,
+                  sw128_desc(do_s + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DP + kk * 8,
+                  sw128_desc(q_s + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(Tr::B_Q_EMPTY + qs));
+        // dQ_i = dS K: A = dS (queries contiguous), B = K (d contiguous)
+        if (i > 0 && !(ok = mbar_wait(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree))) break;
+        tc_fence_after();
+        const uint32_t ds_s = sDS + (i & 1) * Tr::DS_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ss(tmem + Tr::TM_DQ, sw128_desc(ds_s + kk * 16 * 128, BN * 128, 1024),
+                  sw128_desc(sK + kk * 16 * 128, BN * 128, 1024), kIdescDQ, kk > 0 ? 1u : 0u);
+        umma_commit(bar(Tr::B_DQ_FULL));
+        umma_commit(bar(Tr::B_DSBUF_FREE + (i & 1)));
+      }
+      umma_commit(bar(Tr::B_KV_DONE));
+      umma_commit(bar(Tr::B_DRAIN));
+      mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------- P^T, dS^T and dK/dV epilogue
+    const int r = threadIdx.x;  // key row within the tile
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const bool key_valid = kt * BN + r < p.N;
+    bool ok = true;
+    for (int i = 0; i < n_qt; ++i) {
+      const int qs = i % QST;
+      ok = mbar_wait(bar(Tr::B_S_FULL), i & 1, w, kBSiteSFull);
+      ok = ok && mbar_wait(bar(Tr::B_Q_FULL + qs), (i / QST) & 1, w, kBSiteQFullSm);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float* lrow = sL + qs * BM;
+      const float* drow = sDD + qs * BM;
+      float pr[BM];
+      {
+        uint32_t sr[BM / 32][32];
+#pragma unroll
+        for (int c = 0; c < BM / 32; ++c) tmem_ld32(tl + Tr::TM_S + c * 32, sr[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < BM / 32; ++c) reg_fence(sr[c]);
+#pragma unroll
+        for (int j = 0; j < BM; ++j)
+          pr[j] = key_valid ? ex2(__uint_as_float(sr[j / 32][j % 32]) * p.sl2 - lrow[j]) : 0.f;
+      }
+      {
+        uint32_t pk[BM / 2];
+#pragma unroll
+        for (int j = 0; j < BM / 2; ++j) pk[j] = Elem<T>::pack(pr[2 * j], pr[2 * j + 1]);
+#pragma unroll
+        for (int c = 0; c < BM / 32; ++c) tmem_st16(tl + Tr::TM_S + c * 16, &pk[c * 16]);
+      }
+      ok = mbar_wait(bar(Tr::B_DP_FULL), i & 1, w, kBSiteDpFull);
+      if (i >= 2) ok = ok && mbar_wait(bar(Tr::B_DSBUF_FREE + (i & 1)), ((i >> 1) - 1) & 1, w,
+                                       kBSiteDsBuf);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      uint32_t dk16[BM / 2];
+#pragma unroll
+      for (int c = 0; c < BM / 32; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(tl + Tr::TM_DP + c * 32, dr);
+        tmem_wait_ld();
+        reg_fence(dr);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int q0 = c * 32 + 2 * j;
+          const float ds0 = pr[q0] * (__uint_as_float(dr[2 * j]) - drow[q0]);
+          const float ds1 = pr[q0 + 1] * (__uint_as_float(dr[2 * j + 1]) - drow[q0 + 1]);
+          dk16[c * 16 + j] = Elem<T>::pack(ds0, ds1);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BM / 32; ++c) tmem_st16(tl + Tr::TM_DP + c * 16, &dk16[c * 16]);
+      // dS row r into shared memory for the dQ MMA: 128-byte-swizzled,
+      // queries contiguous (two 64-query chunks of 128 key rows each).
+      uint8_t* ds_g = gDS + (i & 1) * Tr::DS_BYTES;
+#pragma unroll
+      for (int u = 0; u < BM / 8; ++u) {
+        const int chunk = u >> 3, unit = u & 7;
+        uint4 val = make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2], dk16[4 * u + 3]);
+        *reinterpret_cast<uint4*>(ds_g + chunk * (BN * 128) + r * 128 + ((unit ^ (r & 7)) * 16)) =
+            val;
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_DS_READY));
+    }
+    // epilogue: dV and scale * dK for this block's key rows
+    if (ok) ok = mbar_wait(bar(Tr::B_KV_DONE), 0, w, kBSiteKvDone);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const int key = kt * BN + r;
+      T* dvrow = reinterpret_cast<T*>(p.dv) + (((size_t)b * p.N + key) * p.H + h) * D;
+      T* dkrow = reinterpret_cast<T*>(p.dk) + (((size_t)b * p.N + key) * p.H + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32], k2[32];
+        tmem_ld32(tl + Tr::TM_DV + c * 32, a);
+        tmem_ld32(tl + Tr::TM_DK + c * 32, k2);
+        tmem_wait_ld();
+        reg_fence(a);
+        reg_fence(k2);
+        uint4 va[4], vk[4];
+        uint32_t* pa = reinterpret_cast<uint32_t*>(va);
+        uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
+          pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
+                                 __uint_as_float(k2[2 * j + 1]) * p.scale);
+        }
+        if (key_valid) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            reinterpret_cast<uint4*>(dvrow + c * 32)[j] = va[j];
+            reinterpret_cast<uint4*>(dkrow + c * 32)[j] = vk[j];
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------- dQ drain (warps 4-7)
+    const int t = threadIdx.x - 128;  // query row within the tile
+    const uint32_t tl = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    bool ok = true;
+    for (int i = 0; i < n_qt; ++i) {
+      ok = mbar_wait(bar(Tr::B_DQ_FULL), i & 1, w, kBSiteDqFull);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      uint32_t v[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tl + Tr::TM_DQ + c * 32, v[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence(v[c]);
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_DQ_FREE));
+      named_bar_sync(1, 128);  // the previous reduce has read the staging tile
+      // Row t of the fp32 staging tile, as two 32-column boxes of 128-byte rows
+      // with the 128-byte swizzle (16-byte unit w of row t at w ^ (t & 7)).
+#pragma unroll
+      for (int u = 0; u < D / 4; ++u) {
+        const int box = u >> 3, wu = u & 7;
+        float4 val = make_float4(__uint_as_float(v[(4 * u) / 32][(4 * u) % 32]),
+                                 __uint_as_float(v[(4 * u + 1) / 32][(4 * u + 1) % 32]),
+                                 __uint_as_float(v[(4 * u + 2) / 32][(4 * u + 2) % 32]),
+                                 __uint_as_float(v[(4 * u + 3) / 32][(4 * u + 3) % 32]));
+        *reinterpret_cast<float4*>(gSTG + box * (BM * 128) + t * 128 + ((wu ^ (t & 7)) * 16)) =
+            val;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (t == 0) {
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM);
+#pragma unroll
+        for (int box = 0; box < D / 32; ++box)
+          tma_reduce_add_2d(&tmacc, sSTG + box * (BM * 128), box * 32, row);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+    }
+    if (t == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Tr::TMEM_COLS);
+  }
+}
+
+// D_i = sum_x dO_ix O_ix; base-2 LSE; zero the dQ accumulator.  One warp per
+// padded row (b, h, i); rows past N get D = 0 and LSE = +inf (so P = 0 there).
+template <class T, int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o,
+                                                         const T* __restrict__ dout,
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ lse2,
+                                                         float* __restrict__ dvec,
+                                                         float* __restrict__ dq_acc, int B, int H,
+                                                         int N, int Npad) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)B * H * Npad) return;
+  const int i = (int)(row % Npad);
+  const int h = (int)((row / Npad) % H);
+  const int b = (int)(row / ((long long)Npad * H));
+  constexpr int PER = D / 32;
+  float acc = 0.f;
+  if (i < N) {
+    const T* orow = o + (((size_t)b * N + i) * H + h) * D + lane * PER;
+    const T* drow = dout + (((size_t)b * N + i) * H + h) * D + lane * PER;
+#pragma unroll
+    for (int j = 0; j < PER; j += 2) {
+      const float2 a = Elem<T>::unpack(*reinterpret_cast<const uint32_t*>(orow + j));
+      const float2 c = Elem<T>::unpack(*reinterpret_cast<const uint32_t*>(drow + j));
+      acc += a.x * c.x + a.y * c.y;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float* arow = dq_acc + (size_t)row * D + lane * PER;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) arow[j] = 0.f;
+  if (lane == 0) {
+    dvec[row] = acc;
+    lse2[row] = (i < N) ? lse[((size_t)b * H + h) * N + i] * kLog2e : INFINITY;
+  }
+}
+
+// dQ = scale * accumulator, rounded; 8 elements per thread.
+template <class T, int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                        T* __restrict__ dq, int B, int H, int N,
+                                                        int Npad, float scale) {
+  const long long idx = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
+  const long long total = (long long)B * N * H * D;
+  if (idx >= total) return;
+  const int x = (int)(idx % D);
+  const int h = (int)((idx / D) % H);
+  const int n = (int)((idx / ((long long)D * H)) % N);
+  const int b = (int)(idx / ((long long)D * H * N));
+  const float* src = dq_acc + (((size_t)b * H + h) * Npad + n) * D + x;
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 c = *reinterpret_cast<const float4*>(src + 4);
+  uint4 out;
+  out.x = Elem<T>::pack(a.x * scale, a.y * scale);
+  out.y = Elem<T>::pack(a.z * scale, a.w * scale);
+  out.z = Elem<T>::pack(c.x * scale, c.y * scale);
+  out.w = Elem<T>::pack(c.z * scale, c.w * scale);
+  *reinterpret_cast<uint4*>(dq + idx) = out;
+}
+
+template <class T, class Tr>
+static int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
+                   cudaStream_t stream) {
+  constexpr int D = Tr::D;
+  const bool bf16 = Elem<T>::kFmt == 1;
+  CUtensorMap tmq, tmk, tmv, tmdo;
+  int rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
+
+  const int n_qt = (N + Tr::BM - 1) / Tr::BM;
+  const int Npad = n_qt * Tr::BM;
+  const size_t rows = (size_t)B * H * Npad;
+  void* ws = nullptr;
+  const size_t ws_bytes = rows * D * sizeof(float) + 2 * rows * sizeof(float);
+  if (cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_NOMEM;
+  }
+  BwdParams p{};
+  p.dq_acc = static_cast<float*>(ws);
+  float* lse2 = p.dq_acc + rows * D;
+  float* dvec = lse2 + rows;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.Npad = Npad;
+  p.n_qt = n_qt;
+  p.sl2 = scale * kLog2e;
+  p.scale = scale;
+  p.limit_ns = 4000000000ull;
+  p.status = device_status_ptr();
+
+  CUtensorMap tmacc;
+  if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::BM)) != FA_OK) {
+    cudaFreeAsync(ws, stream);
+    return rc;
+  }
+
+  fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
+      Npad);
+  rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  if (rc == FA_OK) {
+    auto kern = fa_bwd_kernel<T, Tr>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Tr::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      rc = FA_ERR_LAUNCH;
+    } else {
+      dim3 grid((N + Tr::BN - 1) / Tr::BN, H, B);
+      kern<<<grid, 320, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
+      rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+    }
+  }
+  if (rc == FA_OK) {
+    const long long total = (long long)B * N * H * D;
+    fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
+        p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
+    rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  }
+  cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+template <class T>
+int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+               float scale, cudaStream_t stream) {
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != FA_OK) return rc;
+  switch (d) {
+    case 64:
+      return run_bwd<T, BwdTraits64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, stream);
+    default:
+      return FA_ERR_HEADDIM;
+  }
+}
+
+template int bwd_launch<__nv_bfloat16>(const void*, const void*, const void*, const void*,
+                                       const void*, const float*, void*, void*, void*, int, int,
+                                       int, int, float, cudaStream_t);
+template int bwd_launch<__half>(const void*, const void*, const void*, const void*, const void*,
+                                const float*, void*, void*, void*, int, int, int, int, float,
+                                cudaStream_t);
+
+}  // namespace fa

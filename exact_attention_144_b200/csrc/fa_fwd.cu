@@ -1,0 +1,524 @@
+// fa_fwd.cu -- forward pass of exact attention on sm_100a.
+//
+// O = softmax(scale Q K^T) V and the per-row log-sum-exp, FlashAttention-2
+// style (LLM explainer page, sections 4.1-4.3 and 5.2): each work unit is one
+// 128-row Q tile of one (batch, head), whose inner loop walks the K/V tiles;
+// the online softmax keeps a running max m and running sum l per row and
+// rescales the O accumulator when m grows (YOLO11 page, section 2.2).  S and P
+// live only in tensor memory; O is written once per Q tile.
+//
+// Block layout (224 threads, one block per SM, persistent over work units):
+//   warps 0-3  softmax + epilogue; thread t owns Q row t (TMEM lane t)
+//   warp  4    TMA producer for Q and K tiles
+//   warp  5    TMA producer for V tiles
+//   warp  6    TMEM allocator and the single-thread tcgen05.mma issuer
+// Tensor memory (512 columns): S0 at [0, BN), S1 at [BN, 2BN), O at [2BN, 2BN+d).
+// S is double buffered so QK^T of tile j+1 overlaps the softmax of tile j; P
+// (16-bit) is written back over the first BN/2 columns of its S buffer and
+// consumed from there by the P.V MMA (A operand in tensor memory).
+//
+// When the (batch, head, Q tile) units cannot fill the SMs, the K/V range is
+// split and the partial results (fp32, normalised, with base-2 LSE) are merged
+// by fa_combine_kernel: O = sum_s exp(LSE_s - LSE) O_s, LSE = log sum_s exp(LSE_s).
+#include "fa_common.cuh"
+#include "fa_host.h"
+
+namespace fa {
+
+template <int D_, int BN_, int KST_, int VST_>
+struct FwdTraits {
+  static constexpr int D = D_;
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int KST = KST_;
+  static constexpr int VST = VST_;
+  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  // barrier indices
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
+                       B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
+                       B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
+                       B_O_DONE = B_P_FULL + 2, B_DRAIN = B_O_DONE + 1, NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t TM_O = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(2 * BN + D <= 512, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(D % 64 == 0 && BN % 32 == 0, "tile shape");
+};
+
+struct FwdParams {
+  void* o;          // [B, N, H, D] 16-bit, direct mode
+  float* lse;       // [B, H, N] natural log, direct mode
+  float* o_part;    // [S, B, N, H, D] fp32, split mode (null in direct mode)
+  float* lse_part;  // [S, B, H, N] base-2 log, split mode
+  int B, H, N;
+  int n_qt, n_kvt, n_split, kvt_per_split, n_units;
+  float sl2;        // scale * log2(e)
+  unsigned long long limit_ns;
+  unsigned long long* status;
+};
+
+struct Unit {
+  int b, h, qt, sp, t0, t1;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
+  Unit x;
+  x.qt = u % p.n_qt;
+  int r = u / p.n_qt;
+  x.sp = r % p.n_split;
+  r /= p.n_split;
+  x.h = r % p.H;
+  x.b = r / p.H;
+  x.t0 = x.sp * p.kvt_per_split;
+  x.t1 = min(x.t0 + p.kvt_per_split, p.n_kvt);
+  return x;
+}
+
+// Timeout sites reported in the status word.
+enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull,
+       kSiteSFull, kSiteODone, kSiteEpi };
+
+template <class T, class Tr>
+__global__ void __launch_bounds__(224, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+  constexpr int D = Tr::D, BN = Tr::BN, KST = Tr::KST, VST = Tr::VST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + Tr::OFF_Q, sK = base + Tr::OFF_K, sV = base + Tr::OFF_V;
+  const uint32_t bars = base + Tr::OFF_BAR;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + Tr::OFF_MISC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + Tr::OFF_MISC + 4);
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtl w{abort_flag, p.limit_ns, p.status};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(Tr::B_Q_FULL), 1);
+    mbar_init(bar(Tr::B_Q_EMPTY), 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(bar(Tr::B_K_FULL + s), 1);
+      mbar_init(bar(Tr::B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(bar(Tr::B_V_FULL + s), 1);
+      mbar_init(bar(Tr::B_V_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Tr::B_S_FULL + s), 1);
+      mbar_init(bar(Tr::B_P_FULL + s), 128);
+    }
+    mbar_init(bar(Tr::B_O_DONE), 1);
+    mbar_init(bar(Tr::B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 6) {
+    tmem_alloc(smem_u32(tmem_slot), Tr::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------ Q and K producer
+    if (lane == 0) {
+      uint32_t kc = 0, qc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, p);
+        if (qc > 0 && !(ok = mbar_wait(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
+        mbar_expect_tx(bar(Tr::B_Q_FULL), Tr::Q_BYTES);
+#pragma unroll
+        for (int c = 0; c < Tr::KCH; ++c)
+          tma_load_4d(sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64, un.h,
+                      un.qt * Tr::BM, un.b);
+        ++qc;
+        for (int t = un.t0; t < un.t1; ++t) {
+          const uint32_t ks = kc % KST;
+          if (kc >= (uint32_t)KST &&
+              !(ok = mbar_wait(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
+            break;
+          mbar_expect_tx(bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Tr::KCH; ++c)
+            tma_load_4d(sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
+                        c * 64, un.h, t * BN, un.b);
+          ++kc;
+        }
+      }
+      // Every issued load must land before the block exits.
+      if (qc > 0) mbar_drain(bar(Tr::B_Q_FULL), (qc - 1) & 1u, p.limit_ns);
+      for (uint32_t s = 0; s < (uint32_t)KST; ++s)
+        if (kc > s) mbar_drain(bar(Tr::B_K_FULL + s), ((kc - 1 - s) / KST) & 1u, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------ V producer
+    if (lane == 0) {
+      uint32_t vc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, p);
+        for (int t = un.t0; t < un.t1; ++t) {
+          const uint32_t vs = vc % VST;
+          if (vc >= (uint32_t)VST &&
+              !(ok = mbar_wait(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
+            break;
+          mbar_expect_tx(bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Tr::KCH; ++c)
+            tma_load_4d(sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
+                        c * 64, un.h, t * BN, un.b);
+          ++vc;
+        }
+      }
+      for (uint32_t s = 0; s < (uint32_t)VST; ++s)
+        if (vc > s) mbar_drain(bar(Tr::B_V_FULL + s), ((vc - 1 - s) / VST) & 1u, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ----------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = f16_idesc(Elem<T>::kFmt, 128, BN, false);
+      constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
+      uint32_t kc = 0, vc = 0, g = 0, uc = 0;
+      bool ok = true;
+      // O += P_j V_j for the tile whose S/P buffer use counter is gp.
+      auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+        const uint32_t pb = gp & 1u;
+        if (!mbar_wait(bar(Tr::B_P_FULL + pb), (gp >> 1) & 1u, w, kSitePFull)) return false;
+        const uint32_t vs = vc % VST;
+        if (!mbar_wait(bar(Tr::B_V_FULL + vs), (vc / VST) & 1u, w, kSiteVFull)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sV + vs * Tr::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
+                  sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
+                  (!first || kk > 0) ? 1u : 0u);
+        umma_commit(bar(Tr::B_V_EMPTY + vs));
+        umma_commit(bar(Tr::B_O_DONE));
+        ++vc;
+        return true;
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, p);
+        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
+        tc_fence_after();
+        const int n = un.t1 - un.t0;
+        for (int i = 0; i < n; ++i) {
+          const uint32_t ks = kc % KST;
+          if (!(ok = mbar_wait(bar(Tr::B_K_FULL + ks), (kc / KST) & 1u, w, kSiteKFull))) break;
+          tc_fence_after();
+          const uint32_t sb = g & 1u;
+          const uint32_t kbase = sK + ks * Tr::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
+            umma_ss(tmem + sb * BN, sw128_desc(sQ + ch * (Tr::BM * 128) + in, 16, 1024),
+                    sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(Tr::B_K_EMPTY + ks));
+          umma_commit(bar(Tr::B_S_FULL + sb));
+          if (i == n - 1) umma_commit(bar(Tr::B_Q_EMPTY));
+          ++kc;
+          if (i > 0 && !(ok = issue_pv(g - 1, i == 1))) break;
+          ++g;
+        }
+        if (!ok) break;
+        if (!(ok = issue_pv(g - 1, n == 1))) break;
+        ++uc;
+      }
+      // Every issued MMA must finish before tensor memory is released.
+      umma_commit(bar(Tr::B_DRAIN));
+      mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------ softmax and epilogue
+    const int row = threadIdx.x;  // 0..127, TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(u, p);
+      float m = -INFINITY, l = 0.f;
+      const int n = un.t1 - un.t0;
+      for (int i = 0; i < n; ++i, ++g) {
+        const uint32_t sb = g & 1u;
+        ok = mbar_wait(bar(Tr::B_S_FULL + sb), (g >> 1) & 1u, w, kSiteSFull);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        tc_fence_after();
+        const uint32_t scol = tl + sb * BN;
+        uint32_t r[BN / 32][32];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, r[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) reg_fence(r[c]);
+        // scores in base-2 units: t = s * scale * log2(e); key columns past N are -inf
+        float s[BN];
+        float mx = -INFINITY;
+        const int valid = p.N - (un.t0 + i) * BN;
+        if (valid >= BN) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            s[j] = __uint_as_float(r[j / 32][j % 32]) * p.sl2;
+            mx = fmaxf(mx, s[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            s[j] = (j < valid) ? __uint_as_float(r[j / 32][j % 32]) * p.sl2 : -INFINITY;
+            mx = fmaxf(mx, s[j]);
+          }
+        }
+        const float m_new = fmaxf(m, mx);
+        const float alpha = ex2(m - m_new);
+        float sum = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int j = 0; j < BN / 2; ++j) {
+          const float p0 = ex2(s[2 * j] - m_new);
+          const float p1 = ex2(s[2 * j + 1] - m_new);
+          sum += p0 + p1;
+          pk[j] = Elem<T>::pack(p0, p1);
+        }
+        l = l * alpha + sum;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_st16(scol + c * 16, &pk[c * 16]);
+        tmem_wait_st();
+        if (i > 0) {
+          // O holds P_{<j} V_{<j} scaled by the old max: rescale it once the
+          // previous P.V has landed and before this tile's P.V is issued.
+          ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteODone);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tl + Tr::TM_O + c * 32, o);
+              tmem_wait_ld();
+              reg_fence(o);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              tmem_st32(tl + Tr::TM_O + c * 32, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        m = m_new;
+        tc_fence_before();
+        mbar_arrive(bar(Tr::B_P_FULL + sb));
+      }
+      if (!ok) break;
+      // epilogue: O = O_acc / l, LSE = m + log2(l) (base 2) -> natural log
+      ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteEpi);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const int q_row = un.qt * Tr::BM + row;
+      const bool live = q_row < p.N;
+      const float inv_l = 1.f / l;
+      const float lse2 = m + lg2(l);
+      if (p.o_part == nullptr) {
+        T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tl + Tr::TM_O + c * 32, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          uint4 pkd[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pw[j] = Elem<T>::pack(__uint_as_float(o[2 * j]) * inv_l,
+                                  __uint_as_float(o[2 * j + 1]) * inv_l);
+          if (live) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
+          }
+        }
+        if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = lse2 * kLn2;
+      } else {
+        float* orow =
+            p.o_part + ((((size_t)un.sp * p.B + un.b) * p.N + q_row) * p.H + un.h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tl + Tr::TM_O + c * 32, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          if (live) {
+            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(
+                  __uint_as_float(o[4 * j]) * inv_l, __uint_as_float(o[4 * j + 1]) * inv_l,
+                  __uint_as_float(o[4 * j + 2]) * inv_l, __uint_as_float(o[4 * j + 3]) * inv_l);
+          }
+        }
+        if (live)
+          p.lse_part[(((size_t)un.sp * p.B + un.b) * p.H + un.h) * p.N + q_row] = lse2;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 6) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Tr::TMEM_COLS);
+  }
+}
+
+// Merge of split K/V partial results: one warp per (b, n, h) row.
+// o_part rows are normalised by their own sums; lse_part is base 2.
+template <class T, int D>
+__global__ void __launch_bounds__(256) fa_combine_kernel(const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part,
+                                                         T* __restrict__ o, float* __restrict__ lse,
+                                                         int B, int H, int N, int S) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)B * N * H) return;
+  const int h = (int)(row % H);
+  const int n = (int)((row / H) % N);
+  const int b = (int)(row / ((long long)H * N));
+  float mx = -INFINITY;
+  for (int s = 0; s < S; ++s)
+    mx = fmaxf(mx, lse_part[(((size_t)s * B + b) * H + h) * N + n]);
+  float tot = 0.f;
+  for (int s = 0; s < S; ++s) tot += ex2(lse_part[(((size_t)s * B + b) * H + h) * N + n] - mx);
+  const float L2 = mx + lg2(tot);
+  constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
+  float acc[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float wgt = ex2(lse_part[(((size_t)s * B + b) * H + h) * N + n] - L2);
+    const float* src = o_part + ((((size_t)s * B + b) * N + n) * H + h) * D + lane * PER;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) acc[j] += wgt * src[j];
+  }
+  T* dst = o + (((size_t)b * N + n) * H + h) * D + lane * PER;
+#pragma unroll
+  for (int j = 0; j < PER; j += 2) {
+    uint32_t v = Elem<T>::pack(acc[j], acc[j + 1]);
+    *reinterpret_cast<uint32_t*>(dst + j) = v;
+  }
+  if (lane == 0) lse[((size_t)b * H + h) * N + n] = L2 * kLn2;
+}
+
+template <class T, class Tr>
+static int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
+  const bool bf16 = Elem<T>::kFmt == 1;
+  CUtensorMap tmq, tmk, tmv;
+  int rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, Tr::D, Tr::BM)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, Tr::D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, Tr::D, Tr::BN)) != FA_OK) return rc;
+
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_qt = (N + Tr::BM - 1) / Tr::BM;
+  p.n_kvt = (N + Tr::BN - 1) / Tr::BN;
+  p.sl2 = scale * kLog2e;
+  p.limit_ns = 4000000000ull;
+  p.status = device_status_ptr();
+  const long long base_units = (long long)B * H * p.n_qt;
+  // Split the K/V range only when the units leave most SMs idle and each
+  // split keeps at least 8 K/V tiles.
+  int n_split = 1;
+  if (base_units * 2 <= dev.sm_count) {
+    n_split = (int)(dev.sm_count / base_units);
+    n_split = min(n_split, p.n_kvt / 8);
+    n_split = max(n_split, 1);
+  }
+  p.kvt_per_split = (p.n_kvt + n_split - 1) / n_split;
+  n_split = (p.n_kvt + p.kvt_per_split - 1) / p.kvt_per_split;  // no empty split
+  p.n_split = n_split;
+  p.n_units = (int)(base_units * n_split);
+
+  void* ws = nullptr;
+  if (n_split > 1) {
+    const size_t o_elems = (size_t)n_split * B * N * H * Tr::D;
+    const size_t l_elems = (size_t)n_split * B * H * N;
+    if (cudaMallocAsync(&ws, (o_elems + l_elems) * sizeof(float), stream) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NOMEM;
+    }
+    p.o_part = static_cast<float*>(ws);
+    p.lse_part = p.o_part + o_elems;
+  }
+
+  auto kern = fa_fwd_kernel<T, Tr>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    if (ws) cudaFreeAsync(ws, stream);
+    return FA_ERR_LAUNCH;
+  }
+  const int grid = p.n_units < dev.sm_count ? p.n_units : dev.sm_count;
+  kern<<<grid, 224, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, p);
+  rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  if (rc == FA_OK && n_split > 1) {
+    const long long rows = (long long)B * N * H;
+    fa_combine_kernel<T, Tr::D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        p.o_part, p.lse_part, static_cast<T*>(o), lse, B, H, N, n_split);
+    rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  }
+  if (ws) cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+template <class T>
+int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, cudaStream_t stream) {
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != FA_OK) return rc;
+  switch (d) {
+    case 64:
+      return run_fwd<T, FwdTraits<64, 128, 4, 4>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+    case 128:
+      return run_fwd<T, FwdTraits<128, 128, 3, 2>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+    case 256:
+      return run_fwd<T, FwdTraits<256, 64, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+    default:
+      return FA_ERR_HEADDIM;
+  }
+}
+
+template int fwd_launch<__nv_bfloat16>(const void*, const void*, const void*, void*, float*, int,
+                                       int, int, int, float, cudaStream_t);
+template int fwd_launch<__half>(const void*, const void*, const void*, void*, float*, int, int,
+                                int, int, float, cudaStream_t);
+
+}  // namespace fa

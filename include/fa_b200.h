@@ -1,0 +1,117 @@
+/*
+ * fa_b200.h -- C ABI of the exact-attention library for NVIDIA B200 (sm_100a).
+ *
+ * The operation (every page cites it; the definitions used here):
+ *   Standard attention, "YOLO11 ... FlashAttention-2" page, section 1.2, with
+ *   the 1/sqrt(d) score factor of that page's section 3.2 and of the LLM
+ *   explainer page (aitangshan.cn), section 1:
+ *       S = scale * Q K^T,  P = softmax_rows(S),  O = P V,
+ *       LSE_i = log(sum_j exp(S_ij))            (natural log, per query row)
+ *   computed FlashAttention-2 style (LLM explainer page, sections 4.1-4.3
+ *   and 5.2): outer loop over Q tiles, inner loop over K/V tiles, online
+ *   softmax with a running max and running sum; S and P never reach global
+ *   memory.  The backward pass (same page, section 6.2, recompute strategy)
+ *   rebuilds P from Q, K and the saved LSE and returns the textbook gradients
+ *   dV = P^T dO, dS = P o (dO V^T - rowsum(dO o O)), dQ = scale dS K,
+ *   dK = scale dS^T Q.  Non-causal, no dropout, no bias.
+ *
+ * Layout and types
+ *   q, k, v, o, dout, dq, dk, dv: contiguous [B, N, H, d] device arrays of
+ *   16-bit floats (bf16 for the unsuffixed entry points, fp16 for *_f16);
+ *   token stride H*d elements, head stride d.  lse: contiguous [B, H, N]
+ *   fp32 device array (natural log).  Every pointer must be 16-byte aligned.
+ *   d is 64, 128 or 256 (fa_bwd: 64 or 128); B, H, N >= 1; each tensor
+ *   holds fewer than 2^31 elements.  scale is any finite float (normally
+ *   1/sqrt(d)).  Arithmetic: 16-bit inputs, fp32 accumulation and softmax,
+ *   outputs rounded to nearest even.
+ *
+ * Ownership
+ *   The caller allocates and owns every buffer.  Inputs are read only.
+ *   fa_fwd writes o and lse; fa_bwd overwrites dq, dk, dv (it does not
+ *   accumulate into them).  Scratch memory (split-K/V partial results, the
+ *   fp32 dQ accumulator, the rowsum term) is allocated and released by the
+ *   library, stream-ordered (cudaMallocAsync / cudaFreeAsync) on `stream`.
+ *
+ * Errors and execution
+ *   Every call validates its arguments before any launch and returns FA_OK
+ *   or a negative FA_ERR_* code; on error no output is touched.  Work is
+ *   enqueued on `stream` and runs asynchronously: launch failures are
+ *   reported by the return value, faults inside a kernel surface at the
+ *   caller's next synchronisation.  Device-side waits are bounded: a wait
+ *   that gives up records a code readable with fa_get_device_status() and
+ *   the kernel returns instead of hanging.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *cudaStream_t;
+
+enum fa_status {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,        /* a required pointer is NULL                      */
+    FA_ERR_SHAPE = -2,       /* B, H or N < 1, or a tensor of 2^31+ elements    */
+    FA_ERR_HEADDIM = -3,     /* d not supported by this entry point             */
+    FA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned                */
+    FA_ERR_LAUNCH = -5,      /* the CUDA runtime rejected a launch or a call    */
+    FA_ERR_NOMEM = -6,       /* scratch allocation failed                       */
+    FA_ERR_DEVICE = -7,      /* current device is not compute capability 10.0   */
+    FA_ERR_SCALE = -8        /* scale is NaN or infinite                        */
+};
+
+/*
+ * Forward pass, bf16.  Writes o [B,N,H,d] and lse [B,H,N].
+ * The LLM explainer page, sections 4.1-4.3 and 5.2.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/* Forward pass, fp16; otherwise identical to fa_fwd. */
+int fa_fwd_f16(const void *q, const void *k, const void *v, void *o, float *lse,
+               int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/*
+ * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
+ * Inputs q, k, v, o (the forward output), dout (upstream gradient of o) and
+ * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64 or 128.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o,
+           const void *dout, const float *lse, void *dq, void *dk, void *dv,
+           int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/* Backward pass, fp16; otherwise identical to fa_bwd. */
+int fa_bwd_f16(const void *q, const void *k, const void *v, const void *o,
+               const void *dout, const float *lse, void *dq, void *dk, void *dv,
+               int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/* Static description of a status code.  Never NULL. */
+const char *fa_status_string(int status);
+
+/*
+ * Reads the device-side status word of the current device (0 = no kernel
+ * of this library gave up a bounded wait since the last clear).  Synchronises
+ * the device.  If clear is non-zero the word is reset to 0.  Returns FA_OK or
+ * FA_ERR_LAUNCH.
+ */
+int fa_get_device_status(unsigned long long *status_out, int clear);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on a
+ * barrier nothing will complete, with the given limit in microseconds
+ * (1..10,000,000).  The kernel gives up, records a status and returns; the
+ * call synchronises and writes the recorded status to *status_out (non-zero
+ * when the wait gave up as designed).  Leaves the device usable.
+ */
+int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long *status_out);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,56 @@
+"""Shared pieces of the GPU parity tests.
+
+Tolerances are the ones the benchmark spec fixes for 16-bit I/O with fp32
+accumulation on N(0,1) inputs, each against the fp64 oracle fed the same
+rounded inputs: O max-abs 2e-2 and mean-abs 2e-3, LSE max-abs 1e-3, and
+gradients max-abs 5e-2.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import attn_inputs
+
+O_MAX, O_MEAN, LSE_MAX, GRAD_MAX = 2e-2, 2e-3, 1e-3, 5e-2
+
+GUARD = 4096  # elements of sentinel after every output buffer
+
+
+def guarded(shape, dtype, device="cuda"):
+    """An output tensor followed in memory by GUARD sentinel elements."""
+    n = int(np.prod(shape))
+    flat = torch.empty(n + GUARD, dtype=dtype, device=device)
+    flat[n:].fill_(-12345.0 if dtype == torch.float32 else -1234.0)
+    flat[:n].fill_(float("nan"))
+    return flat[:n].view(shape), flat
+
+
+def guard_intact(flat: torch.Tensor) -> bool:
+    tail = flat[-GUARD:].float()
+    sentinel = -12345.0 if flat.dtype == torch.float32 else -1234.0
+    return bool(torch.all(tail == sentinel).item())
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return attn_inputs.to_f64(t)
+
+
+def err_stats(got: np.ndarray, ref: np.ndarray) -> dict:
+    diff = np.abs(got - ref)
+    rms_ref = float(np.sqrt(np.mean(ref * ref))) or 1.0
+    return {"max": float(diff.max()), "mean": float(diff.mean()),
+            "rms_rel": float(np.sqrt(np.mean(diff * diff)) / rms_ref)}
+
+
+def sample_rows(B, H, N, count, seed=7):
+    """(b, h, i) triples: the first and last rows of every head plus a seeded
+    spread, always including rows of the last (possibly ragged) Q tile."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = set()
+    for b in range(B):
+        for h in range(H):
+            rows.update({(b, h, 0), (b, h, N - 1), (b, h, max(0, (N // 128) * 128 - 1))})
+    while len(rows) < count + 3 * B * H:
+        rows.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))))
+    return sorted(rows)

@@ -1,0 +1,122 @@
+"""The C ABI loads and rejects bad arguments before touching the GPU.
+
+These run without a GPU: every call below fails validation (NULL or
+misaligned pointers, bad shapes, unsupported head size, non-finite scale),
+which happens on the host before any CUDA call.  The pointers passed are
+plain integers that are never dereferenced.
+"""
+import ctypes
+import math
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from exact_attention_144_b200 import build
+    build.build()
+    import exact_attention_144_b200 as fa
+    return fa
+
+
+def test_every_declared_symbol_is_exported(fa):
+    names = fa.declared_functions()
+    assert set(names) >= {"fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_status_string",
+                          "fa_get_device_status", "fa_selftest_bounded_wait", "fa_version"}
+    lib = fa.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the dynamic symbol table holds exactly those fa_* functions
+    out = subprocess.check_output(["nm", "-D", "--defined-only", fa.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {n for n in exported if n.startswith("fa_")} == set(names)
+
+
+def test_library_targets_sm100a_only(fa):
+    from exact_attention_144_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in build.NVCC_FLAGS
+
+
+def test_status_strings(fa):
+    for code in range(0, -9, -1):
+        s = fa.fa_status_string(code)
+        assert s and s != "unknown status"
+    assert fa.fa_status_string(-100) == "unknown status"
+    assert fa.fa_version() >= 100
+
+
+A = 0x10000          # a 16-byte aligned fake address (never dereferenced)
+MIS = 0x10008        # an 8-byte aligned one
+
+
+def _fwd(fa, ptrs, B=1, H=1, N=8, d=64, scale=0.125):
+    return fa.lib().fa_fwd(*ptrs, B, H, N, d, ctypes.c_float(scale), None)
+
+
+def _bwd(fa, ptrs, B=1, H=1, N=8, d=64, scale=0.125):
+    return fa.lib().fa_bwd(*ptrs, B, H, N, d, ctypes.c_float(scale), None)
+
+
+def test_forward_validation(fa):
+    ok = [A] * 5
+    for i in range(5):
+        p = list(ok)
+        p[i] = None
+        assert _fwd(fa, p) == fa.FA_ERR_NULL
+        p[i] = MIS
+        assert _fwd(fa, p) == fa.FA_ERR_ALIGN
+    assert _fwd(fa, ok, B=0) == fa.FA_ERR_SHAPE
+    assert _fwd(fa, ok, H=0) == fa.FA_ERR_SHAPE
+    assert _fwd(fa, ok, N=0) == fa.FA_ERR_SHAPE
+    assert _fwd(fa, ok, B=1 << 10, N=1 << 16, H=1, d=64) == fa.FA_ERR_SHAPE  # 2^32 elements
+    for d in (0, 32, 96, 100, 512):
+        assert _fwd(fa, ok, d=d) == fa.FA_ERR_HEADDIM
+    assert _fwd(fa, ok, scale=math.nan) == fa.FA_ERR_SCALE
+    assert _fwd(fa, ok, scale=math.inf) == fa.FA_ERR_SCALE
+    assert fa.lib().fa_fwd_f16(*ok, 1, 1, 8, 96, ctypes.c_float(1.0), None) == fa.FA_ERR_HEADDIM
+
+
+def test_backward_validation(fa):
+    ok = [A] * 9
+    for i in range(9):
+        p = list(ok)
+        p[i] = None
+        assert _bwd(fa, p) == fa.FA_ERR_NULL
+        p[i] = MIS
+        assert _bwd(fa, p) == fa.FA_ERR_ALIGN
+    assert _bwd(fa, ok, N=-3) == fa.FA_ERR_SHAPE
+    for d in (32, 96, 256):
+        assert _bwd(fa, ok, d=d) == fa.FA_ERR_HEADDIM
+    assert _bwd(fa, ok, scale=-math.inf) == fa.FA_ERR_SCALE
+
+
+def test_status_queries_reject_null(fa):
+    lib = fa.lib()
+    assert lib.fa_get_device_status(None, 0) == fa.FA_ERR_NULL
+    assert lib.fa_selftest_bounded_wait(1000, None) == fa.FA_ERR_NULL
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    # A copy of the package without the .so must refuse to import.
+    import shutil
+    pkg = tmp_path / "exact_attention_144_b200"
+    shutil.copytree(os.path.join(ROOT, "exact_attention_144_b200"), pkg,
+                    ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    (tmp_path / "include").mkdir()
+    code = "import exact_attention_144_b200 as fa; fa.lib()"
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
+    assert r.returncode != 0 and "no fallback" in (r.stderr + r.stdout)
+
+
+def test_product_package_does_not_touch_the_oracle():
+    pkg = os.path.join(ROOT, "exact_attention_144_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f

@@ -1,0 +1,91 @@
+"""Backward pass on the GPU against the fp64 oracle, element by element.
+
+The GPU backward consumes the GPU forward's O and LSE (as a training step
+does); the oracle differentiates the definition from Q, K, V and dO alone.
+Small shapes compare every gradient; the full-size training workload compares
+whole sampled heads.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_inputs
+import oracle
+from tests.gpu_helpers import GRAD_MAX, err_stats, guard_intact, guarded, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import exact_attention_144_b200 as fa
+    fa.fa_get_device_status(clear=True)
+    yield fa
+    assert fa.fa_get_device_status() == 0, "a kernel gave up a bounded wait"
+
+
+def run_bwd(fa, q, k, v, dout, scale):
+    o, lse = fa.forward(q, k, v, scale=scale)
+    shape = tuple(q.shape)
+    bufs = [guarded(shape, q.dtype) for _ in range(3)]
+    dq, dk, dv = (b[0] for b in bufs)
+    fa.backward(q, k, v, o, dout, lse, scale=scale, dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    for _, flat in bufs:
+        assert guard_intact(flat), "write past the end of a gradient"
+    return dq, dk, dv
+
+
+def check_grads(fa, B, N, H, d, dtype, seed, std=1.0):
+    q, k, v, dout = attn_inputs.draw(B, N, H, d, dtype, seed, 4, std=std, device="cuda")
+    scale = float(np.float32(1.0 / math.sqrt(d)))
+    dq, dk, dv = run_bwd(fa, q, k, v, dout, scale)
+    ref = oracle.attn_bwd(to64(q), to64(k), to64(v), to64(dout), scale)
+    stats = {}
+    for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        g = to64(got)
+        assert np.all(np.isfinite(g)), name
+        stats[name] = err_stats(g, r)
+        assert stats[name]["max"] <= GRAD_MAX, (name, stats[name])
+    return stats
+
+
+@pytest.mark.parametrize("N", [1, 2, 17, 64, 65, 127, 128, 129, 300, 640])
+def test_ragged_lengths_bf16(fa, N):
+    check_grads(fa, 2, N, 2, 64, "bf16", 500 + N)
+
+
+@pytest.mark.parametrize("N", [1, 100, 257])
+def test_fp16(fa, N):
+    check_grads(fa, 1, N, 3, 64, "fp16", 600 + N)
+
+
+def test_several_heads_and_batches(fa):
+    check_grads(fa, 3, 200, 5, 64, "bf16", 701)
+
+
+def test_training_workload_sampled_heads(fa):
+    w = attn_inputs.WORKLOADS["c5"]
+    q, k, v, dout = attn_inputs.draw_workload(w, device="cuda")
+    dq, dk, dv = run_bwd(fa, q, k, v, dout, w.scale)
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1), (2, 5)]:
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1), slice(None))
+        ref = oracle.attn_bwd(to64(q[sl]), to64(k[sl]), to64(v[sl]), to64(dout[sl]), w.scale)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            s = err_stats(to64(got[sl]), r)
+            assert s["max"] <= GRAD_MAX, (b, h, name, s)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+
+
+def test_deterministic_dk_dv(fa):
+    # dK and dV are owned by one block each (no atomics): bitwise repeatable.
+    q, k, v, dout = attn_inputs.draw(1, 700, 2, 64, "bf16", 702, 4, device="cuda")
+    a = run_bwd(fa, q, k, v, dout, 0.125)
+    b = run_bwd(fa, q, k, v, dout, 0.125)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2
