@@ -1,0 +1,337 @@
+#!/usr/bin/env python
+"""Benchmark of one exact-attention training step on B200: forward + backward.
+
+A step is one pass of the whole hot path over one batch of the training
+workload (B=4, N=4096, H=8, d=64, bf16, seeded N(0,1) inputs): fa_fwd
+(Q tiles x K/V tiles with online softmax, O and LSE out) then fa_bwd
+(rowsum preprocess, recompute of P from the LSE, dQ/dK/dV).  Throughput counts
+4 B H N^2 d for the forward and 2.5x that for the backward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5]
+  python bench.py --impl reference ...   (the fp64 CPU oracle, timed on a sample)
+
+Under torchrun every rank runs its own replica of the workload (weak scaling,
+no collective on the data path); the step time is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import attn_inputs  # noqa: E402
+
+METRIC = "fused attention fwd/bwd TFLOP/s on 1 B200 and % of bf16 tensor-core peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+# DRAM traffic of the dominant kernel per launch, from an ncu capture of the
+# same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
+# while the kernel sources hash to the recorded value.
+TRAFFIC = {}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("fa_common.cuh", "fa_fwd.cu", "fa_bwd.cu"):
+        with open(os.path.join(ROOT, "exact_attention_144_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period, self.stop_ev, self.thread = period_s, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report nothing rather than guess
+            self.nvml = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self.stop_ev.set()
+        if self.thread:
+            self.thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_oracle_sample(w: attn_inputs.Workload, rows: int, heads: int):
+    """Times the fp64 oracle on a bounded sample of the workload: the first
+    `rows` query rows of `heads` heads (forward rows and their backward
+    contributions).  Returns (TFLOP/s at the workload's FLOP-per-row rate,
+    seconds, threads, description)."""
+    import oracle  # the CPU baseline leg is one of the oracle's permitted users
+    q, k, v, do = attn_inputs.draw_workload(w, count=4)
+    f64 = attn_inputs.to_f64
+    hs = [(b, h) for b in range(w.B) for h in range(w.H)][:heads]
+    qs = np.stack([f64(q[b, :, h]) for b, h in hs], axis=1)[None]  # [1, N, S, d]
+    ks = np.stack([f64(k[b, :, h]) for b, h in hs], axis=1)[None]
+    vs = np.stack([f64(v[b, :, h]) for b, h in hs], axis=1)[None]
+    ds = np.stack([f64(do[b, :, h]) for b, h in hs], axis=1)[None]
+    sel = [(0, s, i) for s in range(len(hs)) for i in range(rows)]
+    t0 = time.perf_counter()
+    oracle.attn_fwd_rows(qs, ks, vs, w.scale, sel)
+    oracle.attn_bwd_rows(qs, ks, vs, ds, w.scale, 0, rows)
+    dt = time.perf_counter() - t0
+    flop = 14.0 * rows * w.N * w.d * len(hs)  # 4 (fwd) + 10 (bwd) per row, N keys, d
+    desc = (f"fp64 oracle fwd+bwd of query rows [0,{rows}) of {len(hs)} of {w.B * w.H} heads "
+            f"(N={w.N}, d={w.d}); {flop / 1e9:.2f} GFLOP of the step's "
+            f"{(w.fwd_flop + w.bwd_flop) / 1e9:.1f}")
+    return flop / dt / 1e12, dt, oracle.num_threads(), desc
+
+
+def run_reference(args, w, rank):
+    """The reference arm: the fp64 CPU oracle, timed as it stands on the host cores."""
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    heads = max(1, min(oracle.num_threads(), w.B * w.H))
+    # a few minutes in total: rows per step shrink as the step count grows
+    rows = int(max(8, min(512, 512 * 40 / max(1, args.steps + args.warmup))))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, rows, heads)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, dt, threads, desc = cpu_oracle_sample(w, rows, heads)
+        vals.append(v)
+        secs.append(dt)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N, "heads": w.H,
+                   "head_dim": w.d, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c5", choices=sorted(attn_inputs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = attn_inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+
+    import exact_attention_144_b200 as fa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # Each rank owns one replica of the workload (its own seeded batch).
+    q, k, v, do = attn_inputs.draw(w.B, w.N, w.H, w.d, w.dtype, w.seed + 7919 * rank, 4,
+                                   std=w.std, device=dev)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    fwd = fa.fa_fwd if w.dtype == "bf16" else fa.fa_fwd_f16
+    bwd = fa.fa_bwd if w.dtype == "bf16" else fa.fa_bwd_f16
+    train = w.backward
+
+    def step():
+        fwd(q, k, v, o=o, lse=lse, scale=w.scale)
+        if train:
+            bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, scale=w.scale)
+
+    flop_step = w.fwd_flop + (w.bwd_flop if train else 0.0)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------- device-timed steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [(mk(), mk(), mk(), mk(), mk(), mk()) for _ in range(args.steps)]
+    launches0 = fa.fa_kernel_launches()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for s0, s1, f0, f1, b0, b1 in ev:
+            flush.zero_()  # write 512 MiB between steps: no input stays in L2
+            fa.fa_set_kernel_events(f0, f1, b0 if train else None, b1 if train else None)
+            s0.record()
+            step()
+            s1.record()
+        torch.cuda.synchronize()
+    barrier()
+    launches = fa.fa_kernel_launches() - launches0
+    step_ms = [s0.elapsed_time(s1) for s0, s1, *_ in ev]
+    fwd_ms = [f0.elapsed_time(f1) for _, _, f0, f1, _, _ in ev]
+    bwd_ms = [b0.elapsed_time(b1) for *_, b0, b1 in ev] if train else []
+    ms = max_over_ranks(statistics.mean(step_ms))
+    value = world * flop_step / (ms * 1e-3) / 1e12
+    status = fa.fa_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"a kernel gave up a bounded wait (status {status:#x})")
+
+    # ------------------------------------- end to end, host buffers, same stream
+    dev_in = (q, k, v, do) if train else (q, k, v)
+    host_in = [t.cpu().pin_memory() for t in dev_in]
+    outs = (o, lse, dq, dk, dv) if train else (o, lse)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_ev = [(mk(), mk()) for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][0].record()
+        for hsrc, dst in zip(host_in, dev_in):
+            dst.copy_(hsrc, non_blocking=True)
+        step()
+        for dsrc, hdst in zip(outs, host_out):
+            hdst.copy_(dsrc, non_blocking=True)
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev))
+
+    # ----------------------------------------- roofline of the dominant kernel
+    pk, pk_src = peaks()
+    if train:
+        dom, dom_ms, dom_flop = "fa_bwd_kernel", statistics.mean(bwd_ms), w.bwd_flop
+    else:
+        dom, dom_ms, dom_flop = "fa_fwd_kernel", statistics.mean(fwd_ms), w.fwd_flop
+    achieved = dom_flop / (dom_ms * 1e-3) / 1e12
+    tr = TRAFFIC.get((dom, w.name))
+    traffic = tr["bytes"] if tr and tr["src"] == kernel_source_hash() else None
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                "kernel": dom, "kernel_ms": dom_ms,
+                "peak_source": f"bf16_tflops (burst) of {pk_src} MEASURED_PEAKS.json",
+                "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
+    kernels = {"fa_fwd_kernel": {"ms": statistics.mean(fwd_ms),
+                                 "tflops": w.fwd_flop / (statistics.mean(fwd_ms) * 1e-3) / 1e12}}
+    if train:
+        kernels["fa_bwd_kernel"] = {"ms": statistics.mean(bwd_ms), "tflops": achieved}
+    for kv in kernels.values():
+        kv["frac"] = kv["tflops"] / pk["bf16_tflops"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = None
+        try:
+            import oracle
+            oracle.build()
+            threads = oracle.num_threads()
+        except Exception as exc:  # the baseline is reported, never the target
+            cpu = {"error": str(exc)}
+        if threads:
+            val, dt, threads, desc = cpu_oracle_sample(w, 1024 if train else 256,
+                                                       max(1, min(threads, w.B * w.H)))
+            cpu = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                   "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
+                       "heads": w.H, "head_dim": w.d, "causal": False,
+                       "parallelism": f"replicas x{world} (batch per rank, no collective)",
+                       "l2": "512 MiB written between timed steps",
+                       "inputs": "seeded N(0,1) draws rounded to the 16-bit type"},
+            "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "roofline": roofline,
+            "kernels": kernels,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

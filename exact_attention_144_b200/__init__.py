@@ -51,6 +51,9 @@ def _load() -> ctypes.CDLL:
     lib.fa_selftest_bounded_wait.argtypes = [ctypes.c_uint, ctypes.POINTER(ctypes.c_ulonglong)]
     lib.fa_selftest_bounded_wait.restype = i
     lib.fa_version.restype = i
+    lib.fa_set_kernel_events.argtypes = [vp, vp, vp, vp]
+    lib.fa_set_kernel_events.restype = i
+    lib.fa_kernel_launches.restype = ctypes.c_ulonglong
     _lib = lib
     return lib
 
@@ -75,7 +78,7 @@ def declared_functions() -> list[str]:
     """Names of the functions include/fa_b200.h declares."""
     text = open(HEADER_PATH).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)
+    return re.findall(r"^[A-Za-z_][\w \t\*]*?\b(fa_\w+)\s*\(", text, flags=re.M)
 
 
 def fa_status_string(status: int) -> str:
@@ -210,3 +213,24 @@ def fa_selftest_bounded_wait(limit_us: int = 20000) -> int:
     if rc != FA_OK:
         raise FAError("fa_selftest_bounded_wait", rc)
     return int(out.value)
+
+
+def _event_handle(ev):
+    if ev is None:
+        return None
+    return ev.cuda_event if isinstance(ev, torch.cuda.Event) else int(ev)
+
+
+def fa_set_kernel_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop=None) -> None:
+    """Arm torch.cuda.Event pairs (enable_timing=True) around the next forward
+    and backward main kernels."""
+    for ev in (fwd_start, fwd_stop, bwd_start, bwd_stop):
+        if isinstance(ev, torch.cuda.Event) and ev.cuda_event == 0:
+            ev.record()  # materialise the underlying CUDA event
+    _load().fa_set_kernel_events(_event_handle(fwd_start), _event_handle(fwd_stop),
+                                 _event_handle(bwd_start), _event_handle(bwd_stop))
+
+
+def fa_kernel_launches() -> int:
+    """Kernel launches this library has issued since it was loaded."""
+    return int(_load().fa_kernel_launches())

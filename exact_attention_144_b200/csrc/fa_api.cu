@@ -1,6 +1,7 @@
 // fa_api.cu -- the C ABI: argument validation, device checks, TMA tensor-map
 // encoding and the device status word.  No torch types cross this boundary.
 #include <math.h>
+#include <atomic>
 #include <mutex>
 
 #include "fa_common.cuh"
@@ -9,6 +10,28 @@
 namespace fa {
 
 __device__ unsigned long long g_status = 0;
+
+static std::atomic<unsigned long long> g_launches{0};
+static std::mutex g_event_mu;
+static cudaEvent_t g_events[4] = {nullptr, nullptr, nullptr, nullptr};
+
+void note_launches(unsigned n) { g_launches.fetch_add(n); }
+
+void take_kernel_events(bool bwd, cudaEvent_t* start, cudaEvent_t* stop) {
+  std::lock_guard<std::mutex> lock(g_event_mu);
+  const int i = bwd ? 2 : 0;
+  *start = g_events[i];
+  *stop = g_events[i + 1];
+  g_events[i] = g_events[i + 1] = nullptr;
+}
+
+static void arm_kernel_events(cudaEvent_t fs, cudaEvent_t fe, cudaEvent_t bs, cudaEvent_t be) {
+  std::lock_guard<std::mutex> lock(g_event_mu);
+  g_events[0] = fs;
+  g_events[1] = fe;
+  g_events[2] = bs;
+  g_events[3] = be;
+}
 
 unsigned long long* device_status_ptr() {
   static std::mutex mu;
@@ -248,12 +271,21 @@ FA_EXPORT int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long
   if ((rc = fa_get_device_status(&prev, 1)) != FA_OK) return rc;
   fa::selftest_wait_kernel<<<1, 32>>>((unsigned long long)limit_us * 1000ull,
                                       fa::device_status_ptr());
+  fa::note_launches(1);
   if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
   }
   return fa_get_device_status(status_out, 1);
 }
+
+FA_EXPORT int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
+                                   cudaEvent_t bwd_start, cudaEvent_t bwd_stop) {
+  fa::arm_kernel_events(fwd_start, fwd_stop, bwd_start, bwd_stop);
+  return FA_OK;
+}
+
+FA_EXPORT unsigned long long fa_kernel_launches(void) { return fa::g_launches.load(); }
 
 FA_EXPORT int fa_version(void) { return 100; }
 

@@ -516,6 +516,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
       static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
       Npad);
   rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  note_launches(1);
   if (rc == FA_OK) {
     auto kern = fa_bwd_kernel<T, Tr>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -524,8 +525,13 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
       rc = FA_ERR_LAUNCH;
     } else {
       dim3 grid((N + Tr::BN - 1) / Tr::BN, H, B);
+      cudaEvent_t ev0, ev1;
+      take_kernel_events(true, &ev0, &ev1);
+      if (ev0) cudaEventRecord(ev0, stream);
       kern<<<grid, 320, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
       rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+      if (ev1) cudaEventRecord(ev1, stream);
+      note_launches(1);
     }
   }
   if (rc == FA_OK) {
@@ -533,6 +539,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
     fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
         p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
     rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+    note_launches(1);
   }
   cudaFreeAsync(ws, stream);
   return rc;

@@ -486,13 +486,19 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
     return FA_ERR_LAUNCH;
   }
   const int grid = p.n_units < dev.sm_count ? p.n_units : dev.sm_count;
+  cudaEvent_t ev0, ev1;
+  take_kernel_events(false, &ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, stream);
   kern<<<grid, 224, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, p);
   rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  if (ev1) cudaEventRecord(ev1, stream);
+  note_launches(1);
   if (rc == FA_OK && n_split > 1) {
     const long long rows = (long long)B * N * H;
     fa_combine_kernel<T, Tr::D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
         p.o_part, p.lse_part, static_cast<T*>(o), lse, B, H, N, n_split);
     rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+    note_launches(1);
   }
   if (ws) cudaFreeAsync(ws, stream);
   return rc;

@@ -20,6 +20,13 @@ struct DeviceInfo {
 // 10.0, or FA_ERR_LAUNCH when the runtime cannot be queried.
 int current_device(DeviceInfo* info);
 
+// Counts kernel launches (fa_kernel_launches).
+void note_launches(unsigned n);
+
+// Takes (and disarms) the event pair armed for the next forward (bwd=false)
+// or backward (bwd=true) main kernel; both are null when none is armed.
+void take_kernel_events(bool bwd, cudaEvent_t* start, cudaEvent_t* stop);
+
 // Device address of this library's status word on the current device.
 unsigned long long* device_status_ptr();
 

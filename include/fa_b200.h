@@ -20,7 +20,7 @@
  *   16-bit floats (bf16 for the unsuffixed entry points, fp16 for *_f16);
  *   token stride H*d elements, head stride d.  lse: contiguous [B, H, N]
  *   fp32 device array (natural log).  Every pointer must be 16-byte aligned.
- *   d is 64, 128 or 256 (fa_bwd: 64 or 128); B, H, N >= 1; each tensor
+ *   d is 64, 128 or 256 (fa_bwd: 64); B, H, N >= 1; each tensor
  *   holds fewer than 2^31 elements.  scale is any finite float (normally
  *   1/sqrt(d)).  Arithmetic: 16-bit inputs, fp32 accumulation and softmax,
  *   outputs rounded to nearest even.
@@ -49,6 +49,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st *cudaStream_t;
+typedef struct CUevent_st *cudaEvent_t;
 
 enum fa_status {
     FA_OK = 0,
@@ -76,7 +77,7 @@ int fa_fwd_f16(const void *q, const void *k, const void *v, void *o, float *lse,
 /*
  * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
  * Inputs q, k, v, o (the forward output), dout (upstream gradient of o) and
- * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64 or 128.
+ * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64.
  */
 int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -106,6 +107,20 @@ int fa_get_device_status(unsigned long long *status_out, int clear);
  * when the wait gave up as designed).  Leaves the device usable.
  */
 int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long *status_out);
+
+/*
+ * Instrumentation for benchmarks.  Arms CUDA events that the library records
+ * on the launching stream immediately before and immediately after the main
+ * kernel (fa_fwd_kernel / fa_bwd_kernel) of the next forward / backward call.
+ * Each armed pair is used once and then disarmed; pass NULL to leave a pair
+ * unarmed.  The events stay owned by the caller.  Process-wide, not tied to a
+ * thread.  Always returns FA_OK.
+ */
+int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
+                         cudaEvent_t bwd_start, cudaEvent_t bwd_stop);
+
+/* Number of kernel launches this library has issued since it was loaded. */
+unsigned long long fa_kernel_launches(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int fa_version(void);

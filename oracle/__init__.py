@@ -20,6 +20,7 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
   attn_fwd_online   as above; otherwise within a rounding bound.
   attn_bwd          central finite differences of L = sum(O * dO); the
                     row-sum identity of dS; closed form at N=1.
+  attn_bwd_rows     the row ranges of a split partition sum to attn_bwd.
 """
 from __future__ import annotations
 
@@ -84,6 +85,7 @@ class Oracle:
         lib.oracle_attn_fwd_rows.argtypes = [dp, dp, dp, ip, i, dp, dp, i, i, i, i, f]
         lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, f]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f]
+        lib.oracle_attn_bwd_rows.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f, i, i]
         lib.oracle_attn_dscores.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f]
         lib.oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
@@ -153,6 +155,20 @@ class Oracle:
                                  B, H, N, d, float(scale))
         return dq, dk, dv
 
+    def attn_bwd_rows(self, q, k, v, dout, scale, row_begin, row_end):
+        """Backward pass restricted to query rows [row_begin, row_end): dq rows
+        in the range are exact; dk, dv are those rows' contributions.  Rows of
+        dq outside the range are returned as zeros."""
+        q, k, v, dout = _c(q), _c(k), _c(v), _c(dout)
+        B, N, H, d = _shape(q)
+        if not 0 <= row_begin <= row_end <= N:
+            raise ValueError("bad row range")
+        dq, dk, dv = np.zeros_like(q), np.empty_like(q), np.empty_like(q)
+        self.lib.oracle_attn_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), B, H, N, d, float(scale), int(row_begin),
+                                      int(row_end))
+        return dq, dk, dv
+
     def attn_dscores(self, q, k, v, dout, scale):
         """dS = P * (dP - D) as [B, H, N, N] (small N only)."""
         q, k, v, dout = _c(q), _c(k), _c(v), _c(dout)
@@ -197,6 +213,10 @@ def attn_probs(q, k, scale):
 
 def attn_bwd(q, k, v, dout, scale):
     return default().attn_bwd(q, k, v, dout, scale)
+
+
+def attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end):
+    return default().attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end)
 
 
 def attn_dscores(q, k, v, dout, scale):

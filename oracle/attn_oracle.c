@@ -247,11 +247,15 @@ void oracle_attn_fwd_online(const double *q, const double *k, const double *v,
  *   dV_j += P_ij dO_i            dP_ij = dO_i . V_j
  *   D_i = sum_j P_ij dP_ij       dS_ij = P_ij (dP_ij - D_i)
  *   dQ_i = scale sum_j dS_ij K_j dK_j += scale dS_ij Q_i
- * dq, dk, dv are overwritten.  OpenMP splits independent (b, h) heads.
+ * Only query rows i in [row_begin, row_end) contribute: dq rows in that range
+ * are exact, dk and dv hold the sum over those rows (all rows when the range
+ * is [0, N)).  dq rows in the range, and all of dk and dv, are overwritten.
+ * OpenMP splits independent (b, h) heads.
  */
-void oracle_attn_bwd(const double *q, const double *k, const double *v,
-                     const double *dout, double *dq, double *dk, double *dv,
-                     int B, int H, int N, int d, double scale)
+void oracle_attn_bwd_rows(const double *q, const double *k, const double *v,
+                          const double *dout, double *dq, double *dk, double *dv,
+                          int B, int H, int N, int d, double scale,
+                          int row_begin, int row_end)
 {
     int heads = B * H;
 #pragma omp parallel
@@ -266,7 +270,7 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v,
                     dk[at(b, j, h, x, N, H, d)] = 0.0;
                     dv[at(b, j, h, x, N, H, d)] = 0.0;
                 }
-            for (int i = 0; i < N; ++i) {
+            for (int i = row_begin; i < row_end; ++i) {
                 double m, l;
                 row_probs(q, k, b, h, i, N, H, d, scale, p, &m, &l);
                 const double *doi = dout + at(b, i, h, 0, N, H, d);
@@ -297,6 +301,14 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v,
         free(p);
         free(dp);
     }
+}
+
+/* Backward pass over every query row (see oracle_attn_bwd_rows). */
+void oracle_attn_bwd(const double *q, const double *k, const double *v,
+                     const double *dout, double *dq, double *dk, double *dv,
+                     int B, int H, int N, int d, double scale)
+{
+    oracle_attn_bwd_rows(q, k, v, dout, dq, dk, dv, B, H, N, d, scale, 0, N);
 }
 
 /* dS for every (b, h): ds is [B, H, N, N] (tests of the row-sum identity). */

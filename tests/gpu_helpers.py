@@ -17,19 +17,21 @@ O_MAX, O_MEAN, LSE_MAX, GRAD_MAX = 2e-2, 2e-3, 1e-3, 5e-2
 GUARD = 4096  # elements of sentinel after every output buffer
 
 
+SENTINEL = -1232.0  # exactly representable in bf16, fp16 and fp32
+
+
 def guarded(shape, dtype, device="cuda"):
     """An output tensor followed in memory by GUARD sentinel elements."""
     n = int(np.prod(shape))
     flat = torch.empty(n + GUARD, dtype=dtype, device=device)
-    flat[n:].fill_(-12345.0 if dtype == torch.float32 else -1234.0)
+    flat[n:].fill_(SENTINEL)
     flat[:n].fill_(float("nan"))
     return flat[:n].view(shape), flat
 
 
 def guard_intact(flat: torch.Tensor) -> bool:
     tail = flat[-GUARD:].float()
-    sentinel = -12345.0 if flat.dtype == torch.float32 else -1234.0
-    return bool(torch.all(tail == sentinel).item())
+    return bool(torch.all(tail == SENTINEL).item())
 
 
 def to64(t: torch.Tensor) -> np.ndarray:

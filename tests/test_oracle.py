@@ -247,6 +247,18 @@ def check_backward_closed_forms(orc):
     assert np.max(np.abs(dk)) == 0.0
 
 
+def check_backward_row_ranges_partition_the_full_backward(orc):
+    # dQ rows come out exact from their own range; dK and dV are sums over
+    # rows, so the pieces of any partition of [0, N) add up to the whole.
+    B, N, H, d = 1, 30, 2, 4
+    q, k, v, dout = (rnd((B, N, H, d), s) for s in (55, 56, 57, 58))
+    full = orc.attn_bwd(q, k, v, dout, 0.6)
+    parts = [orc.attn_bwd_rows(q, k, v, dout, 0.6, a, b) for a, b in ((0, 7), (7, 8), (8, 30))]
+    assert np.array_equal(sum(p[0] for p in parts), full[0])
+    for g in (1, 2):
+        assert np.max(np.abs(sum(p[g] for p in parts) - full[g])) <= 1e-13
+
+
 # ----------------------------------------------------------- page fixtures
 
 def test_page_printed_shapes():
@@ -274,7 +286,7 @@ def test_page_printed_shapes():
 
 # Every check above, in order; tests/test_oracle_mutants.py reruns the same
 # list against oracle copies with planted mistakes.
-CHECKS = [check_probability_rows_sum_to_one, check_zero_queries_give_mean_of_values, check_single_key_gives_its_value, check_constant_values_give_that_value, check_hand_worked_one_dimensional_case, check_shift_of_every_key_leaves_output_and_shifts_lse, check_permutations, check_one_hot_dominance_at_large_scale, check_heads_and_batches_are_independent, check_rows_entry_point_matches_full_forward, check_definition_matches_two_pass_form, check_online_recurrence_bit_equal_with_one_kv_block, check_online_recurrence_bit_equal_when_max_is_in_first_block, check_online_recurrence_equals_definition_to_rounding, check_backward_matches_central_finite_differences, check_score_gradient_rows_sum_to_zero, check_backward_closed_forms]
+CHECKS = [check_probability_rows_sum_to_one, check_zero_queries_give_mean_of_values, check_single_key_gives_its_value, check_constant_values_give_that_value, check_hand_worked_one_dimensional_case, check_shift_of_every_key_leaves_output_and_shifts_lse, check_permutations, check_one_hot_dominance_at_large_scale, check_heads_and_batches_are_independent, check_rows_entry_point_matches_full_forward, check_definition_matches_two_pass_form, check_online_recurrence_bit_equal_with_one_kv_block, check_online_recurrence_bit_equal_when_max_is_in_first_block, check_online_recurrence_equals_definition_to_rounding, check_backward_matches_central_finite_differences, check_score_gradient_rows_sum_to_zero, check_backward_closed_forms, check_backward_row_ranges_partition_the_full_backward]
 
 def test_probability_rows_sum_to_one():
     check_probability_rows_sum_to_one(ORC)
@@ -346,3 +358,7 @@ def test_score_gradient_rows_sum_to_zero():
 
 def test_backward_closed_forms():
     check_backward_closed_forms(ORC)
+
+
+def test_backward_row_ranges_partition_the_full_backward():
+    check_backward_row_ranges_partition_the_full_backward(ORC)

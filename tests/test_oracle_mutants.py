@@ -28,14 +28,14 @@ MUTANTS = [
     ("LSE in base 2", "fwd_row", "*lse_out = m + log(l);", "*lse_out = m + log2(l);"),
     ("head and token strides swapped", "at",
      "(((size_t)b * N + n) * H + h)", "(((size_t)b * H + h) * N + n)"),
-    ("dQ loses the scale", "oracle_attn_bwd",
+    ("dQ loses the scale", "oracle_attn_bwd_rows",
      "dqi[x] += scale * ds * kj[x];", "dqi[x] += ds * kj[x];"),
-    ("D without the probabilities", "oracle_attn_bwd", "Di += p[j] * dp[j];", "Di += dp[j];"),
-    ("dS sign flipped", "oracle_attn_bwd",
+    ("D without the probabilities", "oracle_attn_bwd_rows", "Di += p[j] * dp[j];", "Di += dp[j];"),
+    ("dS sign flipped", "oracle_attn_bwd_rows",
      "double ds = p[j] * (dp[j] - Di);", "double ds = p[j] * (Di - dp[j]);"),
-    ("dV from dS instead of P", "oracle_attn_bwd",
+    ("dV from dS instead of P", "oracle_attn_bwd_rows",
      "dvj[x] += p[j] * doi[x];", "dvj[x] += ds * doi[x];"),
-    ("dK from K instead of Q", "oracle_attn_bwd",
+    ("dK from K instead of Q", "oracle_attn_bwd_rows",
      "dkj[x] += scale * ds * qi[x];", "dkj[x] += scale * ds * kj[x];"),
     ("online sum not rescaled", "oracle_attn_fwd_online", "l[r] = l[r] * alpha;", "l[r] = l[r];"),
     ("online output not rescaled", "oracle_attn_fwd_online",
