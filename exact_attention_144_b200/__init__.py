@@ -42,7 +42,8 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_f16.argtypes = lib.fa_fwd.argtypes
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, f, vp]
     lib.fa_bwd_f16.argtypes = lib.fa_bwd.argtypes
-    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16"):
+    lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes
+    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc"):
         getattr(lib, n).restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -61,6 +62,7 @@ def _load() -> ctypes.CDLL:
 FA_OK = 0
 FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_ALIGN = -1, -2, -3, -4
 FA_ERR_LAUNCH, FA_ERR_NOMEM, FA_ERR_DEVICE, FA_ERR_SCALE = -5, -6, -7, -8
+FA_ERR_SCRATCH = -9
 
 
 class FAError(RuntimeError):
@@ -177,6 +179,18 @@ def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, stream=
 def fa_bwd_f16(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, stream=None):
     """fp16 backward by recompute: returns (dq, dk, dv)."""
     return _bwd("fa_bwd_f16", torch.float16, q, k, v, o, dout, lse, dq, dk, dv, scale, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale=None, stream=None):
+    """bf16 backward that allocates no device memory: the library's fixed
+    64 MiB scratch buffer replaces the stream-ordered scratch of fa_bwd, for
+    callers that must not allocate.  dq, dk, dv must be given (this wrapper
+    allocates nothing either).  Calls that overlap on the GPU share the buffer
+    and race; order them (for example on one stream)."""
+    if dq is None or dk is None or dv is None:
+        raise ValueError("fa_bwd_noalloc needs caller-provided dq, dk, dv")
+    return _bwd("fa_bwd_noalloc", torch.bfloat16, q, k, v, o, dout, lse, dq, dk, dv, scale,
+                stream)
 
 
 _FWD = {torch.bfloat16: fa_fwd, torch.float16: fa_fwd_f16}

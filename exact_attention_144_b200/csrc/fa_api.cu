@@ -178,6 +178,14 @@ static int bwd_entry(const void* q, const void* k, const void* v, const void* o,
   return rc;
 }
 
+int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale) {
+  int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  return rc;
+}
+
 // ---------------------------------------------------- bounded-wait test
 __global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned long long* status) {
   __shared__ __align__(8) uint64_t bar;
@@ -239,6 +247,7 @@ FA_EXPORT const char* fa_status_string(int status) {
     case FA_ERR_NOMEM: return "scratch allocation failed";
     case FA_ERR_DEVICE: return "current device is not compute capability 10.0 (B200)";
     case FA_ERR_SCALE: return "scale is NaN or infinite";
+    case FA_ERR_SCRATCH: return "problem needs more scratch than the fixed no-alloc buffer (64 MiB) holds";
     default: return "unknown status";
   }
 }

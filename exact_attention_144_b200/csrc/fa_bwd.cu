@@ -25,6 +25,8 @@
 // Tensor memory (d = 64): S^T [0,128) (P^T over its first 64 columns),
 // dP^T [128,256) (dS^T over its first 64), dV [256,320), dK [320,384),
 // dQ [384,448).
+#include <mutex>
+
 #include "fa_common.cuh"
 #include "fa_host.h"
 
@@ -567,4 +569,111 @@ template int bwd_launch<__half>(const void*, const void*, const void*, const voi
                                 const float*, void*, void*, void*, int, int, int, int, float,
                                 cudaStream_t);
 
+// ------------------------------------------------------------------------
+// Fixed-scratch backward (fa_bwd_noalloc).  Same kernels as run_bwd, but the
+// scratch (dQ accumulator, base-2 LSE, D) lives in a file-scope device array
+// instead of a stream-ordered allocation, for callers that cannot allocate.
+// Host code cannot pass g_fixed_scratch itself to a kernel (in host code the
+// name denotes a host-side stand-in); its device address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+static constexpr size_t kFixedScratchBytes = (size_t)64 << 20;
+static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+
+static int fixed_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  if (dev < 0 || dev >= 64) return FA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fixed_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    cached[dev] = ptr;
+  }
+  *out = cached[dev];
+  return FA_OK;
+}
+
+template <class T, class Tr>
+static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                 int B, int H, int N, float scale, cudaStream_t stream) {
+  constexpr int D = Tr::D;
+  const int n_qt = (N + Tr::BM - 1) / Tr::BM;
+  const int Npad = n_qt * Tr::BM;
+  const size_t rows = (size_t)B * H * Npad;
+  const size_t ws_bytes = rows * D * sizeof(float) + 2 * rows * sizeof(float);
+  if (ws_bytes > kFixedScratchBytes) return FA_ERR_SCRATCH;
+  void* ws = nullptr;
+  int rc = fixed_scratch_address(&ws);
+  if (rc != FA_OK) return rc;
+
+  const bool bf16 = Elem<T>::kFmt == 1;
+  CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
+  BwdParams p{};
+  p.dq_acc = static_cast<float*>(ws);
+  float* lse2 = p.dq_acc + rows * D;
+  float* dvec = lse2 + rows;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.Npad = Npad;
+  p.n_qt = n_qt;
+  p.sl2 = scale * kLog2e;
+  p.scale = scale;
+  p.limit_ns = 4000000000ull;
+  p.status = device_status_ptr();
+  if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::BM)) != FA_OK) return rc;
+
+  // The pre-pass rewrites every scratch word this call reads (it zeroes the
+  // accumulator), so the previous call's contents never leak into this one.
+  fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
+      Npad);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  auto kern = fa_bwd_kernel<T, Tr>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 320, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv,
+                                                                               tmdo, tmacc, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  const long long total = (long long)B * N * H * D;
+  fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
+      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  note_launches(3);
+  return FA_OK;
+}
+
 }  // namespace fa
+
+extern "C" __attribute__((visibility("default"))) int fa_bwd_noalloc(
+    const void* q, const void* k, const void* v, const void* o, const void* dout,
+    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+    cudaStream_t stream) {
+  int rc = fa::check_bwd_args(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  fa::DeviceInfo dev;
+  if ((rc = fa::current_device(&dev)) != FA_OK) return rc;
+  if (d != 64) return FA_ERR_HEADDIM;
+  return fa::run_bwd_fixed_scratch<__nv_bfloat16, fa::BwdTraits64>(q, k, v, o, dout, lse, dq, dk,
+                                                                   dv, B, H, N, scale, stream);
+}

@@ -41,6 +41,11 @@ int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, 
 int make_tmap_f32_rows(CUtensorMap* map, const void* base, size_t rows, int cols, int box_cols,
                        int box_rows);
 
+// The backward entry points' argument checks (FA_OK or an FA_ERR_* code).
+int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale);
+
 // Launchers (argument validation is done by the callers in fa_api.cu).
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,

@@ -60,7 +60,9 @@ enum fa_status {
     FA_ERR_LAUNCH = -5,      /* the CUDA runtime rejected a launch or a call    */
     FA_ERR_NOMEM = -6,       /* scratch allocation failed                       */
     FA_ERR_DEVICE = -7,      /* current device is not compute capability 10.0   */
-    FA_ERR_SCALE = -8        /* scale is NaN or infinite                        */
+    FA_ERR_SCALE = -8,       /* scale is NaN or infinite                        */
+    FA_ERR_SCRATCH = -9      /* fa_bwd_noalloc: the problem needs more scratch than
+                                its fixed buffer holds                           */
 };
 
 /*
@@ -87,6 +89,35 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
 int fa_bwd_f16(const void *q, const void *k, const void *v, const void *o,
                const void *dout, const float *lse, void *dq, void *dk, void *dv,
                int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/*
+ * Backward pass, bf16, for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for hosts
+ * such as plugin runtimes with their own static memory plan, code that runs
+ * where allocation is forbidden or unsafe, and callers that must not touch
+ * the device allocator at all.  fa_bwd needs scratch memory (an fp32 dQ
+ * accumulator plus two fp32 vectors per query row) and takes it from
+ * cudaMallocAsync; this variant computes the same result with the same
+ * kernels but takes the scratch from one fixed buffer compiled into the
+ * library, so it calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layout, ownership and results are those of fa_bwd (d = 64).
+ * Limit: the scratch needed is B * H * ceil(N/128) * 128 * (4*d + 8) bytes
+ * and must not exceed 64 MiB (67,108,864 bytes); larger problems are
+ * rejected with FA_ERR_SCRATCH before any launch.  Every GPU that loads the
+ * library holds the 64 MiB buffer until the process exits.
+ *
+ * The first call on a device looks up the buffer's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one buffer and it keeps the previous call's
+ * contents (the part that must start at zero is cleared by every call):
+ * calls whose work overlaps on the GPU -- on different streams, or from
+ * different host threads without ordering -- race on it and give wrong
+ * results.  Order such calls, for example on a single stream.
+ */
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                   const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                   int B, int H, int N, int d, float scale, cudaStream_t stream);
 
 /* Static description of a status code.  Never NULL. */
 const char *fa_status_string(int status);

@@ -28,7 +28,7 @@ def test_every_declared_symbol_is_exported(fa):
     names = fa.declared_functions()
     assert set(names) >= {"fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_status_string",
                           "fa_get_device_status", "fa_selftest_bounded_wait", "fa_version",
-                          "fa_set_kernel_events", "fa_kernel_launches"}
+                          "fa_set_kernel_events", "fa_kernel_launches", "fa_bwd_noalloc"}
     lib = fa.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -44,7 +44,7 @@ def test_library_targets_sm100a_only(fa):
 
 
 def test_status_strings(fa):
-    for code in range(0, -9, -1):
+    for code in range(0, -10, -1):
         s = fa.fa_status_string(code)
         assert s and s != "unknown status"
     assert fa.fa_status_string(-100) == "unknown status"
