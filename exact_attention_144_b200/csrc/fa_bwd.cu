@@ -17,11 +17,16 @@
 //   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to 16 bits
 //
 // fa_bwd_kernel layout (320 threads, one block per SM):
-//   warps 0-3  recompute P^T and dS^T; thread t owns key row t (TMEM lane t);
-//              epilogue for dK and dV
-//   warps 4-7  dQ drain: TMEM -> shared memory -> bulk reduce-add to global
+//   warps 0-7  compute: warp w owns TMEM lane quadrant w % 4 and half w / 4 of
+//              the 128 query columns; P and dS are elementwise in (key, query),
+//              so the halves need no exchange.  They recompute P^T and dS^T,
+//              drain the dQ tiles (TMEM -> swizzled shared memory -> TMA
+//              reduce-add into the fp32 accumulator) and store dK, dV
 //   warp  8    TMA producer
 //   warp  9    TMEM allocator and tcgen05.mma issuer
+// MMA issue order per Q tile i: dV += P^T dO_i as soon as P^T is written,
+// then S^T for tile i+1 (so the next P^T can start while dS^T is computed),
+// then dK += dS^T Q_i, dQ_i = dS K and dP^T for tile i+1.
 // Tensor memory (d = 64): S^T [0,128) (P^T over its first 64 columns),
 // dP^T [128,256) (dS^T over its first 64), dV [256,320), dK [320,384),
 // dQ [384,448).
@@ -52,7 +57,8 @@ struct BwdTraits64 {
   static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
                        B_S_FULL = B_Q_EMPTY + QST, B_DP_FULL = B_S_FULL + 1,
-                       B_DS_READY = B_DP_FULL + 1, B_DSBUF_FREE = B_DS_READY + 1,
+                       B_P_READY = B_DP_FULL + 1, B_DS_READY = B_P_READY + 1,
+                       B_DSBUF_FREE = B_DS_READY + 1,
                        B_DQ_FULL = B_DSBUF_FREE + 2, B_DQ_FREE = B_DQ_FULL + 1,
                        B_KV_DONE = B_DQ_FREE + 1, B_DRAIN = B_KV_DONE + 1,
                        NUM_BARS = B_DRAIN + 1;
@@ -77,7 +83,7 @@ struct BwdParams {
 };
 
 enum { kBSiteQEmpty = 0x21, kBSiteKV, kBSiteQFull, kBSiteDsReady, kBSiteDqFree, kBSiteSFull,
-       kBSiteDpFull, kBSiteQFullSm, kBSiteDsBuf, kBSiteDqFull, kBSiteKvDone };
+       kBSiteDpFull, kBSiteQFullSm, kBSiteDsBuf, kBSiteDqFull, kBSiteKvDone, kBSitePReady };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -114,11 +120,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 }
 
 template <class T, class Tr>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __maxnreg__(200)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
                   const __grid_constant__ CUtensorMap tmacc, const BwdParams p) {
   constexpr int D = Tr::D, BN = Tr::BN, BM = Tr::BM, QST = Tr::QST;
+  constexpr int HC = BM / 2;  // query columns per compute warp (one half)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -147,11 +154,12 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(bar(Tr::B_S_FULL), 1);
     mbar_init(bar(Tr::B_DP_FULL), 1);
-    mbar_init(bar(Tr::B_DS_READY), 128);
+    mbar_init(bar(Tr::B_P_READY), 256);
+    mbar_init(bar(Tr::B_DS_READY), 256);
     mbar_init(bar(Tr::B_DSBUF_FREE), 1);
     mbar_init(bar(Tr::B_DSBUF_FREE + 1), 1);
     mbar_init(bar(Tr::B_DQ_FULL), 1);
-    mbar_init(bar(Tr::B_DQ_FREE), 128);
+    mbar_init(bar(Tr::B_DQ_FREE), 256);
     mbar_init(bar(Tr::B_KV_DONE), 1);
     mbar_init(bar(Tr::B_DRAIN), 1);
     fence_mbar_init();
@@ -195,47 +203,69 @@ __global__ void __launch_bounds__(320, 1)
     // ----------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t fmt = Elem<T>::kFmt;
-      constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);       // K-major x K-major
-      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);        // TS, B MN-major
+      constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);            // K-major x K-major
+      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);             // TS, B MN-major
       constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, D, true) | (1u << 15);  // A, B MN-major
-      bool ok = mbar_wait(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
-      tc_fence_after();
-      for (int i = 0; i < n_qt && ok; ++i) {
-        const int qs = i % QST;
-        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL + qs), (i / QST) & 1, w, kBSiteQFull))) break;
-        tc_fence_after();
-        const uint32_t q_s = sQ + qs * Tr::QT_BYTES, do_s = sDO + qs * Tr::QT_BYTES;
-        // S^T = K Q^T and dP^T = V dO^T (both K-major over d)
+      auto q_s = [&](int i) { return sQ + (i % QST) * Tr::QT_BYTES; };
+      auto do_s = [&](int i) { return sDO + (i % QST) * Tr::QT_BYTES; };
+      // S^T = K Q_i^T into TM_S; dP^T = V dO_i^T into TM_DP (K-major over d)
+      auto issue_s = [&](int i) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
           umma_ss(tmem + Tr::TM_S, sw128_desc(sK + ch * (BN * 128) + in, 16, 1024),
-                  sw128_desc(q_s + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
+                  sw128_desc(q_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(Tr::B_S_FULL));
+      };
+      auto issue_dp = [&](int i) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
           umma_ss(tmem + Tr::TM_DP, sw128_desc(sV + ch * (BN * 128) + in, 16, 1024),
-                  sw128_desc(do_s + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
+                  sw128_desc(do_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP,
+                  kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(Tr::B_DP_FULL));
-        // P^T and dS^T written by the softmax warps
-        if (!(ok = mbar_wait(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+      };
+      bool ok = mbar_wait(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
+      if (ok && n_qt > 0) {
+        ok = mbar_wait(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          umma_commit(bar(Tr::B_S_FULL));
+          issue_dp(0);
+          umma_commit(bar(Tr::B_DP_FULL));
+        }
+      }
+      for (int i = 0; i < n_qt && ok; ++i) {
+        // dV += P^T dO_i  (A = P^T from TMEM, B = dO_i: queries x d, MN-major)
+        if (!(ok = mbar_wait(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
         tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q   (A from TMEM, B MN-major: queries x d)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           umma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_S + kk * 8,
-                  sw128_desc(do_s + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
+                  sw128_desc(do_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
+        // the next S^T overwrites TM_S after dV has read P^T (same issue order)
+        const bool more = i + 1 < n_qt;
+        if (more) {
+          if (!(ok = mbar_wait(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                               kBSiteQFull)))
+            break;
+          tc_fence_after();
+          issue_s(i + 1);
+          umma_commit(bar(Tr::B_S_FULL));
+        }
+        // dK += dS^T Q_i  (A = dS^T from TMEM, B = Q_i MN-major)
+        if (!(ok = mbar_wait(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           umma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DP + kk * 8,
-                  sw128_desc(q_s + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
+                  sw128_desc(q_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(Tr::B_Q_EMPTY + qs));
-        // dQ_i = dS K: A = dS (queries contiguous), B = K (d contiguous)
+        umma_commit(bar(Tr::B_Q_EMPTY + i % QST));
+        // dQ_i = dS K  (A = dS from shared memory, queries contiguous; B = K, d contiguous)
         if (i > 0 && !(ok = mbar_wait(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree))) break;
         tc_fence_after();
         const uint32_t ds_s = sDS + (i & 1) * Tr::DS_BYTES;
@@ -245,157 +275,180 @@ __global__ void __launch_bounds__(320, 1)
                   sw128_desc(sK + kk * 16 * 128, BN * 128, 1024), kIdescDQ, kk > 0 ? 1u : 0u);
         umma_commit(bar(Tr::B_DQ_FULL));
         umma_commit(bar(Tr::B_DSBUF_FREE + (i & 1)));
+        // the next dP^T overwrites TM_DP after dK has read dS^T
+        if (more) {
+          issue_dp(i + 1);
+          umma_commit(bar(Tr::B_DP_FULL));
+        }
       }
       umma_commit(bar(Tr::B_KV_DONE));
       umma_commit(bar(Tr::B_DRAIN));
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------- P^T, dS^T and dK/dV epilogue
-    const int r = threadIdx.x;  // key row within the tile
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+  } else {
+    // ----------------------------- compute warps 0-7: P^T, dS^T, dQ drain
+    // Warp w owns TMEM lane quadrant w % 4 (key rows of S^T/dP^T, query rows
+    // of dQ) and half hf = w / 4 of the columns.
+    const int quad = warp & 3, hf = warp >> 2;
+    const int r = quad * 32 + lane;  // key row (S^T, dP^T) and query row (dQ)
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const bool key_valid = kt * BN + r < p.N;
+    const bool issuer = lane == 0 && quad == 0;  // one thread per half issues its reduce
+    const float c = p.sl2;
     bool ok = true;
+
+    // dQ tile i: TMEM -> swizzled fp32 staging box hf -> TMA reduce-add
+    // Every thread of a half reaches both named barriers even when a wait
+    // gave up, so no warp is left waiting on them.
+    auto drain_dq = [&](int i) -> bool {
+      bool good = mbar_wait(bar(Tr::B_DQ_FULL), i & 1, w, kBSiteDqFull);
+      good = __all_sync(0xffffffffu, good);
+      uint32_t v[32];
+      if (good) {
+        tc_fence_after();
+        tmem_ld32(tl + Tr::TM_DQ + hf * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        tc_fence_before();
+        mbar_arrive(bar(Tr::B_DQ_FREE));
+      }
+      if (issuer) bulk_wait_read_all();  // the previous reduce has read the staging box
+      named_bar_sync(1 + hf, 128);
+      if (good) {
+        uint8_t* box = gSTG + hf * (BM * 128);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) =
+              make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                          __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(1 + hf, 128);
+      if (issuer && good && *abort_flag == 0) {
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM);
+        tma_reduce_add_2d(&tmacc, sSTG + hf * (BM * 128), hf * 32, row);
+        bulk_commit();
+      }
+      return good;
+    };
+
     for (int i = 0; i < n_qt; ++i) {
       const int qs = i % QST;
+      // ---- P^T = 2^(c S^T - LSE2) for this warp's 64 query columns
       ok = mbar_wait(bar(Tr::B_S_FULL), i & 1, w, kBSiteSFull);
       ok = ok && mbar_wait(bar(Tr::B_Q_FULL + qs), (i / QST) & 1, w, kBSiteQFullSm);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const float* lrow = sL + qs * BM;
-      const float* drow = sDD + qs * BM;
-      float pr[BM];
+      const float4* l4 = reinterpret_cast<const float4*>(sL + qs * BM + hf * HC);
+      const float4* d4 = reinterpret_cast<const float4*>(sDD + qs * BM + hf * HC);
+      float pr[HC];
       {
-        uint32_t sr[BM / 32][32];
-#pragma unroll
-        for (int c = 0; c < BM / 32; ++c) tmem_ld32(tl + Tr::TM_S + c * 32, sr[c]);
+        uint32_t sr[2][32];
+        tmem_ld32(tl + Tr::TM_S + hf * HC, sr[0]);
+        tmem_ld32(tl + Tr::TM_S + hf * HC + 32, sr[1]);
         tmem_wait_ld();
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
 #pragma unroll
-        for (int c = 0; c < BM / 32; ++c) reg_fence(sr[c]);
+        for (int j4 = 0; j4 < HC / 4; ++j4) {
+          const float4 L = l4[j4];
+          const float Ls[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
-        for (int j = 0; j < BM; ++j)
-          pr[j] = key_valid ? ex2(__uint_as_float(sr[j / 32][j % 32]) * p.sl2 - lrow[j]) : 0.f;
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e;
+            pr[j] = ex2(fmaf(__uint_as_float(sr[j / 32][j % 32]), c, -Ls[e]));
+          }
+        }
+        if (!key_valid) {
+#pragma unroll
+          for (int j = 0; j < HC; ++j) pr[j] = 0.f;
+        }
+        uint32_t pk[HC / 2];
+#pragma unroll
+        for (int j = 0; j < HC / 2; ++j) pk[j] = Elem<T>::pack(pr[2 * j], pr[2 * j + 1]);
+        tmem_st16(tl + Tr::TM_S + hf * (HC / 2), &pk[0]);
+        tmem_st16(tl + Tr::TM_S + hf * (HC / 2) + 16, &pk[16]);
+        tmem_wait_st();
       }
-      {
-        uint32_t pk[BM / 2];
-#pragma unroll
-        for (int j = 0; j < BM / 2; ++j) pk[j] = Elem<T>::pack(pr[2 * j], pr[2 * j + 1]);
-#pragma unroll
-        for (int c = 0; c < BM / 32; ++c) tmem_st16(tl + Tr::TM_S + c * 16, &pk[c * 16]);
-      }
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_P_READY));
+      // ---- dS^T = P^T o (dP^T - D) for the same columns
       ok = mbar_wait(bar(Tr::B_DP_FULL), i & 1, w, kBSiteDpFull);
-      if (i >= 2) ok = ok && mbar_wait(bar(Tr::B_DSBUF_FREE + (i & 1)), ((i >> 1) - 1) & 1, w,
-                                       kBSiteDsBuf);
+      if (i >= 2)
+        ok = ok && mbar_wait(bar(Tr::B_DSBUF_FREE + (i & 1)), ((i >> 1) - 1) & 1, w, kBSiteDsBuf);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      uint32_t dk16[BM / 2];
-#pragma unroll
-      for (int c = 0; c < BM / 32; ++c) {
-        uint32_t dr[32];
-        tmem_ld32(tl + Tr::TM_DP + c * 32, dr);
+      uint32_t dk16[HC / 2];
+      {
+        uint32_t dr[2][32];
+        tmem_ld32(tl + Tr::TM_DP + hf * HC, dr[0]);
+        tmem_ld32(tl + Tr::TM_DP + hf * HC + 32, dr[1]);
         tmem_wait_ld();
-        reg_fence(dr);
+        reg_fence(dr[0]);
+        reg_fence(dr[1]);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int q0 = c * 32 + 2 * j;
-          const float ds0 = pr[q0] * (__uint_as_float(dr[2 * j]) - drow[q0]);
-          const float ds1 = pr[q0 + 1] * (__uint_as_float(dr[2 * j + 1]) - drow[q0 + 1]);
-          dk16[c * 16 + j] = Elem<T>::pack(ds0, ds1);
+        for (int j4 = 0; j4 < HC / 4; ++j4) {
+          const float4 Dv = d4[j4];
+          const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+          float ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e;
+            ds[e] = pr[j] * (__uint_as_float(dr[j / 32][j % 32]) - Ds[e]);
+          }
+          dk16[2 * j4] = Elem<T>::pack(ds[0], ds[1]);
+          dk16[2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
         }
       }
+      tmem_st16(tl + Tr::TM_DP + hf * (HC / 2), &dk16[0]);
+      tmem_st16(tl + Tr::TM_DP + hf * (HC / 2) + 16, &dk16[16]);
+      // dS row r, query chunk hf, into the 128-byte-swizzled shared tile
+      uint8_t* ds_g = gDS + (i & 1) * Tr::DS_BYTES + hf * (BN * 128) + r * 128;
 #pragma unroll
-      for (int c = 0; c < BM / 32; ++c) tmem_st16(tl + Tr::TM_DP + c * 16, &dk16[c * 16]);
-      // dS row r into shared memory for the dQ MMA: 128-byte-swizzled,
-      // queries contiguous (two 64-query chunks of 128 key rows each).
-      uint8_t* ds_g = gDS + (i & 1) * Tr::DS_BYTES;
-#pragma unroll
-      for (int u = 0; u < BM / 8; ++u) {
-        const int chunk = u >> 3, unit = u & 7;
-        uint4 val = make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2], dk16[4 * u + 3]);
-        *reinterpret_cast<uint4*>(ds_g + chunk * (BN * 128) + r * 128 + ((unit ^ (r & 7)) * 16)) =
-            val;
-      }
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(ds_g + ((u ^ (r & 7)) * 16)) =
+            make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2], dk16[4 * u + 3]);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(Tr::B_DS_READY));
+      // ---- dQ of the previous tile
+      if (i > 0 && !(ok = drain_dq(i - 1))) break;
     }
-    // epilogue: dV and scale * dK for this block's key rows
+    if (ok && n_qt > 0) ok = drain_dq(n_qt - 1);
+    if (issuer) bulk_wait_all();
+    // ---- epilogue: dV and scale * dK, this warp's key rows and 32 of the d columns
     if (ok) ok = mbar_wait(bar(Tr::B_KV_DONE), 0, w, kBSiteKvDone);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      T* dvrow = reinterpret_cast<T*>(p.dv) + (((size_t)b * p.N + key) * p.H + h) * D;
-      T* dkrow = reinterpret_cast<T*>(p.dk) + (((size_t)b * p.N + key) * p.H + h) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32], k2[32];
-        tmem_ld32(tl + Tr::TM_DV + c * 32, a);
-        tmem_ld32(tl + Tr::TM_DK + c * 32, k2);
-        tmem_wait_ld();
-        reg_fence(a);
-        reg_fence(k2);
-        uint4 va[4], vk[4];
-        uint32_t* pa = reinterpret_cast<uint32_t*>(va);
-        uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
-          pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
-                                 __uint_as_float(k2[2 * j + 1]) * p.scale);
-        }
-        if (key_valid) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            reinterpret_cast<uint4*>(dvrow + c * 32)[j] = va[j];
-            reinterpret_cast<uint4*>(dkrow + c * 32)[j] = vk[j];
-          }
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------- dQ drain (warps 4-7)
-    const int t = threadIdx.x - 128;  // query row within the tile
-    const uint32_t tl = tmem + ((uint32_t)((warp - 4) * 32) << 16);
-    bool ok = true;
-    for (int i = 0; i < n_qt; ++i) {
-      ok = mbar_wait(bar(Tr::B_DQ_FULL), i & 1, w, kBSiteDqFull);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      tc_fence_after();
-      uint32_t v[D / 32][32];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tl + Tr::TM_DQ + c * 32, v[c]);
+      const size_t off = (((size_t)b * p.N + key) * p.H + h) * D + hf * 32;
+      uint32_t a[32], k2[32];
+      tmem_ld32(tl + Tr::TM_DV + hf * 32, a);
+      tmem_ld32(tl + Tr::TM_DK + hf * 32, k2);
       tmem_wait_ld();
+      reg_fence(a);
+      reg_fence(k2);
+      uint4 va[4], vk[4];
+      uint32_t* pa = reinterpret_cast<uint32_t*>(va);
+      uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) reg_fence(v[c]);
-      tc_fence_before();
-      mbar_arrive(bar(Tr::B_DQ_FREE));
-      named_bar_sync(1, 128);  // the previous reduce has read the staging tile
-      // Row t of the fp32 staging tile, as two 32-column boxes of 128-byte rows
-      // with the 128-byte swizzle (16-byte unit w of row t at w ^ (t & 7)).
-#pragma unroll
-      for (int u = 0; u < D / 4; ++u) {
-        const int box = u >> 3, wu = u & 7;
-        float4 val = make_float4(__uint_as_float(v[(4 * u) / 32][(4 * u) % 32]),
-                                 __uint_as_float(v[(4 * u + 1) / 32][(4 * u + 1) % 32]),
-                                 __uint_as_float(v[(4 * u + 2) / 32][(4 * u + 2) % 32]),
-                                 __uint_as_float(v[(4 * u + 3) / 32][(4 * u + 3) % 32]));
-        *reinterpret_cast<float4*>(gSTG + box * (BM * 128) + t * 128 + ((wu ^ (t & 7)) * 16)) =
-            val;
+      for (int j = 0; j < 16; ++j) {
+        pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
+        pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
+                               __uint_as_float(k2[2 * j + 1]) * p.scale);
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (t == 0) {
-        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM);
+      if (key_valid) {
+        uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dv) + off);
+        uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dk) + off);
 #pragma unroll
-        for (int box = 0; box < D / 32; ++box)
-          tma_reduce_add_2d(&tmacc, sSTG + box * (BM * 128), box * 32, row);
-        bulk_commit();
-        bulk_wait_read_all();
+        for (int j = 0; j < 4; ++j) {
+          dvp[j] = va[j];
+          dkp[j] = vk[j];
+        }
       }
     }
-    if (t == 0) bulk_wait_all();
   }
 
   tc_fence_before();

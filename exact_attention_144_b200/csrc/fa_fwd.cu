@@ -1,57 +1,41 @@
 // fa_fwd.cu -- forward pass of exact attention on sm_100a.
 //
 // O = softmax(scale Q K^T) V and the per-row log-sum-exp, FlashAttention-2
-// style (LLM explainer page, sections 4.1-4.3 and 5.2): each work unit is one
-// 128-row Q tile of one (batch, head), whose inner loop walks the K/V tiles;
-// the online softmax keeps a running max m and running sum l per row and
-// rescales the O accumulator when m grows (YOLO11 page, section 2.2).  S and P
-// live only in tensor memory; O is written once per Q tile.
+// style (LLM explainer page, sections 4.1-4.3 and 5.2): each work unit holds
+// Q tiles of 128 rows of one (batch, head) and walks the K/V tiles; the online
+// softmax keeps a running max m and running sum l per row and rescales the O
+// accumulator when m grows (YOLO11 page, section 2.2).  S and P live only in
+// tensor memory; O is written once per Q tile.
 //
-// Block layout (224 threads, one block per SM, persistent over work units):
-//   warps 0-3  softmax + epilogue; thread t owns Q row t (TMEM lane t)
-//   warp  4    TMA producer for Q and K tiles
-//   warp  5    TMA producer for V tiles
-//   warp  6    TMEM allocator and the single-thread tcgen05.mma issuer
-// Tensor memory (512 columns): S0 at [0, BN), S1 at [BN, 2BN), O at [2BN, 2BN+d).
-// S is double buffered so QK^T of tile j+1 overlaps the softmax of tile j; P
-// (16-bit) is written back over the first BN/2 columns of its S buffer and
-// consumed from there by the P.V MMA (A operand in tensor memory).
+// Two persistent kernels, both one block per SM looping over work units:
 //
-// When the (batch, head, Q tile) units cannot fill the SMs, the K/V range is
-// split and the partial results (fp32, normalised, with base-2 LSE) are merged
-// by fa_combine_kernel: O = sum_s exp(LSE_s - LSE) O_s, LSE = log sum_s exp(LSE_s).
+// fa_fwd_pp_kernel (d = 64, 128; 320 threads) -- two 128-row Q tiles per unit
+//   warps 0-3  softmax + epilogue of Q tile 0 (thread t owns row t, TMEM lane t)
+//   warps 4-7  softmax + epilogue of Q tile 1
+//   warp  8    TMA producer: the Q pair once per unit, then K_j, V_j in turn
+//   warp  9    TMEM allocator and the single-thread tcgen05.mma issuer
+//   TMEM: S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d,256+2d).
+//   MMA order per K/V tile j: P0.V_j, Q0 K_{j+1}^T, P1.V_j, Q1 K_{j+1}^T, so
+//   the tensor cores work on one tile while the other tile's exponentials run,
+//   and both Q tiles share every K/V tile loaded into shared memory.
+//
+// fa_fwd_kernel (any d, used for d = 256 and short sequences; 224 threads) --
+//   one 128-row Q tile per unit, S double buffered in TMEM
+//   warps 0-3 softmax + epilogue, warp 4 Q/K producer, warp 5 V producer,
+//   warp 6 TMEM allocator + MMA issuer.
+//
+// In both, P (16-bit) is written back over the first BN/2 columns of its S
+// buffer and consumed from there by the P.V MMA (A operand in TMEM).  O is
+// rescaled only when a row's max grows by more than 2^8: until then P and l
+// stay relative to the older max (P <= 2^8), which changes rounding only.
+//
+// When the units cannot fill the SMs, the K/V range is split and the partial
+// results (fp32, normalised, base-2 LSE) are merged by fa_combine_kernel:
+// O = sum_s 2^(LSE_s - LSE) O_s,  LSE = log2 sum_s 2^LSE_s.
 #include "fa_common.cuh"
 #include "fa_host.h"
 
 namespace fa {
-
-template <int D_, int BN_, int KST_, int VST_>
-struct FwdTraits {
-  static constexpr int D = D_;
-  static constexpr int BM = 128;
-  static constexpr int BN = BN_;
-  static constexpr int KST = KST_;
-  static constexpr int VST = VST_;
-  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  // barrier indices
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
-                       B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
-                       B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
-                       B_O_DONE = B_P_FULL + 2, B_DRAIN = B_O_DONE + 1, NUM_BARS = B_DRAIN + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t TM_O = 2 * BN;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(2 * BN + D <= 512, "tensor memory budget");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(D % 64 == 0 && BN % 32 == 0, "tile shape");
-};
 
 struct FwdParams {
   void* o;          // [B, N, H, D] 16-bit, direct mode
@@ -59,7 +43,8 @@ struct FwdParams {
   float* o_part;    // [S, B, N, H, D] fp32, split mode (null in direct mode)
   float* lse_part;  // [S, B, H, N] base-2 log, split mode
   int B, H, N;
-  int n_qt, n_kvt, n_split, kvt_per_split, n_units;
+  int n_qt;         // Q units per (b, h): 128-row tiles (fa_fwd_kernel) or 256-row pairs
+  int n_kvt, n_split, kvt_per_split, n_units;
   float sl2;        // scale * log2(e)
   unsigned long long limit_ns;
   unsigned long long* status;
@@ -85,6 +70,438 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
 // Timeout sites reported in the status word.
 enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull,
        kSiteSFull, kSiteODone, kSiteEpi };
+
+// Growth of the running max (base 2) tolerated before O is rescaled.
+constexpr float kRescaleThreshold = 8.0f;
+
+// ---------------------------------------------------------------------------
+// One softmax step for the row a thread owns.  r holds the row's BN raw scores
+// (fp32 bits, unscaled); columns >= valid are keys past N.  c = scale*log2(e).
+// Updates the reference max m (base 2) and the running sum l, returns the
+// factor alpha that O must be multiplied by (1 when the reference max is
+// kept), and packs P = 2^(s*c - m) as 16-bit pairs into pk.
+template <class T, int BN>
+__device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], int valid, float c,
+                                              float& m, float& l, uint32_t (&pk)[BN / 2]) {
+  auto S = [&](int j) { return __uint_as_float(r[j / 32][j % 32]); };
+  // row max of s*c (the min of s when c < 0), 8 independent chains
+  float part[8];
+  const bool full = valid >= BN;
+  const bool neg = c < 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) part[q] = neg ? INFINITY : -INFINITY;
+  if (full) {
+    if (!neg) {
+#pragma unroll
+      for (int j = 0; j < BN; ++j) part[j & 7] = fmaxf(part[j & 7], S(j));
+    } else {
+#pragma unroll
+      for (int j = 0; j < BN; ++j) part[j & 7] = fminf(part[j & 7], S(j));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < BN; ++j)
+      if (j < valid) part[j & 7] = neg ? fminf(part[j & 7], S(j)) : fmaxf(part[j & 7], S(j));
+  }
+  float mx;
+  if (!neg)
+    mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
+               fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
+  else
+    mx = fminf(fminf(fminf(part[0], part[1]), fminf(part[2], part[3])),
+               fminf(fminf(part[4], part[5]), fminf(part[6], part[7])));
+  const float mc = mx * c;  // max of s*c over the valid columns
+  float alpha = 1.f;
+  if (mc > m + kRescaleThreshold) {
+    alpha = ex2(m - mc);  // m = -inf on the first tile: alpha = 0
+    m = mc;
+  }
+  const float neg_m = -m;
+  float sum[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) sum[q] = 0.f;
+  if (full) {
+#pragma unroll
+    for (int j = 0; j < BN / 2; ++j) {
+      const float p0 = ex2(fmaf(S(2 * j), c, neg_m));
+      const float p1 = ex2(fmaf(S(2 * j + 1), c, neg_m));
+      sum[j & 7] += p0 + p1;
+      pk[j] = Elem<T>::pack(p0, p1);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < BN / 2; ++j) {
+      const float p0 = (2 * j < valid) ? ex2(fmaf(S(2 * j), c, neg_m)) : 0.f;
+      const float p1 = (2 * j + 1 < valid) ? ex2(fmaf(S(2 * j + 1), c, neg_m)) : 0.f;
+      sum[j & 7] += p0 + p1;
+      pk[j] = Elem<T>::pack(p0, p1);
+    }
+  }
+  const float rs = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+  l = l * alpha + rs;
+  return alpha;
+}
+
+// Multiplies this thread's O row (D fp32 columns at taddr) by alpha.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(taddr + c * 32, o);
+    tmem_wait_ld();
+    reg_fence(o);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+    tmem_st32(taddr + c * 32, o);
+  }
+  tmem_wait_st();
+}
+
+// Epilogue for one row: O = O_acc / l (16-bit, or fp32 partial in split mode)
+// and the LSE (natural log, or base 2 in split mode).  Collective over the warp.
+template <class T, int D>
+__device__ __forceinline__ void store_row(const FwdParams& p, const Unit& un, uint32_t taddr,
+                                          int q_row, float m, float l) {
+  const bool live = q_row < p.N;
+  const float inv_l = 1.f / l;
+  const float lse2 = m + lg2(l);
+  if (p.o_part == nullptr) {
+    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(taddr + c * 32, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      uint4 pkd[4];
+      uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        pw[j] = Elem<T>::pack(__uint_as_float(o[2 * j]) * inv_l,
+                              __uint_as_float(o[2 * j + 1]) * inv_l);
+      if (live) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
+      }
+    }
+    if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = lse2 * kLn2;
+  } else {
+    float* orow = p.o_part + ((((size_t)un.sp * p.B + un.b) * p.N + q_row) * p.H + un.h) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(taddr + c * 32, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      if (live) {
+        float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[j] = make_float4(__uint_as_float(o[4 * j]) * inv_l,
+                               __uint_as_float(o[4 * j + 1]) * inv_l,
+                               __uint_as_float(o[4 * j + 2]) * inv_l,
+                               __uint_as_float(o[4 * j + 3]) * inv_l);
+      }
+    }
+    if (live) p.lse_part[(((size_t)un.sp * p.B + un.b) * p.H + un.h) * p.N + q_row] = lse2;
+  }
+}
+
+// ===========================================================================
+// fa_fwd_pp_kernel: two Q tiles per unit
+// ===========================================================================
+template <int D_, int KST_, int VST_>
+struct FwdPPTraits {
+  static constexpr int D = D_;
+  static constexpr int BM = 128;  // rows per Q tile; a unit holds two
+  static constexpr int BN = 128;
+  static constexpr int KST = KST_;
+  static constexpr int VST = VST_;
+  static constexpr int KCH = D / 64;
+  static constexpr int QT_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
+                       B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
+                       B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
+                       B_O_DONE = B_P_FULL + 2, B_DRAIN = B_O_DONE + 2, NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TM_O = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(2 * BN + 2 * D <= 512, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <class T, class Tr>
+__global__ void __maxnreg__(200)
+    fa_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmq,
+                     const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+  constexpr int D = Tr::D, BN = Tr::BN, BM = Tr::BM, KST = Tr::KST, VST = Tr::VST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + Tr::OFF_Q, sK = base + Tr::OFF_K, sV = base + Tr::OFF_V;
+  const uint32_t bars = base + Tr::OFF_BAR;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + Tr::OFF_MISC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + Tr::OFF_MISC + 4);
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtl w{abort_flag, p.limit_ns, p.status};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(Tr::B_Q_FULL), 1);
+    mbar_init(bar(Tr::B_Q_EMPTY), 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(bar(Tr::B_K_FULL + s), 1);
+      mbar_init(bar(Tr::B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(bar(Tr::B_V_FULL + s), 1);
+      mbar_init(bar(Tr::B_V_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Tr::B_S_FULL + s), 1);
+      mbar_init(bar(Tr::B_P_FULL + s), 128);
+      mbar_init(bar(Tr::B_O_DONE + s), 1);
+    }
+    mbar_init(bar(Tr::B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), Tr::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------- producer
+    if (lane == 0) {
+      uint32_t kc = 0, vc = 0, qc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, p);
+        if (qc > 0 && !(ok = mbar_wait(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
+        mbar_expect_tx(bar(Tr::B_Q_FULL), 2 * Tr::QT_BYTES);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int c = 0; c < Tr::KCH; ++c)
+            tma_load_4d(sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64,
+                        un.h, (2 * un.qt + t) * BM, un.b);
+        ++qc;
+        for (int t = un.t0; t < un.t1; ++t) {
+          const uint32_t ks = kc % KST;
+          if (kc >= (uint32_t)KST &&
+              !(ok = mbar_wait(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
+            break;
+          mbar_expect_tx(bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Tr::KCH; ++c)
+            tma_load_4d(sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
+                        c * 64, un.h, t * BN, un.b);
+          ++kc;
+          const uint32_t vs = vc % VST;
+          if (vc >= (uint32_t)VST &&
+              !(ok = mbar_wait(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
+            break;
+          mbar_expect_tx(bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
+#pragma unroll
+          for (int c = 0; c < Tr::KCH; ++c)
+            tma_load_4d(sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
+                        c * 64, un.h, t * BN, un.b);
+          ++vc;
+        }
+      }
+      // Every issued load must land before the block exits.
+      if (qc > 0) mbar_drain(bar(Tr::B_Q_FULL), (qc - 1) & 1u, p.limit_ns);
+      for (uint32_t s = 0; s < (uint32_t)KST; ++s)
+        if (kc > s) mbar_drain(bar(Tr::B_K_FULL + s), ((kc - 1 - s) / KST) & 1u, p.limit_ns);
+      for (uint32_t s = 0; s < (uint32_t)VST; ++s)
+        if (vc > s) mbar_drain(bar(Tr::B_V_FULL + s), ((vc - 1 - s) / VST) & 1u, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ----------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = f16_idesc(Elem<T>::kFmt, 128, BN, false);
+      constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
+      uint32_t kc = 0, vc = 0, g = 0, uc = 0;
+      bool ok = true;
+      // S_t = Q_t K^T for the K stage of counter kc (t = 0, 1)
+      auto issue_qk = [&](int t) {
+        const uint32_t kbase = sK + (kc % KST) * Tr::KV_BYTES;
+        const uint32_t qbase = sQ + t * Tr::QT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
+          umma_ss(tmem + t * BN, sw128_desc(qbase + ch * (BM * 128) + in, 16, 1024),
+                  sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
+                  kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t (+)= P_t V for the V stage of counter vc
+      auto issue_pv = [&](int t, bool first) {
+        const uint32_t vbase = sV + (vc % VST) * Tr::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
+                  sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
+                  (!first || kk > 0) ? 1u : 0u);
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, p);
+        const int n = un.t1 - un.t0;
+        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
+        if (!(ok = mbar_wait(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))) break;
+        tc_fence_after();
+        issue_qk(0);
+        umma_commit(bar(Tr::B_S_FULL + 0));
+        issue_qk(1);
+        umma_commit(bar(Tr::B_S_FULL + 1));
+        umma_commit(bar(Tr::B_K_EMPTY + kc % KST));
+        if (n == 1) umma_commit(bar(Tr::B_Q_EMPTY));
+        ++kc;
+        for (int j = 0; j < n; ++j, ++g) {
+          // tile 0: P0 V_j, then S0 for the next K tile
+          if (!(ok = mbar_wait(bar(Tr::B_P_FULL + 0), g & 1u, w, kSitePFull))) break;
+          if (!(ok = mbar_wait(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
+            break;
+          tc_fence_after();
+          issue_pv(0, j == 0);
+          umma_commit(bar(Tr::B_O_DONE + 0));
+          const bool more = j + 1 < n;
+          if (more) {
+            if (!(ok = mbar_wait(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull)))
+              break;
+            tc_fence_after();
+            issue_qk(0);
+            umma_commit(bar(Tr::B_S_FULL + 0));
+          }
+          // tile 1: P1 V_j, then S1 for the next K tile
+          if (!(ok = mbar_wait(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
+          tc_fence_after();
+          issue_pv(1, j == 0);
+          umma_commit(bar(Tr::B_O_DONE + 1));
+          umma_commit(bar(Tr::B_V_EMPTY + vc % VST));
+          ++vc;
+          if (more) {
+            issue_qk(1);
+            umma_commit(bar(Tr::B_S_FULL + 1));
+            umma_commit(bar(Tr::B_K_EMPTY + kc % KST));
+            if (j + 2 == n) umma_commit(bar(Tr::B_Q_EMPTY));
+            ++kc;
+          }
+        }
+        if (!ok) break;
+        ++uc;
+      }
+      // Every issued MMA must finish before tensor memory is released.
+      umma_commit(bar(Tr::B_DRAIN));
+      mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------- softmax and epilogue, Q tile wg
+    const int wg = warp >> 2;           // which Q tile
+    const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_col = tl + wg * BN;
+    const uint32_t o_col = tl + Tr::TM_O + wg * D;
+    const float c = p.sl2;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(u, p);
+      float m = -INFINITY, l = 0.f;
+      const int n = un.t1 - un.t0;
+      for (int j = 0; j < n; ++j, ++g) {
+        ok = mbar_wait(bar(Tr::B_S_FULL + wg), g & 1u, w, kSiteSFull);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        tc_fence_after();
+        uint32_t r[BN / 32][32];
+#pragma unroll
+        for (int q = 0; q < BN / 32; ++q) tmem_ld32(s_col + q * 32, r[q]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
+        uint32_t pk[BN / 2];
+        const float alpha = softmax_step<T, BN>(r, p.N - (un.t0 + j) * BN, c, m, l, pk);
+#pragma unroll
+        for (int q = 0; q < BN / 32; ++q) tmem_st16(s_col + q * 16, &pk[q * 16]);
+        tmem_wait_st();
+        if (j > 0) {
+          // the previous P.V into this O must have landed before O is touched
+          // or the next P.V is issued (every phase is waited once, in order)
+          ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteODone);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Tr::B_P_FULL + wg));
+      }
+      if (!ok) break;
+      ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteEpi);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      store_row<T, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Tr::TMEM_COLS);
+  }
+}
+
+// ===========================================================================
+// fa_fwd_kernel: one Q tile per unit, S double buffered
+// ===========================================================================
+template <int D_, int BN_, int KST_, int VST_>
+struct FwdTraits {
+  static constexpr int D = D_;
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int KST = KST_;
+  static constexpr int VST = VST_;
+  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
+                       B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
+                       B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
+                       B_O_DONE = B_P_FULL + 2, B_DRAIN = B_O_DONE + 1, NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t TM_O = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(2 * BN + D <= 512, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(D % 64 == 0 && BN % 32 == 0, "tile shape");
+};
 
 template <class T, class Tr>
 __global__ void __launch_bounds__(224, 1)
@@ -257,6 +674,7 @@ __global__ void __launch_bounds__(224, 1)
     // ------------------------------------------ softmax and epilogue
     const int row = threadIdx.x;  // 0..127, TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const float c = p.sl2;
     uint32_t g = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -271,117 +689,31 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t scol = tl + sb * BN;
         uint32_t r[BN / 32][32];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, r[c]);
+        for (int q = 0; q < BN / 32; ++q) tmem_ld32(scol + q * 32, r[q]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) reg_fence(r[c]);
-        // scores in base-2 units: t = s * scale * log2(e); key columns past N are -inf
-        float s[BN];
-        float mx = -INFINITY;
-        const int valid = p.N - (un.t0 + i) * BN;
-        if (valid >= BN) {
-#pragma unroll
-          for (int j = 0; j < BN; ++j) {
-            s[j] = __uint_as_float(r[j / 32][j % 32]) * p.sl2;
-            mx = fmaxf(mx, s[j]);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < BN; ++j) {
-            s[j] = (j < valid) ? __uint_as_float(r[j / 32][j % 32]) * p.sl2 : -INFINITY;
-            mx = fmaxf(mx, s[j]);
-          }
-        }
-        const float m_new = fmaxf(m, mx);
-        const float alpha = ex2(m - m_new);
-        float sum = 0.f;
+        for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
         uint32_t pk[BN / 2];
+        const float alpha = softmax_step<T, BN>(r, p.N - (un.t0 + i) * BN, c, m, l, pk);
 #pragma unroll
-        for (int j = 0; j < BN / 2; ++j) {
-          const float p0 = ex2(s[2 * j] - m_new);
-          const float p1 = ex2(s[2 * j + 1] - m_new);
-          sum += p0 + p1;
-          pk[j] = Elem<T>::pack(p0, p1);
-        }
-        l = l * alpha + sum;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_st16(scol + c * 16, &pk[c * 16]);
+        for (int q = 0; q < BN / 32; ++q) tmem_st16(scol + q * 16, &pk[q * 16]);
         tmem_wait_st();
         if (i > 0) {
-          // O holds P_{<j} V_{<j} scaled by the old max: rescale it once the
-          // previous P.V has landed and before this tile's P.V is issued.
+          // O holds P_{<j} V_{<j}: once the previous P.V has landed, rescale it
+          // (if a row's reference max moved) before this tile's P.V is issued.
           ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteODone);
           if (!(ok = __all_sync(0xffffffffu, ok))) break;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha < 1.f)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tl + Tr::TM_O + c * 32, o);
-              tmem_wait_ld();
-              reg_fence(o);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st32(tl + Tr::TM_O + c * 32, o);
-            }
-            tmem_wait_st();
-          }
+          if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(tl + Tr::TM_O, alpha);
         }
-        m = m_new;
         tc_fence_before();
         mbar_arrive(bar(Tr::B_P_FULL + sb));
       }
       if (!ok) break;
-      // epilogue: O = O_acc / l, LSE = m + log2(l) (base 2) -> natural log
       ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const int q_row = un.qt * Tr::BM + row;
-      const bool live = q_row < p.N;
-      const float inv_l = 1.f / l;
-      const float lse2 = m + lg2(l);
-      if (p.o_part == nullptr) {
-        T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tl + Tr::TM_O + c * 32, o);
-          tmem_wait_ld();
-          reg_fence(o);
-          uint4 pkd[4];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pw[j] = Elem<T>::pack(__uint_as_float(o[2 * j]) * inv_l,
-                                  __uint_as_float(o[2 * j + 1]) * inv_l);
-          if (live) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
-          }
-        }
-        if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = lse2 * kLn2;
-      } else {
-        float* orow =
-            p.o_part + ((((size_t)un.sp * p.B + un.b) * p.N + q_row) * p.H + un.h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tl + Tr::TM_O + c * 32, o);
-          tmem_wait_ld();
-          reg_fence(o);
-          if (live) {
-            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(
-                  __uint_as_float(o[4 * j]) * inv_l, __uint_as_float(o[4 * j + 1]) * inv_l,
-                  __uint_as_float(o[4 * j + 2]) * inv_l, __uint_as_float(o[4 * j + 3]) * inv_l);
-          }
-        }
-        if (live)
-          p.lse_part[(((size_t)un.sp * p.B + un.b) * p.H + un.h) * p.N + q_row] = lse2;
-      }
+      store_row<T, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l);
     }
   }
 
@@ -431,15 +763,29 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float* __restrict
   if (lane == 0) lse[((size_t)b * H + h) * N + n] = L2 * kLn2;
 }
 
-template <class T, class Tr>
-static int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                   int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
+// ---------------------------------------------------------------- launchers
+// Number of K/V splits: only when the units leave most SMs idle, and only so
+// far that every split keeps at least 8 K/V tiles.
+static int choose_splits(long long base_units, int n_kvt, int sm_count) {
+  int n_split = 1;
+  if (base_units * 2 <= sm_count) {
+    n_split = (int)(sm_count / base_units);
+    n_split = min(n_split, n_kvt / 8);
+    n_split = max(n_split, 1);
+  }
+  return n_split;
+}
+
+template <class T, int D, int BM_UNIT, int BN, int THREADS, int SMEM, class Kernel>
+static int launch_fwd(Kernel kern, const void* q, const void* k, const void* v, void* o,
+                      float* lse, int B, int H, int N, float scale, cudaStream_t stream,
+                      const DeviceInfo& dev) {
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, Tr::D, Tr::BM)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, Tr::D, Tr::BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, Tr::D, Tr::BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, 128)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, BN)) != FA_OK) return rc;
 
   FwdParams p{};
   p.o = o;
@@ -447,20 +793,13 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   p.B = B;
   p.H = H;
   p.N = N;
-  p.n_qt = (N + Tr::BM - 1) / Tr::BM;
-  p.n_kvt = (N + Tr::BN - 1) / Tr::BN;
+  p.n_qt = (N + BM_UNIT - 1) / BM_UNIT;
+  p.n_kvt = (N + BN - 1) / BN;
   p.sl2 = scale * kLog2e;
   p.limit_ns = 4000000000ull;
   p.status = device_status_ptr();
   const long long base_units = (long long)B * H * p.n_qt;
-  // Split the K/V range only when the units leave most SMs idle and each
-  // split keeps at least 8 K/V tiles.
-  int n_split = 1;
-  if (base_units * 2 <= dev.sm_count) {
-    n_split = (int)(dev.sm_count / base_units);
-    n_split = min(n_split, p.n_kvt / 8);
-    n_split = max(n_split, 1);
-  }
+  int n_split = choose_splits(base_units, p.n_kvt, dev.sm_count);
   p.kvt_per_split = (p.n_kvt + n_split - 1) / n_split;
   n_split = (p.n_kvt + p.kvt_per_split - 1) / p.kvt_per_split;  // no empty split
   p.n_split = n_split;
@@ -468,7 +807,7 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
 
   void* ws = nullptr;
   if (n_split > 1) {
-    const size_t o_elems = (size_t)n_split * B * N * H * Tr::D;
+    const size_t o_elems = (size_t)n_split * B * N * H * D;
     const size_t l_elems = (size_t)n_split * B * H * N;
     if (cudaMallocAsync(&ws, (o_elems + l_elems) * sizeof(float), stream) != cudaSuccess) {
       cudaGetLastError();
@@ -477,9 +816,7 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
     p.o_part = static_cast<float*>(ws);
     p.lse_part = p.o_part + o_elems;
   }
-
-  auto kern = fa_fwd_kernel<T, Tr>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
     cudaGetLastError();
     if (ws) cudaFreeAsync(ws, stream);
@@ -489,13 +826,13 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   cudaEvent_t ev0, ev1;
   take_kernel_events(false, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  kern<<<grid, 224, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, p);
+  kern<<<grid, THREADS, SMEM, stream>>>(tmq, tmk, tmv, p);
   rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);
   if (rc == FA_OK && n_split > 1) {
     const long long rows = (long long)B * N * H;
-    fa_combine_kernel<T, Tr::D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+    fa_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
         p.o_part, p.lse_part, static_cast<T*>(o), lse, B, H, N, n_split);
     rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
     note_launches(1);
@@ -504,19 +841,43 @@ static int run_fwd(const void* q, const void* k, const void* v, void* o, float* 
   return rc;
 }
 
+template <class T, class Tr>
+static int run_single(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_fwd<T, Tr::D, 128, Tr::BN, 224, Tr::SMEM_BYTES>(
+      fa_fwd_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
+}
+
+template <class T, class Tr>
+static int run_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_fwd<T, Tr::D, 256, Tr::BN, 320, Tr::SMEM_BYTES>(
+      fa_fwd_pp_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
+}
+
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int N, int d, float scale, cudaStream_t stream) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
+  // Two Q tiles per unit once a head has more than one tile's worth of rows;
+  // a single tile per unit for short sequences and for d = 256 (whose O
+  // accumulator leaves tensor memory room for only one Q tile).
+  const bool pair = N > 128;
   switch (d) {
     case 64:
-      return run_fwd<T, FwdTraits<64, 128, 4, 4>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+      return pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(q, k, v, o, lse, B, H, N, scale, stream, dev)
+                  : run_single<T, FwdTraits<64, 128, 4, 4>>(q, k, v, o, lse, B, H, N, scale,
+                                                             stream, dev);
     case 128:
-      return run_fwd<T, FwdTraits<128, 128, 3, 2>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+      return pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream,
+                                                      dev)
+                  : run_single<T, FwdTraits<128, 128, 3, 2>>(q, k, v, o, lse, B, H, N, scale,
+                                                              stream, dev);
     case 256:
-      return run_fwd<T, FwdTraits<256, 64, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream, dev);
+      return run_single<T, FwdTraits<256, 64, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream,
+                                                     dev);
     default:
       return FA_ERR_HEADDIM;
   }
