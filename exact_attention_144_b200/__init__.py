@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
     lib.fa_set_kernel_events.argtypes = [vp, vp, vp, vp]
     lib.fa_set_kernel_events.restype = i
     lib.fa_kernel_launches.restype = ctypes.c_ulonglong
+    lib.fa_last_cuda_error.restype = i
     _lib = lib
     return lib
 
@@ -67,7 +68,10 @@ FA_ERR_SCRATCH = -9
 
 class FAError(RuntimeError):
     def __init__(self, where: str, status: int):
-        super().__init__(f"{where}: {fa_status_string(status)} (status {status})")
+        msg = f"{where}: {fa_status_string(status)} (status {status})"
+        if status == FA_ERR_LAUNCH:
+            msg += f", cudaError {_load().fa_last_cuda_error()}"
+        super().__init__(msg)
         self.status = status
 
 

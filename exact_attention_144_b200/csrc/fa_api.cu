@@ -12,6 +12,23 @@ namespace fa {
 __device__ unsigned long long g_status = 0;
 
 static std::atomic<unsigned long long> g_launches{0};
+static std::atomic<int> g_last_cuda_error{0};
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return FA_OK;
+  g_last_cuda_error.store((int)e);
+  return FA_ERR_LAUNCH;
+}
+
+int check_launch_regs(const void* kernel) {
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kernel);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return launch_status(e);
+  }
+  return attr.numRegs >= kLaunchRegs ? FA_OK : launch_status(cudaErrorInvalidConfiguration);
+}
 static std::mutex g_event_mu;
 static cudaEvent_t g_events[4] = {nullptr, nullptr, nullptr, nullptr};
 
@@ -295,6 +312,8 @@ FA_EXPORT int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
 }
 
 FA_EXPORT unsigned long long fa_kernel_launches(void) { return fa::g_launches.load(); }
+
+FA_EXPORT int fa_last_cuda_error(void) { return fa::g_last_cuda_error.load(); }
 
 FA_EXPORT int fa_version(void) { return 100; }
 

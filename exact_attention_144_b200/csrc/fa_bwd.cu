@@ -16,7 +16,7 @@
 //                       loop walks the Q tiles of 128 queries
 //   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to 16 bits
 //
-// fa_bwd_kernel layout (320 threads, one block per SM):
+// fa_bwd_kernel layout (384 threads, one block per SM):
 //   warps 0-7  compute: warp w owns TMEM lane quadrant w % 4 and half w / 4 of
 //              the 128 query columns; P and dS are elementwise in (key, query),
 //              so the halves need no exchange.  They recompute P^T and dS^T,
@@ -24,6 +24,8 @@
 //              reduce-add into the fp32 accumulator) and store dK, dV
 //   warp  8    TMA producer
 //   warp  9    TMEM allocator and tcgen05.mma issuer
+//   warps 10-11 idle (three whole warpgroups, so registers can move from the
+//              producer/MMA warpgroup to the compute ones)
 // MMA issue order per Q tile i: dV += P^T dO_i as soon as P^T is written,
 // then S^T for tile i+1 (so the next P^T can start while dS^T is computed),
 // then dK += dS^T Q_i, dQ_i = dS K and dP^T for tile i+1.
@@ -120,7 +122,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 }
 
 template <class T, class Tr>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(384, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
                   const __grid_constant__ CUtensorMap tmacc, const BwdParams p) {
@@ -172,7 +174,8 @@ __global__ void __maxnreg__(200)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    regs_shrink();  // all four warps of the producer/MMA warpgroup
   if (warp == 8) {
     // -------------------------------------------------------- producer
     if (lane == 0) {
@@ -286,7 +289,9 @@ __global__ void __maxnreg__(200)
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();
+  }  // warps 10 and 11 have no role
   } else {
+    regs_grow();  // both compute warpgroups
     // ----------------------------- compute warps 0-7: P^T, dS^T, dQ drain
     // Warp w owns TMEM lane quadrant w % 4 (key rows of S^T/dP^T, query rows
     // of dQ) and half hf = w / 4 of the columns.
@@ -570,21 +575,22 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
   fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
       Npad);
-  rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  rc = launch_status(cudaGetLastError());
   note_launches(1);
   if (rc == FA_OK) {
     auto kern = fa_bwd_kernel<T, Tr>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Tr::SMEM_BYTES) != cudaSuccess) {
-      cudaGetLastError();
-      rc = FA_ERR_LAUNCH;
+    if ((rc = check_launch_regs((const void*)kern)) != FA_OK) {
+      // refused: the register split would not fit this build's allocation
+    } else if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Tr::SMEM_BYTES) != cudaSuccess) {
+      rc = launch_status(cudaGetLastError());
     } else {
       dim3 grid((N + Tr::BN - 1) / Tr::BN, H, B);
       cudaEvent_t ev0, ev1;
       take_kernel_events(true, &ev0, &ev1);
       if (ev0) cudaEventRecord(ev0, stream);
-      kern<<<grid, 320, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
-      rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+      kern<<<grid, 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
+      rc = launch_status(cudaGetLastError());
       if (ev1) cudaEventRecord(ev1, stream);
       note_launches(1);
     }
@@ -593,7 +599,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
     const long long total = (long long)B * N * H * D;
     fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
         p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
-    rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+    rc = launch_status(cudaGetLastError());
     note_launches(1);
   }
   cudaFreeAsync(ws, stream);
@@ -698,20 +704,19 @@ static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, co
   fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
       Npad);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
   auto kern = fa_bwd_kernel<T, Tr>;
+  if ((rc = check_launch_regs((const void*)kern)) != FA_OK) return rc;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_LAUNCH;
-  }
-  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 320, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv,
+      cudaSuccess)
+    return launch_status(cudaGetLastError());
+  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv,
                                                                                tmdo, tmacc, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
   const long long total = (long long)B * N * H * D;
   fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
       p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
   note_launches(3);
   return FA_OK;
 }

@@ -77,7 +77,7 @@ struct WaitCtl {
   unsigned long long* status;
 };
 
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtl w, int site) {
+static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtl w, int site) {
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
@@ -98,7 +98,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WaitCtl
 }
 
 // Wait used while draining at exit: ignores the abort flag, bounded by time.
-static __device__ __noinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+static __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
@@ -266,6 +266,21 @@ struct Elem<__half> {
     return __half22float2(v);
   }
 };
+
+// ------------------------------------------------------ register rebalance
+// Per-warpgroup register limits for the 384-thread kernels: launched with 168
+// registers a thread (64,512 in all), the two compute warpgroups grow to 208
+// and the producer/MMA warpgroup shrinks to 88 (2*128*208 + 128*88 = 64,512).
+// Executed by all four warps of a warpgroup.
+constexpr int kLaunchRegs = 168, kComputeRegs = 208, kControlRegs = 88;
+static_assert(2 * 128 * kComputeRegs + 128 * kControlRegs <= 384 * kLaunchRegs,
+              "register split exceeds the launch allocation");
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kComputeRegs) : "memory");
+}
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs) : "memory");
+}
 
 // --------------------------------------------------------------- fast math
 // Hardware base-2 exponential and logarithm (PTX ex2.approx / lg2.approx).

@@ -9,11 +9,13 @@
 //
 // Two persistent kernels, both one block per SM looping over work units:
 //
-// fa_fwd_pp_kernel (d = 64, 128; 320 threads) -- two 128-row Q tiles per unit
+// fa_fwd_pp_kernel (d = 64, 128; 384 threads) -- two 128-row Q tiles per unit
 //   warps 0-3  softmax + epilogue of Q tile 0 (thread t owns row t, TMEM lane t)
 //   warps 4-7  softmax + epilogue of Q tile 1
 //   warp  8    TMA producer: the Q pair once per unit, then K_j, V_j in turn
 //   warp  9    TMEM allocator and the single-thread tcgen05.mma issuer
+//   warps 10-11 idle (the block is three whole warpgroups so that registers
+//              can move from the producer/MMA warpgroup to the softmax ones)
 //   TMEM: S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d,256+2d).
 //   MMA order per K/V tile j: P0.V_j, Q0 K_{j+1}^T, P1.V_j, Q1 K_{j+1}^T, so
 //   the tensor cores work on one tile while the other tile's exponentials run,
@@ -239,7 +241,7 @@ struct FwdPPTraits {
 };
 
 template <class T, class Tr>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -289,7 +291,8 @@ __global__ void __maxnreg__(200)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    regs_shrink();  // all four warps of the producer/MMA warpgroup
   if (warp == 8) {
     // ------------------------------------------------------- producer
     if (lane == 0) {
@@ -417,7 +420,9 @@ __global__ void __maxnreg__(200)
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();
+  }  // warps 10 and 11 have no role
   } else {
+    regs_grow();  // both compute warpgroups
     // ------------------------------- softmax and epilogue, Q tile wg
     const int wg = warp >> 2;           // which Q tile
     const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
@@ -776,7 +781,8 @@ static int choose_splits(long long base_units, int n_kvt, int sm_count) {
   return n_split;
 }
 
-template <class T, int D, int BM_UNIT, int BN, int THREADS, int SMEM, class Kernel>
+template <class T, int D, int BM_UNIT, int BN, int THREADS, int SMEM, bool SPLIT_REGS,
+          class Kernel>
 static int launch_fwd(Kernel kern, const void* q, const void* k, const void* v, void* o,
                       float* lse, int B, int H, int N, float scale, cudaStream_t stream,
                       const DeviceInfo& dev) {
@@ -816,25 +822,29 @@ static int launch_fwd(Kernel kern, const void* q, const void* k, const void* v, 
     p.o_part = static_cast<float*>(ws);
     p.lse_part = p.o_part + o_elems;
   }
+  if (SPLIT_REGS && (rc = check_launch_regs((const void*)kern)) != FA_OK) {
+    if (ws) cudaFreeAsync(ws, stream);
+    return rc;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
-    cudaGetLastError();
+    rc = launch_status(cudaGetLastError());
     if (ws) cudaFreeAsync(ws, stream);
-    return FA_ERR_LAUNCH;
+    return rc;
   }
   const int grid = p.n_units < dev.sm_count ? p.n_units : dev.sm_count;
   cudaEvent_t ev0, ev1;
   take_kernel_events(false, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
   kern<<<grid, THREADS, SMEM, stream>>>(tmq, tmk, tmv, p);
-  rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+  rc = launch_status(cudaGetLastError());
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);
   if (rc == FA_OK && n_split > 1) {
     const long long rows = (long long)B * N * H;
     fa_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
         p.o_part, p.lse_part, static_cast<T*>(o), lse, B, H, N, n_split);
-    rc = (cudaGetLastError() == cudaSuccess) ? FA_OK : FA_ERR_LAUNCH;
+    rc = launch_status(cudaGetLastError());
     note_launches(1);
   }
   if (ws) cudaFreeAsync(ws, stream);
@@ -844,14 +854,14 @@ static int launch_fwd(Kernel kern, const void* q, const void* k, const void* v, 
 template <class T, class Tr>
 static int run_single(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
-  return launch_fwd<T, Tr::D, 128, Tr::BN, 224, Tr::SMEM_BYTES>(
+  return launch_fwd<T, Tr::D, 128, Tr::BN, 224, Tr::SMEM_BYTES, false>(
       fa_fwd_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
 }
 
 template <class T, class Tr>
 static int run_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                   int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
-  return launch_fwd<T, Tr::D, 256, Tr::BN, 320, Tr::SMEM_BYTES>(
+  return launch_fwd<T, Tr::D, 256, Tr::BN, 384, Tr::SMEM_BYTES, true>(
       fa_fwd_pp_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
 }
 

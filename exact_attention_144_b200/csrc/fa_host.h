@@ -20,6 +20,14 @@ struct DeviceInfo {
 // 10.0, or FA_ERR_LAUNCH when the runtime cannot be queried.
 int current_device(DeviceInfo* info);
 
+// FA_OK when e is cudaSuccess; otherwise records e (fa_last_cuda_error) and
+// returns FA_ERR_LAUNCH.
+int launch_status(cudaError_t e);
+
+// FA_OK when the kernel was compiled with the register count its warpgroup
+// register split assumes (kLaunchRegs a thread at 384 threads).
+int check_launch_regs(const void* kernel);
+
 // Counts kernel launches (fa_kernel_launches).
 void note_launches(unsigned n);
 

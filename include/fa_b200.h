@@ -153,6 +153,12 @@ int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
 /* Number of kernel launches this library has issued since it was loaded. */
 unsigned long long fa_kernel_launches(void);
 
+/*
+ * The cudaError_t value behind the most recent FA_ERR_LAUNCH returned by any
+ * call of this library in the process (0 if none).  Diagnostic only.
+ */
+int fa_last_cuda_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int fa_version(void);
 

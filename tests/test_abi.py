@@ -28,7 +28,8 @@ def test_every_declared_symbol_is_exported(fa):
     names = fa.declared_functions()
     assert set(names) >= {"fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_status_string",
                           "fa_get_device_status", "fa_selftest_bounded_wait", "fa_version",
-                          "fa_set_kernel_events", "fa_kernel_launches", "fa_bwd_noalloc"}
+                          "fa_set_kernel_events", "fa_kernel_launches", "fa_bwd_noalloc",
+                          "fa_last_cuda_error"}
     lib = fa.lib()
     for n in names:
         assert hasattr(lib, n), n
