@@ -29,9 +29,9 @@
 // MMA issue order per Q tile i: dV += P^T dO_i as soon as P^T is written,
 // then S^T for tile i+1 (so the next P^T can start while dS^T is computed),
 // then dK += dS^T Q_i, dQ_i = dS K and dP^T for tile i+1.
-// Tensor memory (d = 64): S^T [0,128) (P^T over its first 64 columns),
-// dP^T [128,256) (dS^T over its first 64), dV [256,320), dK [320,384),
-// dQ [384,448).
+// Tensor memory (d = 64): S^T [0,128), dP^T [128,256), dV [256,320),
+// dK [320,384), dQ [384,448).  Packed 16-bit P^T and dS^T overwrite the first
+// 32 columns of each 64-column query half of S^T and dP^T.
 #include <mutex>
 
 #include "fa_common.cuh"
@@ -210,6 +210,12 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);             // TS, B MN-major
       constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, D, true) | (1u << 15);  // A, B MN-major
       auto q_s = [&](int i) { return sQ + (i % QST) * Tr::QT_BYTES; };
+      // Packed 16-bit P^T / dS^T: query half hf sits in the first 32 columns of
+      // its own 64-column half of the S^T / dP^T region (a half never writes
+      // columns that the other half may still be reading).
+      auto packed_col = [](int kk) -> uint32_t {
+        return (uint32_t)((kk / (HC / 16)) * HC + (kk % (HC / 16)) * 8);
+      };
       auto do_s = [&](int i) { return sDO + (i % QST) * Tr::QT_BYTES; };
       // S^T = K Q_i^T into TM_S; dP^T = V dO_i^T into TM_DP (K-major over d)
       auto issue_s = [&](int i) {
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_S + kk * 8,
+          umma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
                   sw128_desc(do_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
         // the next S^T overwrites TM_S after dV has read P^T (same issue order)
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DP + kk * 8,
+          umma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
                   sw128_desc(q_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(Tr::B_Q_EMPTY + i % QST));
@@ -372,8 +378,8 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t pk[HC / 2];
 #pragma unroll
         for (int j = 0; j < HC / 2; ++j) pk[j] = Elem<T>::pack(pr[2 * j], pr[2 * j + 1]);
-        tmem_st16(tl + Tr::TM_S + hf * (HC / 2), &pk[0]);
-        tmem_st16(tl + Tr::TM_S + hf * (HC / 2) + 16, &pk[16]);
+        tmem_st16(tl + Tr::TM_S + hf * HC, &pk[0]);
+        tmem_st16(tl + Tr::TM_S + hf * HC + 16, &pk[16]);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -406,8 +412,8 @@ __global__ void __launch_bounds__(384, 1)
           dk16[2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
         }
       }
-      tmem_st16(tl + Tr::TM_DP + hf * (HC / 2), &dk16[0]);
-      tmem_st16(tl + Tr::TM_DP + hf * (HC / 2) + 16, &dk16[16]);
+      tmem_st16(tl + Tr::TM_DP + hf * HC, &dk16[0]);
+      tmem_st16(tl + Tr::TM_DP + hf * HC + 16, &dk16[16]);
       // dS row r, query chunk hf, into the 128-byte-swizzled shared tile
       uint8_t* ds_g = gDS + (i & 1) * Tr::DS_BYTES + hf * (BN * 128) + r * 128;
 #pragma unroll
