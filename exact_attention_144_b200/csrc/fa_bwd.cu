@@ -87,12 +87,13 @@ struct BwdParams {
 enum { kBSiteQEmpty = 0x21, kBSiteKV, kBSiteQFull, kBSiteDsReady, kBSiteDqFree, kBSiteSFull,
        kBSiteDpFull, kBSiteQFullSm, kBSiteDsBuf, kBSiteDqFull, kBSiteKvDone, kBSitePReady };
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
+__device__ __forceinline__ void bulk_load(bool issue, uint32_t dst, const void* src,
+                                          uint32_t bytes, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      "\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "r"((uint32_t)issue)
       : "memory");
 }
 // Reduce-add of a shared-memory tile into global memory through a tensor map
@@ -178,23 +179,24 @@ __global__ void __launch_bounds__(384, 1)
     regs_shrink();  // all four warps of the producer/MMA warpgroup
   if (warp == 8) {
     // -------------------------------------------------------- producer
-    if (lane == 0) {
-      mbar_expect_tx(bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
-      tma_load_4d(sK, &tmk, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
-      tma_load_4d(sV, &tmv, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
+      mbar_expect_tx(leader, bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
+      tma_load_4d(leader, sK, &tmk, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
+      tma_load_4d(leader, sV, &tmv, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
       const size_t row0 = ((size_t)b * p.H + h) * p.Npad;
       int issued = 0;
       for (int i = 0; i < n_qt; ++i) {
         const int qs = i % QST;
         if (i >= QST &&
-            !mbar_wait(bar(Tr::B_Q_EMPTY + qs), ((i / QST) - 1) & 1, w, kBSiteQEmpty))
+            !mbar_wait_warp(bar(Tr::B_Q_EMPTY + qs), ((i / QST) - 1) & 1, w, kBSiteQEmpty))
           break;
         const uint32_t fb = bar(Tr::B_Q_FULL + qs);
-        mbar_expect_tx(fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
-        tma_load_4d(sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, i * BM, b);
-        tma_load_4d(sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, i * BM, b);
-        bulk_load(base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
-        bulk_load(base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
+        mbar_expect_tx(leader, fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
+        tma_load_4d(leader, sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, i * BM, b);
+        tma_load_4d(leader, sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, i * BM, b);
+        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
+        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
         ++issued;
       }
       mbar_drain(bar(Tr::B_KV_FULL), 0, p.limit_ns);
@@ -204,7 +206,8 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ----------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t fmt = Elem<T>::kFmt;
       constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);            // K-major x K-major
       constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);             // TS, B MN-major
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(tmem + Tr::TM_S, sw128_desc(sK + ch * (BN * 128) + in, 16, 1024),
+          umma_ss(leader, tmem + Tr::TM_S, sw128_desc(sK + ch * (BN * 128) + in, 16, 1024),
                   sw128_desc(q_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
         }
       };
@@ -230,68 +233,68 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(tmem + Tr::TM_DP, sw128_desc(sV + ch * (BN * 128) + in, 16, 1024),
+          umma_ss(leader, tmem + Tr::TM_DP, sw128_desc(sV + ch * (BN * 128) + in, 16, 1024),
                   sw128_desc(do_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP,
                   kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
+      bool ok = mbar_wait_warp(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
       if (ok && n_qt > 0) {
-        ok = mbar_wait(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull);
+        ok = mbar_wait_warp(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull);
         if (ok) {
           tc_fence_after();
           issue_s(0);
-          umma_commit(bar(Tr::B_S_FULL));
+          umma_commit(leader, bar(Tr::B_S_FULL));
           issue_dp(0);
-          umma_commit(bar(Tr::B_DP_FULL));
+          umma_commit(leader, bar(Tr::B_DP_FULL));
         }
       }
       for (int i = 0; i < n_qt && ok; ++i) {
         // dV += P^T dO_i  (A = P^T from TMEM, B = dO_i: queries x d, MN-major)
-        if (!(ok = mbar_wait(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
+        if (!(ok = mbar_wait_warp(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
+          umma_ts(leader, tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
                   sw128_desc(do_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
         // the next S^T overwrites TM_S after dV has read P^T (same issue order)
         const bool more = i + 1 < n_qt;
         if (more) {
-          if (!(ok = mbar_wait(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
                                kBSiteQFull)))
             break;
           tc_fence_after();
           issue_s(i + 1);
-          umma_commit(bar(Tr::B_S_FULL));
+          umma_commit(leader, bar(Tr::B_S_FULL));
         }
         // dK += dS^T Q_i  (A = dS^T from TMEM, B = Q_i MN-major)
-        if (!(ok = mbar_wait(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+        if (!(ok = mbar_wait_warp(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
+          umma_ts(leader, tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
                   sw128_desc(q_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
                   (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(Tr::B_Q_EMPTY + i % QST));
+        umma_commit(leader, bar(Tr::B_Q_EMPTY + i % QST));
         // dQ_i = dS K  (A = dS from shared memory, queries contiguous; B = K, d contiguous)
-        if (i > 0 && !(ok = mbar_wait(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree))) break;
+        if (i > 0 && !(ok = mbar_wait_warp(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree))) break;
         tc_fence_after();
         const uint32_t ds_s = sDS + (i & 1) * Tr::DS_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ss(tmem + Tr::TM_DQ, sw128_desc(ds_s + kk * 16 * 128, BN * 128, 1024),
+          umma_ss(leader, tmem + Tr::TM_DQ, sw128_desc(ds_s + kk * 16 * 128, BN * 128, 1024),
                   sw128_desc(sK + kk * 16 * 128, BN * 128, 1024), kIdescDQ, kk > 0 ? 1u : 0u);
-        umma_commit(bar(Tr::B_DQ_FULL));
-        umma_commit(bar(Tr::B_DSBUF_FREE + (i & 1)));
+        umma_commit(leader, bar(Tr::B_DQ_FULL));
+        umma_commit(leader, bar(Tr::B_DSBUF_FREE + (i & 1)));
         // the next dP^T overwrites TM_DP after dK has read dS^T
         if (more) {
           issue_dp(i + 1);
-          umma_commit(bar(Tr::B_DP_FULL));
+          umma_commit(leader, bar(Tr::B_DP_FULL));
         }
       }
-      umma_commit(bar(Tr::B_KV_DONE));
-      umma_commit(bar(Tr::B_DRAIN));
+      umma_commit(leader, bar(Tr::B_KV_DONE));
+      umma_commit(leader, bar(Tr::B_DRAIN));
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();

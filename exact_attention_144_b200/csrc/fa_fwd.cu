@@ -295,39 +295,40 @@ __global__ void __launch_bounds__(384, 1)
     regs_shrink();  // all four warps of the producer/MMA warpgroup
   if (warp == 8) {
     // ------------------------------------------------------- producer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, vc = 0, qc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, p);
-        if (qc > 0 && !(ok = mbar_wait(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
-        mbar_expect_tx(bar(Tr::B_Q_FULL), 2 * Tr::QT_BYTES);
+        if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
+        mbar_expect_tx(leader, bar(Tr::B_Q_FULL), 2 * Tr::QT_BYTES);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64,
+            tma_load_4d(leader, sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64,
                         un.h, (2 * un.qt + t) * BM, un.b);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t ks = kc % KST;
           if (kc >= (uint32_t)KST &&
-              !(ok = mbar_wait(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
+              !(ok = mbar_wait_warp(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
             break;
-          mbar_expect_tx(bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
+          mbar_expect_tx(leader, bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
+            tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
                         c * 64, un.h, t * BN, un.b);
           ++kc;
           const uint32_t vs = vc % VST;
           if (vc >= (uint32_t)VST &&
-              !(ok = mbar_wait(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
+              !(ok = mbar_wait_warp(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
             break;
-          mbar_expect_tx(bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
+          mbar_expect_tx(leader, bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
+            tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
                         c * 64, un.h, t * BN, un.b);
           ++vc;
         }
@@ -342,7 +343,8 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ----------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t kIdescQK = f16_idesc(Elem<T>::kFmt, 128, BN, false);
       constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
       uint32_t kc = 0, vc = 0, g = 0, uc = 0;
@@ -354,7 +356,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(tmem + t * BN, sw128_desc(qbase + ch * (BM * 128) + in, 16, 1024),
+          umma_ss(leader, tmem + t * BN, sw128_desc(qbase + ch * (BM * 128) + in, 16, 1024),
                   sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
                   kk > 0 ? 1u : 0u);
         }
@@ -364,51 +366,51 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t vbase = sV + (vc % VST) * Tr::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
+          umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
                   sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
                   (!first || kk > 0) ? 1u : 0u);
       };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, p);
         const int n = un.t1 - un.t0;
-        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
-        if (!(ok = mbar_wait(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))) break;
+        if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
+        if (!(ok = mbar_wait_warp(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))) break;
         tc_fence_after();
         issue_qk(0);
-        umma_commit(bar(Tr::B_S_FULL + 0));
+        umma_commit(leader, bar(Tr::B_S_FULL + 0));
         issue_qk(1);
-        umma_commit(bar(Tr::B_S_FULL + 1));
-        umma_commit(bar(Tr::B_K_EMPTY + kc % KST));
-        if (n == 1) umma_commit(bar(Tr::B_Q_EMPTY));
+        umma_commit(leader, bar(Tr::B_S_FULL + 1));
+        umma_commit(leader, bar(Tr::B_K_EMPTY + kc % KST));
+        if (n == 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
         ++kc;
         for (int j = 0; j < n; ++j, ++g) {
           // tile 0: P0 V_j, then S0 for the next K tile
-          if (!(ok = mbar_wait(bar(Tr::B_P_FULL + 0), g & 1u, w, kSitePFull))) break;
-          if (!(ok = mbar_wait(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
+          if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 0), g & 1u, w, kSitePFull))) break;
+          if (!(ok = mbar_wait_warp(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
             break;
           tc_fence_after();
           issue_pv(0, j == 0);
-          umma_commit(bar(Tr::B_O_DONE + 0));
+          umma_commit(leader, bar(Tr::B_O_DONE + 0));
           const bool more = j + 1 < n;
           if (more) {
-            if (!(ok = mbar_wait(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull)))
+            if (!(ok = mbar_wait_warp(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull)))
               break;
             tc_fence_after();
             issue_qk(0);
-            umma_commit(bar(Tr::B_S_FULL + 0));
+            umma_commit(leader, bar(Tr::B_S_FULL + 0));
           }
           // tile 1: P1 V_j, then S1 for the next K tile
-          if (!(ok = mbar_wait(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
+          if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
           tc_fence_after();
           issue_pv(1, j == 0);
-          umma_commit(bar(Tr::B_O_DONE + 1));
-          umma_commit(bar(Tr::B_V_EMPTY + vc % VST));
+          umma_commit(leader, bar(Tr::B_O_DONE + 1));
+          umma_commit(leader, bar(Tr::B_V_EMPTY + vc % VST));
           ++vc;
           if (more) {
             issue_qk(1);
-            umma_commit(bar(Tr::B_S_FULL + 1));
-            umma_commit(bar(Tr::B_K_EMPTY + kc % KST));
-            if (j + 2 == n) umma_commit(bar(Tr::B_Q_EMPTY));
+            umma_commit(leader, bar(Tr::B_S_FULL + 1));
+            umma_commit(leader, bar(Tr::B_K_EMPTY + kc % KST));
+            if (j + 2 == n) umma_commit(leader, bar(Tr::B_Q_EMPTY));
             ++kc;
           }
         }
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
         ++uc;
       }
       // Every issued MMA must finish before tensor memory is released.
-      umma_commit(bar(Tr::B_DRAIN));
+      umma_commit(leader, bar(Tr::B_DRAIN));
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();
@@ -561,27 +563,28 @@ __global__ void __launch_bounds__(224, 1)
 
   if (warp == 4) {
     // ------------------------------------------------ Q and K producer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, qc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, p);
-        if (qc > 0 && !(ok = mbar_wait(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
-        mbar_expect_tx(bar(Tr::B_Q_FULL), Tr::Q_BYTES);
+        if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
+        mbar_expect_tx(leader, bar(Tr::B_Q_FULL), Tr::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < Tr::KCH; ++c)
-          tma_load_4d(sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64, un.h,
+          tma_load_4d(leader, sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64, un.h,
                       un.qt * Tr::BM, un.b);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t ks = kc % KST;
           if (kc >= (uint32_t)KST &&
-              !(ok = mbar_wait(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
+              !(ok = mbar_wait_warp(bar(Tr::B_K_EMPTY + ks), ((kc / KST) - 1) & 1u, w, kSiteKEmpty)))
             break;
-          mbar_expect_tx(bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
+          mbar_expect_tx(leader, bar(Tr::B_K_FULL + ks), Tr::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
+            tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
                         c * 64, un.h, t * BN, un.b);
           ++kc;
         }
@@ -594,7 +597,8 @@ __global__ void __launch_bounds__(224, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------ V producer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t vc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -602,12 +606,12 @@ __global__ void __launch_bounds__(224, 1)
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t vs = vc % VST;
           if (vc >= (uint32_t)VST &&
-              !(ok = mbar_wait(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
+              !(ok = mbar_wait_warp(bar(Tr::B_V_EMPTY + vs), ((vc / VST) - 1) & 1u, w, kSiteVEmpty)))
             break;
-          mbar_expect_tx(bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
+          mbar_expect_tx(leader, bar(Tr::B_V_FULL + vs), Tr::KV_BYTES);
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
+            tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
                         c * 64, un.h, t * BN, un.b);
           ++vc;
         }
@@ -618,7 +622,8 @@ __global__ void __launch_bounds__(224, 1)
     __syncwarp();
   } else if (warp == 6) {
     // ----------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t kIdescQK = f16_idesc(Elem<T>::kFmt, 128, BN, false);
       constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
       uint32_t kc = 0, vc = 0, g = 0, uc = 0;
@@ -626,42 +631,42 @@ __global__ void __launch_bounds__(224, 1)
       // O += P_j V_j for the tile whose S/P buffer use counter is gp.
       auto issue_pv = [&](uint32_t gp, bool first) -> bool {
         const uint32_t pb = gp & 1u;
-        if (!mbar_wait(bar(Tr::B_P_FULL + pb), (gp >> 1) & 1u, w, kSitePFull)) return false;
+        if (!mbar_wait_warp(bar(Tr::B_P_FULL + pb), (gp >> 1) & 1u, w, kSitePFull)) return false;
         const uint32_t vs = vc % VST;
-        if (!mbar_wait(bar(Tr::B_V_FULL + vs), (vc / VST) & 1u, w, kSiteVFull)) return false;
+        if (!mbar_wait_warp(bar(Tr::B_V_FULL + vs), (vc / VST) & 1u, w, kSiteVFull)) return false;
         tc_fence_after();
         const uint32_t vbase = sV + vs * Tr::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
+          umma_ts(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
                   sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
                   (!first || kk > 0) ? 1u : 0u);
-        umma_commit(bar(Tr::B_V_EMPTY + vs));
-        umma_commit(bar(Tr::B_O_DONE));
+        umma_commit(leader, bar(Tr::B_V_EMPTY + vs));
+        umma_commit(leader, bar(Tr::B_O_DONE));
         ++vc;
         return true;
       };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, p);
-        if (!(ok = mbar_wait(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
+        if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
         tc_fence_after();
         const int n = un.t1 - un.t0;
         for (int i = 0; i < n; ++i) {
           const uint32_t ks = kc % KST;
-          if (!(ok = mbar_wait(bar(Tr::B_K_FULL + ks), (kc / KST) & 1u, w, kSiteKFull))) break;
+          if (!(ok = mbar_wait_warp(bar(Tr::B_K_FULL + ks), (kc / KST) & 1u, w, kSiteKFull))) break;
           tc_fence_after();
           const uint32_t sb = g & 1u;
           const uint32_t kbase = sK + ks * Tr::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-            umma_ss(tmem + sb * BN, sw128_desc(sQ + ch * (Tr::BM * 128) + in, 16, 1024),
+            umma_ss(leader, tmem + sb * BN, sw128_desc(sQ + ch * (Tr::BM * 128) + in, 16, 1024),
                     sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
                     kk > 0 ? 1u : 0u);
           }
-          umma_commit(bar(Tr::B_K_EMPTY + ks));
-          umma_commit(bar(Tr::B_S_FULL + sb));
-          if (i == n - 1) umma_commit(bar(Tr::B_Q_EMPTY));
+          umma_commit(leader, bar(Tr::B_K_EMPTY + ks));
+          umma_commit(leader, bar(Tr::B_S_FULL + sb));
+          if (i == n - 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
           ++kc;
           if (i > 0 && !(ok = issue_pv(g - 1, i == 1))) break;
           ++g;
@@ -671,7 +676,7 @@ __global__ void __launch_bounds__(224, 1)
         ++uc;
       }
       // Every issued MMA must finish before tensor memory is released.
-      umma_commit(bar(Tr::B_DRAIN));
+      umma_commit(leader, bar(Tr::B_DRAIN));
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();

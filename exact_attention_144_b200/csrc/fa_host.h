@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/fa_b200.h"
+#include "fa_b200.h"  // include/ is on the include path
 
 namespace fa {
 
