@@ -116,12 +116,32 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+def replica_seed(w: attn_inputs.Workload, rank: int) -> int:
+    """Each rank owns one replica of the workload with its own seeded batch."""
+    return w.seed + 7919 * rank
+
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The slowest rank's value (timing is reported as the max over ranks)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flop_per_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job throughput: every rank processes flop_per_step in ms_per_step."""
+    return world * flop_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def cpu_oracle_sample(w: attn_inputs.Workload, rows: int, heads: int):
     """Times the fp64 oracle on a bounded sample of the workload: the first
-    `rows` query rows of `heads` heads (forward rows and their backward
-    contributions).  Returns (TFLOP/s at the workload's FLOP-per-row rate,
-    seconds, threads, description)."""
+    `rows` query rows of `heads` heads (forward rows and, for the training
+    workload, their backward contributions).  Returns (TFLOP/s at the
+    workload's FLOP-per-row rate, seconds, threads, description)."""
     import oracle  # the CPU baseline leg is one of the oracle's permitted users
+    rows = max(1, min(rows, w.N))
     q, k, v, do = attn_inputs.draw_workload(w, count=4)
     f64 = attn_inputs.to_f64
     hs = [(b, h) for b in range(w.B) for h in range(w.H)][:heads]
@@ -132,12 +152,15 @@ def cpu_oracle_sample(w: attn_inputs.Workload, rows: int, heads: int):
     sel = [(0, s, i) for s in range(len(hs)) for i in range(rows)]
     t0 = time.perf_counter()
     oracle.attn_fwd_rows(qs, ks, vs, w.scale, sel)
-    oracle.attn_bwd_rows(qs, ks, vs, ds, w.scale, 0, rows)
+    if w.backward:
+        oracle.attn_bwd_rows(qs, ks, vs, ds, w.scale, 0, rows)
     dt = time.perf_counter() - t0
-    flop = 14.0 * rows * w.N * w.d * len(hs)  # 4 (fwd) + 10 (bwd) per row, N keys, d
-    desc = (f"fp64 oracle fwd+bwd of query rows [0,{rows}) of {len(hs)} of {w.B * w.H} heads "
-            f"(N={w.N}, d={w.d}); {flop / 1e9:.2f} GFLOP of the step's "
-            f"{(w.fwd_flop + w.bwd_flop) / 1e9:.1f}")
+    per_row = 14.0 if w.backward else 4.0  # 4 (fwd) + 10 (bwd) per row, N keys, d
+    flop = per_row * rows * w.N * w.d * len(hs)
+    step = (w.fwd_flop + w.bwd_flop) if w.backward else w.fwd_flop
+    desc = (f"fp64 oracle {'fwd+bwd' if w.backward else 'fwd'} of query rows [0,{rows}) of "
+            f"{len(hs)} of {w.B * w.H} heads (N={w.N}, d={w.d}); {flop / 1e9:.2f} GFLOP of the "
+            f"step's {step / 1e9:.1f}")
     return flop / dt / 1e12, dt, oracle.num_threads(), desc
 
 
@@ -203,15 +226,8 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # Each rank owns one replica of the workload (its own seeded batch).
-    q, k, v, do = attn_inputs.draw(w.B, w.N, w.H, w.d, w.dtype, w.seed + 7919 * rank, 4,
+    q, k, v, do = attn_inputs.draw(w.B, w.N, w.H, w.d, w.dtype, replica_seed(w, rank), 4,
                                    std=w.std, device=dev)
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -249,8 +265,8 @@ def main():
     step_ms = [s0.elapsed_time(s1) for s0, s1, *_ in ev]
     fwd_ms = [f0.elapsed_time(f1) for _, _, f0, f1, _, _ in ev]
     bwd_ms = [b0.elapsed_time(b1) for *_, b0, b1 in ev] if train else []
-    ms = max_over_ranks(statistics.mean(step_ms))
-    value = world * flop_step / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(statistics.mean(step_ms), dist, dev)
+    value = job_tflops(flop_step, ms, world)
     status = fa.fa_get_device_status()
     if status != 0:
         raise RuntimeError(f"a kernel gave up a bounded wait (status {status:#x})")
@@ -274,7 +290,7 @@ def main():
         if i >= args.warmup:
             e2e_ev[i - args.warmup][1].record()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev))
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), dist, dev)
 
     # ----------------------------------------- roofline of the dominant kernel
     pk, pk_src = peaks()
@@ -323,7 +339,7 @@ def main():
                        "parallelism": f"replicas x{world} (batch per rank, no collective)",
                        "l2": "512 MiB written between timed steps",
                        "inputs": "seeded N(0,1) draws rounded to the 16-bit type"},
-            "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "e2e": {"value": job_tflops(flop_step, e2e_ms, world), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "roofline": roofline,
