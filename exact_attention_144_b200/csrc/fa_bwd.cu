@@ -23,12 +23,13 @@
 //              drain the dQ tiles (TMEM -> swizzled shared memory -> TMA
 //              reduce-add into the fp32 accumulator) and store dK, dV
 //   warp  8    TMA producer
-//   warp  9    TMEM allocator and tcgen05.mma issuer
-//   warps 10-11 idle (three whole warpgroups, so registers can move from the
+//   warp  9    TMEM allocator; issues S^T and dV
+//   warp 10    issues dP^T, dK and dQ
+//   warp 11    idle (three whole warpgroups, so registers can move from the
 //              producer/MMA warpgroup to the compute ones)
-// MMA issue order per Q tile i: dV += P^T dO_i as soon as P^T is written,
-// then S^T for tile i+1 (so the next P^T can start while dS^T is computed),
-// then dK += dS^T Q_i, dQ_i = dS K and dP^T for tile i+1.
+// Per Q tile i: dV += P^T dO_i as soon as P^T is written, then S^T for tile
+// i+1 (so the next P^T can start while dS^T is computed); dK += dS^T Q_i and
+// dQ_i = dS K as soon as dS^T is written, then dP^T for tile i+1.
 // Tensor memory (d = 64): S^T [0,128), dP^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448).  Packed 16-bit P^T and dS^T overwrite the first
 // 32 columns of each 64-column query half of S^T and dP^T.
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(Tr::B_KV_FULL), 1);
     for (int s = 0; s < QST; ++s) {
       mbar_init(bar(Tr::B_Q_FULL + s), 1);
-      mbar_init(bar(Tr::B_Q_EMPTY + s), 1);
+      mbar_init(bar(Tr::B_Q_EMPTY + s), 2);  // one commit from each MMA warp
     }
     mbar_init(bar(Tr::B_S_FULL), 1);
     mbar_init(bar(Tr::B_DP_FULL), 1);
@@ -163,8 +164,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(Tr::B_DSBUF_FREE + 1), 1);
     mbar_init(bar(Tr::B_DQ_FULL), 1);
     mbar_init(bar(Tr::B_DQ_FREE), 256);
-    mbar_init(bar(Tr::B_KV_DONE), 1);
-    mbar_init(bar(Tr::B_DRAIN), 1);
+    mbar_init(bar(Tr::B_KV_DONE), 2);
+    mbar_init(bar(Tr::B_DRAIN), 2);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -204,93 +205,92 @@ __global__ void __launch_bounds__(384, 1)
         if (issued > s) mbar_drain(bar(Tr::B_Q_FULL + s), ((issued - 1 - s) / QST) & 1, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ----------------------------------------------------- MMA issuer
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------ MMA issuers
+    // Two independent streams on two SM sub-partitions (an issuing warp
+    // shares its sub-partition's issue slots with two compute warps):
+    //   warp 9:  S^T = K Q_i^T and dV += P^T dO_i   (TMEM S^T and dV only)
+    //   warp 10: dP^T = V dO_i^T, dK += dS^T Q_i, dQ_i = dS K  (dP^T, dK, dQ)
+    // They share no TMEM columns; the Q/dO stage release and the final
+    // "all done" barriers count one commit from each.
     {
+      const bool stream_a = warp == 9;
       const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t fmt = Elem<T>::kFmt;
       constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);            // K-major x K-major
       constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);             // TS, B MN-major
       constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, D, true) | (1u << 15);  // A, B MN-major
-      auto q_s = [&](int i) { return sQ + (i % QST) * Tr::QT_BYTES; };
       // Packed 16-bit P^T / dS^T: query half hf sits in the first 32 columns of
       // its own 64-column half of the S^T / dP^T region (a half never writes
       // columns that the other half may still be reading).
       auto packed_col = [](int kk) -> uint32_t {
         return (uint32_t)((kk / (HC / 16)) * HC + (kk % (HC / 16)) * 8);
       };
-      auto do_s = [&](int i) { return sDO + (i % QST) * Tr::QT_BYTES; };
-      // S^T = K Q_i^T into TM_S; dP^T = V dO_i^T into TM_DP (K-major over d)
-      auto issue_s = [&](int i) {
+      // Descriptors are built once; each MMA only advances a start address.
+      const uint64_t k_kmaj = sw128_desc(sK, 16, 1024), v_kmaj = sw128_desc(sV, 16, 1024),
+                     q_kmaj = sw128_desc(sQ, 16, 1024), do_kmaj = sw128_desc(sDO, 16, 1024),
+                     q_mn = sw128_desc(sQ, BM * 128, 1024), do_mn = sw128_desc(sDO, BM * 128, 1024),
+                     ds_mn = sw128_desc(sDS, BN * 128, 1024), k_mn = sw128_desc(sK, BN * 128, 1024);
+      // S^T = K Q_i^T into TM_S (stream a); dP^T = V dO_i^T into TM_DP (stream b)
+      auto issue_first = [&](int i) {
+        const uint64_t a0 = stream_a ? k_kmaj : v_kmaj;
+        const uint64_t b0 = desc_advance(stream_a ? q_kmaj : do_kmaj, (i % QST) * Tr::QT_BYTES);
+        const uint32_t d_tmem = tmem + (stream_a ? Tr::TM_S : Tr::TM_DP);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(leader, tmem + Tr::TM_S, sw128_desc(sK + ch * (BN * 128) + in, 16, 1024),
-                  sw128_desc(q_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP, kk > 0 ? 1u : 0u);
+          umma_ss(leader, d_tmem, desc_advance(a0, ch * (BN * 128) + in),
+                  desc_advance(b0, ch * (BM * 128) + in), kIdescSP, kk > 0 ? 1u : 0u);
         }
-      };
-      auto issue_dp = [&](int i) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(leader, tmem + Tr::TM_DP, sw128_desc(sV + ch * (BN * 128) + in, 16, 1024),
-                  sw128_desc(do_s(i) + ch * (BM * 128) + in, 16, 1024), kIdescSP,
-                  kk > 0 ? 1u : 0u);
-        }
+        umma_commit(leader, bar(stream_a ? Tr::B_S_FULL : Tr::B_DP_FULL));
       };
       bool ok = mbar_wait_warp(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
-      if (ok && n_qt > 0) {
-        ok = mbar_wait_warp(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-          umma_commit(leader, bar(Tr::B_S_FULL));
-          issue_dp(0);
-          umma_commit(leader, bar(Tr::B_DP_FULL));
-        }
+      if (ok && n_qt > 0 && (ok = mbar_wait_warp(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull))) {
+        tc_fence_after();
+        issue_first(0);
       }
       for (int i = 0; i < n_qt && ok; ++i) {
-        // dV += P^T dO_i  (A = P^T from TMEM, B = dO_i: queries x d, MN-major)
-        if (!(ok = mbar_wait_warp(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
-                  sw128_desc(do_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
-                  (i > 0 || kk > 0) ? 1u : 0u);
-        // the next S^T overwrites TM_S after dV has read P^T (same issue order)
         const bool more = i + 1 < n_qt;
-        if (more) {
-          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
-                               kBSiteQFull)))
+        if (stream_a) {
+          // dV += P^T dO_i  (A = P^T from TMEM, B = dO_i: queries x d, MN-major)
+          if (!(ok = mbar_wait_warp(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(leader, tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
+                    desc_advance(do_mn, (i % QST) * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_Q_EMPTY + i % QST));
+        } else {
+          // dK += dS^T Q_i  (A = dS^T from TMEM, B = Q_i MN-major)
+          if (!(ok = mbar_wait_warp(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(leader, tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
+                    desc_advance(q_mn, (i % QST) * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_Q_EMPTY + i % QST));
+          // dQ_i = dS K  (A = dS from shared memory, queries contiguous; B = K, d contiguous)
+          if (i > 0 && !(ok = mbar_wait_warp(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree)))
             break;
           tc_fence_after();
-          issue_s(i + 1);
-          umma_commit(leader, bar(Tr::B_S_FULL));
+          const uint64_t dsd = desc_advance(ds_mn, (i & 1) * Tr::DS_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ss(leader, tmem + Tr::TM_DQ, desc_advance(dsd, kk * 16 * 128),
+                    desc_advance(k_mn, kk * 16 * 128), kIdescDQ, kk > 0 ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_DQ_FULL));
+          umma_commit(leader, bar(Tr::B_DSBUF_FREE + (i & 1)));
         }
-        // dK += dS^T Q_i  (A = dS^T from TMEM, B = Q_i MN-major)
-        if (!(ok = mbar_wait_warp(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
-                  sw128_desc(q_s(i) + kk * 16 * 128, BM * 128, 1024), kIdescAcc,
-                  (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(leader, bar(Tr::B_Q_EMPTY + i % QST));
-        // dQ_i = dS K  (A = dS from shared memory, queries contiguous; B = K, d contiguous)
-        if (i > 0 && !(ok = mbar_wait_warp(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree))) break;
-        tc_fence_after();
-        const uint32_t ds_s = sDS + (i & 1) * Tr::DS_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ss(leader, tmem + Tr::TM_DQ, sw128_desc(ds_s + kk * 16 * 128, BN * 128, 1024),
-                  sw128_desc(sK + kk * 16 * 128, BN * 128, 1024), kIdescDQ, kk > 0 ? 1u : 0u);
-        umma_commit(leader, bar(Tr::B_DQ_FULL));
-        umma_commit(leader, bar(Tr::B_DSBUF_FREE + (i & 1)));
-        // the next dP^T overwrites TM_DP after dK has read dS^T
+        // the next S^T (dP^T) overwrites TM_S (TM_DP) after dV (dK) has read
+        // P^T (dS^T): same issuing thread, so the tensor pipe keeps the order
         if (more) {
-          issue_dp(i + 1);
-          umma_commit(leader, bar(Tr::B_DP_FULL));
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                                    kBSiteQFull)))
+            break;
+          tc_fence_after();
+          issue_first(i + 1);
         }
       }
       umma_commit(leader, bar(Tr::B_KV_DONE));
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
     }
     __syncwarp();
-  }  // warps 10 and 11 have no role
+  }  // warp 11 has no role
   } else {
     regs_grow();  // both compute warpgroups
     // ----------------------------- compute warps 0-7: P^T, dS^T, dQ drain

@@ -249,6 +249,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The descriptor of the same layout starting `bytes` further on (bytes is a
+// multiple of 16; the start field cannot carry out: shared addresses fit it).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 // fmt: 0 = fp16, 1 = bf16 (same for A and B).  b_mn: B operand is MN-major.
 __host__ __device__ constexpr uint32_t f16_idesc(uint32_t fmt, int M, int N, bool b_mn) {

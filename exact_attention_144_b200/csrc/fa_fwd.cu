@@ -349,26 +349,27 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
       uint32_t kc = 0, vc = 0, g = 0, uc = 0;
       bool ok = true;
+      // Descriptors are built once; each MMA only advances a start address.
+      const uint64_t q_desc0 = sw128_desc(sQ, 16, 1024), k_desc0 = sw128_desc(sK, 16, 1024),
+                     v_desc0 = sw128_desc(sV, BN * 128, 1024);
       // S_t = Q_t K^T for the K stage of counter kc (t = 0, 1)
       auto issue_qk = [&](int t) {
-        const uint32_t kbase = sK + (kc % KST) * Tr::KV_BYTES;
-        const uint32_t qbase = sQ + t * Tr::QT_BYTES;
+        const uint64_t kd = desc_advance(k_desc0, (kc % KST) * Tr::KV_BYTES);
+        const uint64_t qd = desc_advance(q_desc0, t * Tr::QT_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(leader, tmem + t * BN, sw128_desc(qbase + ch * (BM * 128) + in, 16, 1024),
-                  sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(leader, tmem + t * BN, desc_advance(qd, ch * (BM * 128) + in),
+                  desc_advance(kd, ch * (BN * 128) + in), kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V for the V stage of counter vc
       auto issue_pv = [&](int t, bool first) {
-        const uint32_t vbase = sV + (vc % VST) * Tr::KV_BYTES;
+        const uint64_t vd = desc_advance(v_desc0, (vc % VST) * Tr::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
-                  sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
-                  (!first || kk > 0) ? 1u : 0u);
+                  desc_advance(vd, kk * 16 * 128), kIdescPV, (!first || kk > 0) ? 1u : 0u);
       };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, p);
@@ -628,6 +629,8 @@ __global__ void __launch_bounds__(224, 1)
       constexpr uint32_t kIdescPV = f16_idesc(Elem<T>::kFmt, 128, D, true);
       uint32_t kc = 0, vc = 0, g = 0, uc = 0;
       bool ok = true;
+      const uint64_t q_desc0 = sw128_desc(sQ, 16, 1024), k_desc0 = sw128_desc(sK, 16, 1024),
+                     v_desc0 = sw128_desc(sV, BN * 128, 1024);
       // O += P_j V_j for the tile whose S/P buffer use counter is gp.
       auto issue_pv = [&](uint32_t gp, bool first) -> bool {
         const uint32_t pb = gp & 1u;
@@ -635,12 +638,11 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t vs = vc % VST;
         if (!mbar_wait_warp(bar(Tr::B_V_FULL + vs), (vc / VST) & 1u, w, kSiteVFull)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + vs * Tr::KV_BYTES;
+        const uint64_t vd = desc_advance(v_desc0, vs * Tr::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
-                  sw128_desc(vbase + kk * 16 * 128, BN * 128, 1024), kIdescPV,
-                  (!first || kk > 0) ? 1u : 0u);
+          umma_ts(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8, desc_advance(vd, kk * 16 * 128),
+                  kIdescPV, (!first || kk > 0) ? 1u : 0u);
         umma_commit(leader, bar(Tr::B_V_EMPTY + vs));
         umma_commit(leader, bar(Tr::B_O_DONE));
         ++vc;
@@ -656,13 +658,12 @@ __global__ void __launch_bounds__(224, 1)
           if (!(ok = mbar_wait_warp(bar(Tr::B_K_FULL + ks), (kc / KST) & 1u, w, kSiteKFull))) break;
           tc_fence_after();
           const uint32_t sb = g & 1u;
-          const uint32_t kbase = sK + ks * Tr::KV_BYTES;
+          const uint64_t kd = desc_advance(k_desc0, ks * Tr::KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-            umma_ss(leader, tmem + sb * BN, sw128_desc(sQ + ch * (Tr::BM * 128) + in, 16, 1024),
-                    sw128_desc(kbase + ch * (BN * 128) + in, 16, 1024), kIdescQK,
-                    kk > 0 ? 1u : 0u);
+            umma_ss(leader, tmem + sb * BN, desc_advance(q_desc0, ch * (Tr::BM * 128) + in),
+                    desc_advance(kd, ch * (BN * 128) + in), kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(leader, bar(Tr::B_K_EMPTY + ks));
           umma_commit(leader, bar(Tr::B_S_FULL + sb));
