@@ -27,6 +27,17 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa_b200.h")
 _lib = None
 
 
+class FwdPlan(ctypes.Structure):
+    """fa_fwd_plan_t: how the forward decomposes a problem (see fa_fwd_plan)."""
+    _fields_ = [("kernel", ctypes.c_int), ("unit_rows", ctypes.c_int),
+                ("kv_tile_rows", ctypes.c_int), ("n_units", ctypes.c_int),
+                ("n_kv_tiles", ctypes.c_int), ("n_split", ctypes.c_int), ("grid", ctypes.c_int),
+                ("balanced", ctypes.c_int), ("scratch_bytes", ctypes.c_longlong)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
 def _load() -> ctypes.CDLL:
     """Load libfa_b200.so once; raise if it has not been built."""
     global _lib
@@ -56,6 +67,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_set_kernel_events.restype = i
     lib.fa_kernel_launches.restype = ctypes.c_ulonglong
     lib.fa_last_cuda_error.restype = i
+    lib.fa_fwd_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(FwdPlan)]
+    lib.fa_fwd_plan.restype = i
+    lib.fa_fwd_plan_pieces.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int), i]
+    lib.fa_fwd_plan_pieces.restype = i
     _lib = lib
     return lib
 
@@ -213,6 +228,31 @@ def backward(q, k, v, o, dout, lse, scale=None, dq=None, dk=None, dv=None, strea
     if q.dtype not in _BWD:
         raise TypeError(f"unsupported element type {q.dtype}")
     return _BWD[q.dtype](q, k, v, o, dout, lse, dq=dq, dk=dk, dv=dv, scale=scale, stream=stream)
+
+
+def fa_fwd_plan(B: int, H: int, N: int, d: int, sm_count: int) -> dict:
+    """The forward's work decomposition for a device with sm_count SMs (host
+    logic only; needs no GPU)."""
+    plan = FwdPlan()
+    rc = _load().fa_fwd_plan(B, H, N, d, sm_count, ctypes.byref(plan))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_plan", rc)
+    return plan.as_dict()
+
+
+def fa_fwd_plan_pieces(B: int, H: int, N: int, d: int, sm_count: int, block: int) -> list:
+    """The pieces one forward block processes, as (unit, first K/V tile, end
+    K/V tile, kind, first peer, peer count) tuples; kind 0 = whole result,
+    1 = partial rows, 2 = merge with the peers' partial rows."""
+    lib_ = _load()
+    n = lib_.fa_fwd_plan_pieces(B, H, N, d, sm_count, block, None, 0)
+    if n < 0:
+        raise FAError("fa_fwd_plan_pieces", n)
+    buf = (ctypes.c_int * (6 * max(n, 1)))()
+    got = lib_.fa_fwd_plan_pieces(B, H, N, d, sm_count, block, buf, n)
+    if got != n:
+        raise FAError("fa_fwd_plan_pieces", got if got < 0 else FA_ERR_SHAPE)
+    return [tuple(buf[6 * i:6 * i + 6]) for i in range(n)]
 
 
 def fa_get_device_status(clear: bool = False) -> int:

@@ -69,6 +69,50 @@ unsigned long long* device_status_ptr() {
   return cached[dev];
 }
 
+// ------------------------------------------------------------ scratch pool
+static cudaMemPool_t scratch_pool(int dev) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {nullptr};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (pools[dev] == nullptr) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    unsigned long long keep = kScratchRetainBytes;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+      cudaGetLastError();  // still usable, only without retention
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
+int scratch_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_NOMEM;
+  }
+  cudaMemPool_t pool = scratch_pool(dev);
+  if (pool == nullptr || cudaMallocFromPoolAsync(ptr, bytes, pool, stream) != cudaSuccess) {
+    cudaGetLastError();
+    *ptr = nullptr;
+    return FA_ERR_NOMEM;
+  }
+  return FA_OK;
+}
+
+void scratch_free(void* ptr, cudaStream_t stream) {
+  if (ptr != nullptr && cudaFreeAsync(ptr, stream) != cudaSuccess) cudaGetLastError();
+}
+
 // ------------------------------------------------------------ device info
 int current_device(DeviceInfo* info) {
   static std::mutex mu;
@@ -251,6 +295,33 @@ FA_EXPORT int fa_bwd_f16(const void* q, const void* k, const void* v, const void
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                float scale, cudaStream_t stream) {
   return fa::bwd_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, stream);
+}
+
+FA_EXPORT int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t* plan) {
+  if (plan == nullptr) return FA_ERR_NULL;
+  fa::FwdSchedule s;
+  const int rc = fa::plan_fwd(B, H, N, d, sm_count, &s);
+  if (rc != FA_OK) return rc;
+  plan->kernel = s.pair;
+  plan->unit_rows = s.unit_rows;
+  plan->kv_tile_rows = s.bn;
+  plan->n_units = s.n_units;
+  plan->n_kv_tiles = s.n_kvt;
+  plan->n_split = s.n_split;
+  plan->grid = s.grid;
+  plan->balanced = s.n_iter > 0 ? 1 : 0;
+  plan->scratch_bytes = (long long)fa::fwd_scratch_bytes(s);
+  return FA_OK;
+}
+
+FA_EXPORT int fa_fwd_plan_pieces(int B, int H, int N, int d, int sm_count, int block,
+                                 int* pieces, int max_pieces) {
+  if (pieces == nullptr && max_pieces > 0) return FA_ERR_NULL;
+  fa::FwdSchedule s;
+  const int rc = fa::plan_fwd(B, H, N, d, sm_count, &s);
+  if (rc != FA_OK) return rc;
+  if (block < 0 || block >= s.grid) return FA_ERR_SHAPE;
+  return fa::fwd_block_pieces(s, block, pieces, max_pieces < 0 ? 0 : max_pieces);
 }
 
 FA_EXPORT const char* fa_status_string(int status) {

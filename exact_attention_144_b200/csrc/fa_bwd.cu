@@ -553,10 +553,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
   const size_t rows = (size_t)B * H * Npad;
   void* ws = nullptr;
   const size_t ws_bytes = rows * D * sizeof(float) + 2 * rows * sizeof(float);
-  if (cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_NOMEM;
-  }
+  if ((rc = scratch_alloc(&ws, ws_bytes, stream)) != FA_OK) return rc;
   BwdParams p{};
   p.dq_acc = static_cast<float*>(ws);
   float* lse2 = p.dq_acc + rows * D;
@@ -577,7 +574,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
 
   CUtensorMap tmacc;
   if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::BM)) != FA_OK) {
-    cudaFreeAsync(ws, stream);
+    scratch_free(ws, stream);
     return rc;
   }
 
@@ -611,7 +608,7 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
     rc = launch_status(cudaGetLastError());
     note_launches(1);
   }
-  cudaFreeAsync(ws, stream);
+  scratch_free(ws, stream);
   return rc;
 }
 

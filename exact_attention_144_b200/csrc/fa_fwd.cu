@@ -39,39 +39,110 @@
 
 namespace fa {
 
-struct FwdParams {
+// How a unit's result leaves the block.
+enum : int {
+  kStoreWhole = 0,    // every K/V tile of the unit (or of its split-mode share)
+  kStorePartial = 1,  // K/V tiles [t0 > 0, t1): normalised fp32 rows + LSE to the block's slot
+  kStoreMerge = 2     // K/V tiles [0, t1 < n_kvt): merged with the partial rows of the
+                      // blocks peer0 .. peer0 + npeer - 1, then stored
+};
+
+struct Unit {
+  int u;  // unit index
+  int b, h, qt, sp, t0, t1;
+  int kind, peer0, npeer;
+};
+
+__host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+
+// First step of block c's range in the balanced schedule (c <= grid).
+__host__ __device__ __forceinline__ int range_begin(const FwdSchedule& s, int c) {
+  return c * s.iter_per + imin(c, s.iter_rem);
+}
+
+__host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s) {
+  Unit x;
+  x.u = u;
+  x.qt = u % s.n_qt;
+  int r = u / s.n_qt;
+  x.sp = r % s.n_split;
+  r /= s.n_split;
+  x.h = r % s.H;
+  x.b = r / s.H;
+  x.t0 = x.sp * s.kvt_per_split;
+  x.t1 = imin(x.t0 + s.kvt_per_split, s.n_kvt);
+  x.kind = kStoreWhole;
+  x.peer0 = x.npeer = 0;
+  return x;
+}
+
+// The units (or pieces of units) block `blk` processes, in order.  Every role
+// of the block walks its own copy and sees the same sequence.
+//   plain:    units blk, blk + grid, blk + 2 grid, ...
+//   balanced: the steps [range_begin(blk), range_begin(blk + 1)) cut at unit
+//             boundaries.  Only a block's first piece can start inside a unit
+//             (kStorePartial); the piece holding K/V tile 0 of a unit cut in
+//             pieces is its block's last piece and merges the others
+//             (kStoreMerge), whose blocks all come after it.
+struct UnitIter {
+  int i, end, blk;
+  __host__ __device__ __forceinline__ UnitIter(const FwdSchedule& s, int blk_) : blk(blk_) {
+    if (s.n_iter > 0) {
+      i = range_begin(s, blk);
+      end = range_begin(s, blk + 1);
+    } else {
+      i = blk;
+      end = s.n_units;
+    }
+  }
+  __host__ __device__ __forceinline__ bool next(const FwdSchedule& s, Unit& x) {
+    if (i >= end) return false;
+    if (s.n_iter == 0) {
+      x = decode_unit(i, s);
+      i += s.grid;
+      return true;
+    }
+    const int u = i / s.n_kvt;
+    const int ubeg = u * s.n_kvt, uend = ubeg + s.n_kvt;
+    x = decode_unit(u, s);  // n_split = 1: the whole K/V range
+    x.t0 = i - ubeg;
+    x.t1 = imin(end, uend) - ubeg;
+    if (x.t0 > 0) {
+      x.kind = kStorePartial;
+    } else if (x.t1 < s.n_kvt) {
+      x.kind = kStoreMerge;
+      x.peer0 = blk + 1;
+      int c = x.peer0;
+      while (c < s.grid && range_begin(s, c) < uend) ++c;
+      x.npeer = c - x.peer0;
+    }
+    i = imin(end, uend);
+    return true;
+  }
+};
+
+struct FwdParams : FwdSchedule {
   void* o;          // [B, N, H, D] 16-bit, direct mode
   float* lse;       // [B, H, N] natural log, direct mode
   float* o_part;    // [S, B, N, H, D] fp32, split mode (null in direct mode)
   float* lse_part;  // [S, B, H, N] base-2 log, split mode
-  int B, H, N;
-  int n_qt;         // Q units per (b, h): 128-row tiles (fa_fwd_kernel) or 256-row pairs
-  int n_kvt, n_split, kvt_per_split, n_units;
+  float* bal_o;     // balanced: [grid, unit_rows, D] fp32 partial rows, normalised
+  float* bal_lse;   // balanced: [grid, unit_rows] base-2 LSE of those rows
+  unsigned* bal_flag;  // balanced: [grid] warps that have stored their partial rows; zeroed
   float sl2;        // scale * log2(e)
   unsigned long long limit_ns;
   unsigned long long* status;
 };
 
-struct Unit {
-  int b, h, qt, sp, t0, t1;
-};
-
-__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
-  Unit x;
-  x.qt = u % p.n_qt;
-  int r = u / p.n_qt;
-  x.sp = r % p.n_split;
-  r /= p.n_split;
-  x.h = r % p.H;
-  x.b = r / p.H;
-  x.t0 = x.sp * p.kvt_per_split;
-  x.t1 = min(x.t0 + p.kvt_per_split, p.n_kvt);
-  return x;
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
 }
 
 // Timeout sites reported in the status word.
 enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull,
-       kSiteSFull, kSiteODone, kSiteEpi };
+       kSiteSFull, kSiteODone, kSiteEpi, kSitePeer };
 
 // Growth of the running max (base 2) tolerated before O is rescaled.
 constexpr float kRescaleThreshold = 8.0f;
@@ -162,12 +233,106 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
 
 // Epilogue for one row: O = O_acc / l (16-bit, or fp32 partial in split mode)
 // and the LSE (natural log, or base 2 in split mode).  Collective over the warp.
+// Balanced schedule: a kStorePartial piece stores its rows into the block's
+// slot; a kStoreMerge piece first waits (bounded) until every peer block's 8
+// softmax warps have stored theirs, then merges
+//   O = sum_x 2^(LSE_x - L) O_x,  L = log2 sum_x 2^LSE_x  (x = own + peers).
+// Returns false when a wait gave up.
 template <class T, int D>
-__device__ __forceinline__ void store_row(const FwdParams& p, const Unit& un, uint32_t taddr,
-                                          int q_row, float m, float l) {
+__device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, uint32_t taddr,
+                                          int q_row, float m, float l, const WaitCtl& w) {
   const bool live = q_row < p.N;
   const float inv_l = 1.f / l;
   const float lse2 = m + lg2(l);
+  if (un.kind == kStorePartial) {
+    const int ur = q_row - un.qt * p.unit_rows;
+    float* orow = p.bal_o + ((size_t)blockIdx.x * p.unit_rows + ur) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(taddr + c * 32, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      if (live) {
+        float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[j] = make_float4(__uint_as_float(o[4 * j]) * inv_l,
+                               __uint_as_float(o[4 * j + 1]) * inv_l,
+                               __uint_as_float(o[4 * j + 2]) * inv_l,
+                               __uint_as_float(o[4 * j + 3]) * inv_l);
+      }
+    }
+    if (live) p.bal_lse[(size_t)blockIdx.x * p.unit_rows + ur] = lse2;
+    __threadfence();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicAdd(p.bal_flag + blockIdx.x, 1u);
+    return true;
+  }
+  if (un.kind == kStoreMerge) {
+    const int ur = q_row - un.qt * p.unit_rows;
+    bool good = true;
+    for (int c = un.peer0; c < un.peer0 + un.npeer && good; ++c) {
+      const uint64_t t0 = global_ns();
+      for (uint32_t it = 1; ld_acquire_gpu(p.bal_flag + c) < 8u; ++it) {
+        if ((it & 63u) == 0) {
+          if (*w.abort) { good = false; break; }
+          if (global_ns() - t0 > w.limit_ns) {
+            report_timeout(w.status, kSitePeer);
+            *w.abort = 1;
+            good = false;
+            break;
+          }
+        }
+      }
+    }
+    if (!__all_sync(0xffffffffu, good)) return false;
+    float mx = lse2;
+    if (live)
+      for (int c = un.peer0; c < un.peer0 + un.npeer; ++c)
+        mx = fmaxf(mx, __ldcg(p.bal_lse + (size_t)c * p.unit_rows + ur));
+    float tot = ex2(lse2 - mx);
+    if (live)
+      for (int c = un.peer0; c < un.peer0 + un.npeer; ++c)
+        tot += ex2(__ldcg(p.bal_lse + (size_t)c * p.unit_rows + ur) - mx);
+    const float L2 = mx + lg2(tot);
+    const float w_own = ex2(lse2 - L2) * inv_l;
+    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(taddr + c * 32, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      float acc[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(o[j]) * w_own;
+      if (live) {
+        for (int pc = un.peer0; pc < un.peer0 + un.npeer; ++pc) {
+          const float wp = ex2(__ldcg(p.bal_lse + (size_t)pc * p.unit_rows + ur) - L2);
+          const float4* src = reinterpret_cast<const float4*>(
+              p.bal_o + ((size_t)pc * p.unit_rows + ur) * D + c * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 v = __ldcg(src + j);
+            acc[4 * j] = fmaf(wp, v.x, acc[4 * j]);
+            acc[4 * j + 1] = fmaf(wp, v.y, acc[4 * j + 1]);
+            acc[4 * j + 2] = fmaf(wp, v.z, acc[4 * j + 2]);
+            acc[4 * j + 3] = fmaf(wp, v.w, acc[4 * j + 3]);
+          }
+        }
+        uint4 pkd[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pw[j] = Elem<T>::pack(acc[2 * j], acc[2 * j + 1]);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
+      }
+    }
+    if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = L2 * kLn2;
+    return true;
+  }
   if (p.o_part == nullptr) {
     T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
 #pragma unroll
@@ -209,6 +374,7 @@ __device__ __forceinline__ void store_row(const FwdParams& p, const Unit& un, ui
     }
     if (live) p.lse_part[(((size_t)un.sp * p.B + un.b) * p.H + un.h) * p.N + q_row] = lse2;
   }
+  return true;
 }
 
 // ===========================================================================
@@ -299,8 +465,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, vc = 0, qc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, p);
+      UnitIter it(p, blockIdx.x);
+      for (Unit un; ok && it.next(p, un);) {
         if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
         mbar_expect_tx(leader, bar(Tr::B_Q_FULL), 2 * Tr::QT_BYTES);
 #pragma unroll
@@ -371,8 +537,8 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
                   desc_advance(vd, kk * 16 * 128), kIdescPV, (!first || kk > 0) ? 1u : 0u);
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, p);
+      UnitIter it(p, blockIdx.x);
+      for (Unit un; ok && it.next(p, un);) {
         const int n = un.t1 - un.t0;
         if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
         if (!(ok = mbar_wait_warp(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))) break;
@@ -435,8 +601,8 @@ __global__ void __launch_bounds__(384, 1)
     const float c = p.sl2;
     uint32_t g = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit un = decode_unit(u, p);
+    UnitIter it(p, blockIdx.x);
+    for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
       for (int j = 0; j < n; ++j, ++g) {
@@ -469,7 +635,7 @@ __global__ void __launch_bounds__(384, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      store_row<T, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l);
+      ok = store_row<T, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l, w);
     }
   }
 
@@ -568,8 +734,8 @@ __global__ void __launch_bounds__(224, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, qc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, p);
+      UnitIter it(p, blockIdx.x);
+      for (Unit un; ok && it.next(p, un);) {
         if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
         mbar_expect_tx(leader, bar(Tr::B_Q_FULL), Tr::Q_BYTES);
 #pragma unroll
@@ -602,8 +768,8 @@ __global__ void __launch_bounds__(224, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t vc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, p);
+      UnitIter it(p, blockIdx.x);
+      for (Unit un; ok && it.next(p, un);) {
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t vs = vc % VST;
           if (vc >= (uint32_t)VST &&
@@ -648,8 +814,8 @@ __global__ void __launch_bounds__(224, 1)
         ++vc;
         return true;
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, p);
+      UnitIter it(p, blockIdx.x);
+      for (Unit un; ok && it.next(p, un);) {
         if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
         tc_fence_after();
         const int n = un.t1 - un.t0;
@@ -688,8 +854,8 @@ __global__ void __launch_bounds__(224, 1)
     const float c = p.sl2;
     uint32_t g = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit un = decode_unit(u, p);
+    UnitIter it(p, blockIdx.x);
+    for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
       for (int i = 0; i < n; ++i, ++g) {
@@ -724,7 +890,7 @@ __global__ void __launch_bounds__(224, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      store_row<T, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l);
+      ok = store_row<T, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l, w);
     }
   }
 
@@ -781,94 +947,177 @@ static int choose_splits(long long base_units, int n_kvt, int sm_count) {
   int n_split = 1;
   if (base_units * 2 <= sm_count) {
     n_split = (int)(sm_count / base_units);
-    n_split = min(n_split, n_kvt / 8);
-    n_split = max(n_split, 1);
+    n_split = n_split < n_kvt / 8 ? n_split : n_kvt / 8;
+    n_split = n_split > 1 ? n_split : 1;
   }
   return n_split;
 }
 
-template <class T, int D, int BM_UNIT, int BN, int THREADS, int SMEM, bool SPLIT_REGS,
-          class Kernel>
-static int launch_fwd(Kernel kern, const void* q, const void* k, const void* v, void* o,
-                      float* lse, int B, int H, int N, float scale, cudaStream_t stream,
-                      const DeviceInfo& dev) {
+// Balanced schedule: when whole units would leave the last wave of blocks
+// partly idle (waves = ceil(units / SMs), efficiency = units / (waves * SMs)),
+// give every SM the same number of (unit, K/V tile) steps instead.  Units are
+// then cut into pieces across neighbouring blocks and merged in the kernel,
+// so it is kept for units long enough (>= 16 K/V tiles) that the extra
+// Q loads and merges stay small, and for at least 4 steps a block.
+static bool use_balanced(long long units, int n_kvt, int sm_count) {
+  if (n_kvt < 16 || units * n_kvt < 4ll * sm_count || units * n_kvt >= (1ll << 31)) return false;
+  const long long waves = (units + sm_count - 1) / sm_count;
+  return (double)units / (double)(waves * sm_count) < 0.95;
+}
+
+int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s) {
+  if (B < 1 || H < 1 || N < 1 || sm_count < 1) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
+  FwdSchedule x{};
+  x.B = B;
+  x.H = H;
+  x.N = N;
+  x.d = d;
+  // Two Q tiles per unit once a head has more than one tile's worth of rows;
+  // a single tile per unit for short sequences and for d = 256 (whose O
+  // accumulator leaves tensor memory room for only one Q tile).
+  x.pair = (N > 128 && d <= 128) ? 1 : 0;
+  x.unit_rows = x.pair ? 256 : 128;
+  x.bn = d == 256 ? 64 : 128;
+  x.n_qt = (N + x.unit_rows - 1) / x.unit_rows;
+  x.n_kvt = (N + x.bn - 1) / x.bn;
+  const long long base_units = (long long)B * H * x.n_qt;
+  if (base_units >= (1ll << 31)) return FA_ERR_SHAPE;
+  int n_split = choose_splits(base_units, x.n_kvt, sm_count);
+  x.kvt_per_split = (x.n_kvt + n_split - 1) / n_split;
+  x.n_split = (x.n_kvt + x.kvt_per_split - 1) / x.kvt_per_split;  // no empty split
+  x.n_units = (int)(base_units * x.n_split);
+  const bool balanced =
+      x.pair && x.n_split == 1 && use_balanced(base_units, x.n_kvt, sm_count);
+  x.grid = balanced ? sm_count : (x.n_units < sm_count ? x.n_units : sm_count);
+  if (balanced) {
+    x.n_iter = (int)(base_units * x.n_kvt);
+    x.iter_per = x.n_iter / x.grid;
+    x.iter_rem = x.n_iter % x.grid;
+  }
+  *s = x;
+  return FA_OK;
+}
+
+size_t fwd_scratch_bytes(const FwdSchedule& s) {
+  if (s.n_split > 1)
+    return ((size_t)s.n_split * s.B * s.N * s.H * s.d + (size_t)s.n_split * s.B * s.H * s.N) *
+           sizeof(float);
+  if (s.n_iter > 0)  // one partial slot per block: rows x d fp32, rows LSE, a flag
+    return ((size_t)s.grid * s.unit_rows * s.d + (size_t)s.grid * s.unit_rows + s.grid) *
+           sizeof(float);
+  return 0;
+}
+
+int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces) {
+  UnitIter it(s, blk);
+  int n = 0;
+  for (Unit x; it.next(s, x); ++n) {
+    if (n < max_pieces) {
+      int* o = out + 6 * n;
+      o[0] = x.u;
+      o[1] = x.t0;
+      o[2] = x.t1;
+      o[3] = x.kind;
+      o[4] = x.peer0;
+      o[5] = x.npeer;
+    }
+  }
+  return n;
+}
+
+template <class T, int D, int BN, int THREADS, int SMEM, bool SPLIT_REGS, class Kernel>
+static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const void* k,
+                      const void* v, void* o, float* lse, float scale, cudaStream_t stream) {
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, 128)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, s.B, s.N, s.H, D, 128)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, s.B, s.N, s.H, D, BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, s.B, s.N, s.H, D, BN)) != FA_OK) return rc;
 
   FwdParams p{};
+  static_cast<FwdSchedule&>(p) = s;
   p.o = o;
   p.lse = lse;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.n_qt = (N + BM_UNIT - 1) / BM_UNIT;
-  p.n_kvt = (N + BN - 1) / BN;
   p.sl2 = scale * kLog2e;
   p.limit_ns = 4000000000ull;
   p.status = device_status_ptr();
-  const long long base_units = (long long)B * H * p.n_qt;
-  int n_split = choose_splits(base_units, p.n_kvt, dev.sm_count);
-  p.kvt_per_split = (p.n_kvt + n_split - 1) / n_split;
-  n_split = (p.n_kvt + p.kvt_per_split - 1) / p.kvt_per_split;  // no empty split
-  p.n_split = n_split;
-  p.n_units = (int)(base_units * n_split);
 
   void* ws = nullptr;
-  if (n_split > 1) {
-    const size_t o_elems = (size_t)n_split * B * N * H * D;
-    const size_t l_elems = (size_t)n_split * B * H * N;
-    if (cudaMallocAsync(&ws, (o_elems + l_elems) * sizeof(float), stream) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_NOMEM;
-    }
+  const size_t ws_bytes = fwd_scratch_bytes(s);
+  if (ws_bytes > 0 && (rc = scratch_alloc(&ws, ws_bytes, stream)) != FA_OK) return rc;
+  if (s.n_split > 1) {
     p.o_part = static_cast<float*>(ws);
-    p.lse_part = p.o_part + o_elems;
+    p.lse_part = p.o_part + (size_t)s.n_split * s.B * s.N * s.H * D;
+  } else if (s.n_iter > 0) {
+    p.bal_o = static_cast<float*>(ws);
+    p.bal_lse = p.bal_o + (size_t)s.grid * s.unit_rows * D;
+    p.bal_flag = reinterpret_cast<unsigned*>(p.bal_lse + (size_t)s.grid * s.unit_rows);
+    if (cudaMemsetAsync(p.bal_flag, 0, s.grid * sizeof(unsigned), stream) != cudaSuccess) {
+      rc = launch_status(cudaGetLastError());
+      scratch_free(ws, stream);
+      return rc;
+    }
   }
   if (SPLIT_REGS && (rc = check_launch_regs((const void*)kern)) != FA_OK) {
-    if (ws) cudaFreeAsync(ws, stream);
+    scratch_free(ws, stream);
     return rc;
   }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
     rc = launch_status(cudaGetLastError());
-    if (ws) cudaFreeAsync(ws, stream);
+    scratch_free(ws, stream);
     return rc;
   }
-  const int grid = p.n_units < dev.sm_count ? p.n_units : dev.sm_count;
   cudaEvent_t ev0, ev1;
   take_kernel_events(false, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  kern<<<grid, THREADS, SMEM, stream>>>(tmq, tmk, tmv, p);
-  rc = launch_status(cudaGetLastError());
+  if (s.n_iter > 0) {
+    // A merging block waits for its neighbours' partial rows, so all blocks
+    // must be resident at once: a cooperative launch guarantees it (or fails).
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(s.grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    rc = launch_status(cudaLaunchKernelEx(&cfg, kern, tmq, tmk, tmv, p));
+  } else {
+    kern<<<s.grid, THREADS, SMEM, stream>>>(tmq, tmk, tmv, p);
+    rc = launch_status(cudaGetLastError());
+  }
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);
-  if (rc == FA_OK && n_split > 1) {
-    const long long rows = (long long)B * N * H;
+  if (rc == FA_OK && s.n_split > 1) {
+    const long long rows = (long long)s.B * s.N * s.H;
     fa_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-        p.o_part, p.lse_part, static_cast<T*>(o), lse, B, H, N, n_split);
+        p.o_part, p.lse_part, static_cast<T*>(o), lse, s.B, s.H, s.N, s.n_split);
     rc = launch_status(cudaGetLastError());
     note_launches(1);
   }
-  if (ws) cudaFreeAsync(ws, stream);
+  scratch_free(ws, stream);
   return rc;
 }
 
 template <class T, class Tr>
-static int run_single(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                      int H, int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
-  return launch_fwd<T, Tr::D, 128, Tr::BN, 224, Tr::SMEM_BYTES, false>(
-      fa_fwd_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
+static int run_single(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
+                      float* lse, float scale, cudaStream_t stream) {
+  static_assert(Tr::BM == 128, "unit rows");
+  return launch_fwd<T, Tr::D, Tr::BN, 224, Tr::SMEM_BYTES, false>(fa_fwd_kernel<T, Tr>, s, q, k,
+                                                                   v, o, lse, scale, stream);
 }
 
 template <class T, class Tr>
-static int run_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                  int N, float scale, cudaStream_t stream, const DeviceInfo& dev) {
-  return launch_fwd<T, Tr::D, 256, Tr::BN, 384, Tr::SMEM_BYTES, true>(
-      fa_fwd_pp_kernel<T, Tr>, q, k, v, o, lse, B, H, N, scale, stream, dev);
+static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
+                  float* lse, float scale, cudaStream_t stream) {
+  static_assert(2 * Tr::BM == 256, "unit rows");
+  return launch_fwd<T, Tr::D, Tr::BN, 384, Tr::SMEM_BYTES, true>(fa_fwd_pp_kernel<T, Tr>, s, q, k,
+                                                                 v, o, lse, scale, stream);
 }
 
 template <class T>
@@ -877,23 +1126,17 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
-  // Two Q tiles per unit once a head has more than one tile's worth of rows;
-  // a single tile per unit for short sequences and for d = 256 (whose O
-  // accumulator leaves tensor memory room for only one Q tile).
-  const bool pair = N > 128;
+  FwdSchedule s;
+  if ((rc = plan_fwd(B, H, N, d, dev.sm_count, &s)) != FA_OK) return rc;
   switch (d) {
     case 64:
-      return pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(q, k, v, o, lse, B, H, N, scale, stream, dev)
-                  : run_single<T, FwdTraits<64, 128, 4, 4>>(q, k, v, o, lse, B, H, N, scale,
-                                                             stream, dev);
+      return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, stream)
+                    : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale, stream);
     case 128:
-      return pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream,
-                                                      dev)
-                  : run_single<T, FwdTraits<128, 128, 3, 2>>(q, k, v, o, lse, B, H, N, scale,
-                                                              stream, dev);
+      return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, stream)
+                    : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale, stream);
     case 256:
-      return run_single<T, FwdTraits<256, 64, 2, 2>>(q, k, v, o, lse, B, H, N, scale, stream,
-                                                     dev);
+      return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, stream);
     default:
       return FA_ERR_HEADDIM;
   }

@@ -35,6 +35,15 @@ void note_launches(unsigned n);
 // or backward (bwd=true) main kernel; both are null when none is armed.
 void take_kernel_events(bool bwd, cudaEvent_t* start, cudaEvent_t* stop);
 
+// Stream-ordered scratch from this library's own memory pool on the current
+// device (created on first use).  The pool keeps up to kScratchRetainBytes of
+// freed scratch mapped across synchronisations, so repeated calls do not map
+// and unmap device memory each time (the default pool releases everything at
+// every synchronisation).  FA_OK or FA_ERR_NOMEM.
+constexpr unsigned long long kScratchRetainBytes = 1ull << 30;
+int scratch_alloc(void** ptr, size_t bytes, cudaStream_t stream);
+void scratch_free(void* ptr, cudaStream_t stream);
+
 // Device address of this library's status word on the current device.
 unsigned long long* device_status_ptr();
 
@@ -53,6 +62,39 @@ int make_tmap_f32_rows(CUtensorMap* map, const void* base, size_t rows, int cols
 int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale);
+
+// Work decomposition of one forward call (fa_fwd.cu).  A unit is unit_rows
+// query rows of one (batch, head), possibly limited to one share of the K/V
+// tiles (split mode); blocks walk units round-robin, or in the balanced
+// schedule each block takes a contiguous range of (unit, K/V tile) steps.
+struct FwdSchedule {
+  int B, H, N, d;
+  int pair;           // 1: fa_fwd_pp_kernel (two 128-row Q tiles a unit), 0: fa_fwd_kernel
+  int unit_rows;      // 256 (pair) or 128
+  int bn;             // K/V tile rows
+  int n_qt;           // units per (b, h) along the queries
+  int n_kvt;          // K/V tiles per head
+  int n_split;        // K/V shares per unit (> 1: partials merged by fa_combine_kernel)
+  int kvt_per_split;
+  int n_units;        // B * H * n_qt * n_split
+  int grid;           // blocks launched (at most one per SM)
+  int n_iter;         // balanced: n_units * n_kvt steps (0 = round-robin schedule)
+  int iter_per, iter_rem;  // balanced: block c takes iter_per (+1 if c < iter_rem) steps
+};
+
+// Fills *s for a forward call on a device with sm_count SMs (pure host logic).
+// FA_OK, or FA_ERR_SHAPE / FA_ERR_HEADDIM for shapes the forward rejects.
+int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s);
+
+// Scratch bytes the forward needs for schedule s (split partials, or the
+// balanced schedule's partial-row slots and flags).
+size_t fwd_scratch_bytes(const FwdSchedule& s);
+
+// The pieces block `blk` of schedule s processes, in order: for each, the
+// unit index, first and end K/V tile, store kind (0 whole, 1 partial,
+// 2 merge), first peer block and peer count, written as 6 ints to out.
+// Returns the number of pieces (writes at most max_pieces).
+int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 
 // Launchers (argument validation is done by the callers in fa_api.cu).
 template <class T>

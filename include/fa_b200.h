@@ -30,7 +30,11 @@
  *   fa_fwd writes o and lse; fa_bwd overwrites dq, dk, dv (it does not
  *   accumulate into them).  Scratch memory (split-K/V partial results, the
  *   fp32 dQ accumulator, the rowsum term) is allocated and released by the
- *   library, stream-ordered (cudaMallocAsync / cudaFreeAsync) on `stream`.
+ *   library, stream-ordered on `stream`, from a memory pool the library
+ *   creates per device (cudaMemPoolCreate, cudaMallocFromPoolAsync,
+ *   cudaFreeAsync).  The pool keeps up to 1 GiB of freed scratch mapped
+ *   between calls, so that a call after a synchronisation does not map new
+ *   device memory; the caller's default memory pool is not touched.
  *
  * Errors and execution
  *   Every call validates its arguments before any launch and returns FA_OK
@@ -96,8 +100,8 @@ int fa_bwd_f16(const void *q, const void *k, const void *v, const void *o,
  * such as plugin runtimes with their own static memory plan, code that runs
  * where allocation is forbidden or unsafe, and callers that must not touch
  * the device allocator at all.  fa_bwd needs scratch memory (an fp32 dQ
- * accumulator plus two fp32 vectors per query row) and takes it from
- * cudaMallocAsync; this variant computes the same result with the same
+ * accumulator plus two fp32 vectors per query row) and takes it from a
+ * stream-ordered memory pool; this variant computes the same result with the same
  * kernels but takes the scratch from one fixed buffer compiled into the
  * library, so it calls no cudaMalloc, cudaFree or other allocating routine.
  *
@@ -118,6 +122,46 @@ int fa_bwd_f16(const void *q, const void *k, const void *v, const void *o,
 int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                    const void *dout, const float *lse, void *dq, void *dk, void *dv,
                    int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/*
+ * Forward work decomposition (host logic only: no GPU, no CUDA call).
+ * Describes how fa_fwd / fa_fwd_f16 split a [B,N,H,d] problem over a device
+ * with sm_count SMs, for tests and tuning.  A unit is unit_rows query rows of
+ * one (batch, head); with n_split > 1 each unit covers one share of the K/V
+ * tiles and a second kernel merges the shares' partial results (exactly, by
+ * their log-sum-exps); with balanced = 1 every block takes an equal,
+ * contiguous range of (unit, K/V tile) steps, so units are cut into pieces
+ * whose partial results the block holding K/V tile 0 merges.
+ */
+typedef struct fa_fwd_plan {
+    int kernel;          /* 1: two 128-row Q tiles a unit, 0: one tile a unit   */
+    int unit_rows;       /* query rows per unit (256 or 128)                    */
+    int kv_tile_rows;    /* rows per K/V tile (128, or 64 at d = 256)           */
+    int n_units;         /* B * H * ceil(N / unit_rows) * n_split               */
+    int n_kv_tiles;      /* ceil(N / kv_tile_rows)                              */
+    int n_split;         /* K/V shares per unit                                 */
+    int grid;            /* blocks launched (at most sm_count)                  */
+    int balanced;        /* 1: balanced step ranges (cooperative launch)        */
+    long long scratch_bytes; /* device scratch the call allocates               */
+} fa_fwd_plan_t;
+
+/*
+ * Fills *plan.  Returns FA_OK, FA_ERR_NULL, FA_ERR_SHAPE (B, H, N or
+ * sm_count below 1) or FA_ERR_HEADDIM.
+ */
+int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t *plan);
+
+/*
+ * The pieces block `block` (0 <= block < plan.grid) processes, in order,
+ * 6 ints each: unit index, first K/V tile, end K/V tile, store kind
+ * (0: whole result, 1: partial rows to the block's slot, 2: merge with the
+ * partial rows of blocks first_peer .. first_peer + n_peers - 1), first_peer,
+ * n_peers.  Writes at most max_pieces pieces and returns the number the block
+ * has (>= 0), or a negative FA_ERR_* code.  The same code decides the pieces
+ * inside the kernel.
+ */
+int fa_fwd_plan_pieces(int B, int H, int N, int d, int sm_count, int block, int *pieces,
+                       int max_pieces);
 
 /* Static description of a status code.  Never NULL. */
 const char *fa_status_string(int status);

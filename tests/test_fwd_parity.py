@@ -72,6 +72,17 @@ def test_split_kv_path(fa):
     check_full(fa, 1, 1900, 1, 256, "bf16", 303)
 
 
+@pytest.mark.parametrize("B,N,H,d,dtype", [(1, 2000, 10, 64, "bf16"), (1, 2000, 10, 128, "fp16"),
+                                             (1, 4096, 5, 64, "bf16")])
+def test_balanced_schedule(fa, B, N, H, d, dtype):
+    # 80 units of 256 query rows on 148 SMs: every block takes an equal range
+    # of (unit, K/V tile) steps, so units are cut in two or three pieces on
+    # neighbouring blocks and merged in the kernel by their log-sum-exps
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert fa.fa_fwd_plan(B, H, N, d, sms)["balanced"] == 1
+    check_full(fa, B, N, H, d, dtype, 310 + d + N)
+
+
 def test_workload_c1_tiny(fa):
     w = attn_inputs.WORKLOADS["c1"]
     check_full(fa, w.B, w.N, w.H, w.d, w.dtype, w.seed)
