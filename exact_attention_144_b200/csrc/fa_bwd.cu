@@ -69,6 +69,7 @@ struct BwdTraits64 {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
   static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int ACC_BOX_ROWS = BM;  // dQ reduce box: 32 d columns x 128 queries
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -473,6 +474,405 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
+// ===========================================================================
+// fa_bwd_tq_kernel: d = 128.  At 128 queries per inner tile the five
+// accumulators (S^T, dP^T, dQ, dV, dK: 5 x 128 columns) exceed tensor memory,
+// so the inner tile holds 64 queries and dQ is produced transposed,
+//   dQ_i^T = K^T dS_i^T   (M = d = 128 lanes, N = 64 queries, K = 128 keys),
+// into one of two 64-column buffers; the compute warps drain it through a
+// per-warp staging box (32 queries x 32 d, fp32) that the warp reduce-adds
+// into the accumulator itself.
+// Tensor memory: S^T [0,64), dP^T [64,128), dQ^T [128,256) (two buffers),
+// dV [256,384), dK [384,512).  Warps as in fa_bwd_kernel; compute warp w owns
+// lane quadrant w % 4 and query half w / 4 (32 columns) of S^T and dP^T, and
+// d quadrant w % 4, query half w / 4 of dQ^T.
+// The single dS^T staging tile needs no release barrier: the compute warps
+// rewrite it for tile i only after dP^T_i has completed, and dP^T_i is
+// committed after the dQ MMA of tile i - 1 (its last reader) by the same
+// thread, so that commit also covers the read.
+// ===========================================================================
+template <int D_, int QST_>
+struct BwdTqTraits {
+  static constexpr int D = D_;
+  static constexpr int BN = 128;  // keys per block
+  static constexpr int BM = 64;   // queries per inner tile
+  static constexpr int QST = QST_;
+  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int QT_BYTES = BM * D * 2;
+  static constexpr int DS_BYTES = BN * BM * 2;       // dS^T tile: keys x 64 queries, 16-bit
+  static constexpr int BOX_BYTES = 32 * 32 * 4;      // a warp's dQ staging box
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + QST * QT_BYTES;
+  static constexpr int OFF_DS = OFF_DO + QST * QT_BYTES;
+  static constexpr int OFF_STG = OFF_DS + DS_BYTES;
+  static constexpr int OFF_L = OFF_STG + 8 * BOX_BYTES;  // base-2 LSE per stage
+  static constexpr int OFF_DD = OFF_L + QST * BM * 4;    // D per stage
+  static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
+  static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
+                       B_S_FULL = B_Q_EMPTY + QST, B_DP_FULL = B_S_FULL + 1,
+                       B_P_READY = B_DP_FULL + 1, B_DS_READY = B_P_READY + 1,
+                       B_DQ_FULL = B_DS_READY + 1, B_DQ_FREE = B_DQ_FULL + 2,
+                       B_KV_DONE = B_DQ_FREE + 2, B_DRAIN = B_KV_DONE + 1, NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries
+  static_assert(D == 128, "the transposed-dQ layout is laid out for d = 128");
+  static_assert(TM_DK + D <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0 && OFF_DS % 1024 == 0 &&
+                    OFF_STG % 1024 == 0 && QT_BYTES % 1024 == 0,
+                "swizzled tiles start on 1024-byte boundaries");
+};
+
+using BwdTq128 = BwdTqTraits<128, 3>;
+
+template <class T, class Tr>
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_tq_kernel(const __grid_constant__ CUtensorMap tmq,
+                     const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv,
+                     const __grid_constant__ CUtensorMap tmdo,
+                     const __grid_constant__ CUtensorMap tmacc, const BwdParams p) {
+  constexpr int D = Tr::D, BN = Tr::BN, BM = Tr::BM, QST = Tr::QST, KCH = Tr::KCH;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + Tr::OFF_K, sV = base + Tr::OFF_V, sQ = base + Tr::OFF_Q,
+                 sDO = base + Tr::OFF_DO, sDS = base + Tr::OFF_DS, sSTG = base + Tr::OFF_STG;
+  const float* sL = reinterpret_cast<const float*>(gbase + Tr::OFF_L);
+  const float* sDD = reinterpret_cast<const float*>(gbase + Tr::OFF_DD);
+  uint8_t* gDS = gbase + Tr::OFF_DS;
+  uint8_t* gSTG = gbase + Tr::OFF_STG;
+  const uint32_t bars = base + Tr::OFF_BAR;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + Tr::OFF_MISC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + Tr::OFF_MISC + 4);
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtl w{abort_flag, p.limit_ns, p.status};
+  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n_qt = p.n_qt;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(Tr::B_KV_FULL), 1);
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(bar(Tr::B_Q_FULL + s), 1);
+      mbar_init(bar(Tr::B_Q_EMPTY + s), 2);  // one commit from each MMA warp
+    }
+    mbar_init(bar(Tr::B_S_FULL), 1);
+    mbar_init(bar(Tr::B_DP_FULL), 1);
+    mbar_init(bar(Tr::B_P_READY), 256);
+    mbar_init(bar(Tr::B_DS_READY), 256);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Tr::B_DQ_FULL + s), 1);
+      mbar_init(bar(Tr::B_DQ_FREE + s), 256);
+    }
+    mbar_init(bar(Tr::B_KV_DONE), 2);
+    mbar_init(bar(Tr::B_DRAIN), 2);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), Tr::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+    tma_prefetch_desc(&tmdo);
+    tma_prefetch_desc(&tmacc);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp >= 8) {
+    regs_shrink();  // all four warps of the producer/MMA warpgroup
+  if (warp == 8) {
+    // -------------------------------------------------------- producer
+    {
+      const bool leader = lane == 0;  // issues; all lanes run the loop
+      mbar_expect_tx(leader, bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < KCH; ++c) {
+        tma_load_4d(leader, sK + c * (BN * 128), &tmk, bar(Tr::B_KV_FULL), c * 64, h, kt * BN, b);
+        tma_load_4d(leader, sV + c * (BN * 128), &tmv, bar(Tr::B_KV_FULL), c * 64, h, kt * BN, b);
+      }
+      const size_t row0 = ((size_t)b * p.H + h) * p.Npad;
+      int issued = 0;
+      for (int i = 0; i < n_qt; ++i) {
+        const int qs = i % QST;
+        if (i >= QST &&
+            !mbar_wait_warp(bar(Tr::B_Q_EMPTY + qs), ((i / QST) - 1) & 1, w, kBSiteQEmpty))
+          break;
+        const uint32_t fb = bar(Tr::B_Q_FULL + qs);
+        mbar_expect_tx(leader, fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
+#pragma unroll
+        for (int c = 0; c < KCH; ++c) {
+          tma_load_4d(leader, sQ + qs * Tr::QT_BYTES + c * (BM * 128), &tmq, fb, c * 64, h, i * BM, b);
+          tma_load_4d(leader, sDO + qs * Tr::QT_BYTES + c * (BM * 128), &tmdo, fb, c * 64, h, i * BM,
+                      b);
+        }
+        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
+        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
+        ++issued;
+      }
+      mbar_drain(bar(Tr::B_KV_FULL), 0, p.limit_ns);
+      for (int s = 0; s < QST; ++s)
+        if (issued > s) mbar_drain(bar(Tr::B_Q_FULL + s), ((issued - 1 - s) / QST) & 1, p.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------ MMA issuers
+    //   warp 9:  S^T = K Q_i^T and dV += P^T dO_i         (TMEM S^T, dV)
+    //   warp 10: dP^T = V dO_i^T, dK += dS^T Q_i, dQ_i^T  (TMEM dP^T, dK, dQ^T)
+    {
+      const bool stream_a = warp == 9;
+      const bool leader = lane == 0;  // issues; all lanes run the loop
+      constexpr uint32_t fmt = Elem<T>::kFmt;
+      constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);              // K-major x K-major
+      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);               // TS, B MN-major
+      constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, BM, true) | (1u << 15);  // A, B MN-major
+      // Packed 16-bit P^T / dS^T: query half hf sits in the first 16 columns of
+      // its own 32-column half of the S^T / dP^T region.
+      auto packed_col = [](int kk) -> uint32_t { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); };
+      const uint64_t k_kmaj = sw128_desc(sK, 16, 1024), v_kmaj = sw128_desc(sV, 16, 1024),
+                     q_kmaj = sw128_desc(sQ, 16, 1024), do_kmaj = sw128_desc(sDO, 16, 1024),
+                     q_mn = sw128_desc(sQ, BM * 128, 1024), do_mn = sw128_desc(sDO, BM * 128, 1024),
+                     k_mn = sw128_desc(sK, BN * 128, 1024), ds_mn = sw128_desc(sDS, BN * 128, 1024);
+      // S^T = K Q_i^T into TM_S (stream a); dP^T = V dO_i^T into TM_DP (stream b)
+      auto issue_first = [&](int i) {
+        const uint64_t a0 = stream_a ? k_kmaj : v_kmaj;
+        const uint64_t b0 = desc_advance(stream_a ? q_kmaj : do_kmaj, (i % QST) * Tr::QT_BYTES);
+        const uint32_t d_tmem = tmem + (stream_a ? Tr::TM_S : Tr::TM_DP);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
+          umma_ss(leader, d_tmem, desc_advance(a0, ch * (BN * 128) + in),
+                  desc_advance(b0, ch * (BM * 128) + in), kIdescSP, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(leader, bar(stream_a ? Tr::B_S_FULL : Tr::B_DP_FULL));
+      };
+      bool ok = mbar_wait_warp(bar(Tr::B_KV_FULL), 0, w, kBSiteKV);
+      if (ok && n_qt > 0 && (ok = mbar_wait_warp(bar(Tr::B_Q_FULL), 0, w, kBSiteQFull))) {
+        tc_fence_after();
+        issue_first(0);
+      }
+      for (int i = 0; i < n_qt && ok; ++i) {
+        const bool more = i + 1 < n_qt;
+        const int qs = i % QST;
+        if (stream_a) {
+          // dV += P^T dO_i  (A = P^T from TMEM, B = dO_i: queries x d, MN-major)
+          if (!(ok = mbar_wait_warp(bar(Tr::B_P_READY), i & 1, w, kBSitePReady))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(leader, tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
+                    desc_advance(do_mn, qs * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_Q_EMPTY + qs));
+        } else {
+          // dK += dS^T Q_i  (A = dS^T from TMEM, B = Q_i MN-major)
+          if (!(ok = mbar_wait_warp(bar(Tr::B_DS_READY), i & 1, w, kBSiteDsReady))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(leader, tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
+                    desc_advance(q_mn, qs * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_Q_EMPTY + qs));
+          // dQ_i^T = K^T dS_i^T  (A = K: d contiguous, MN-major; B = dS^T: queries
+          // contiguous, MN-major) into buffer i & 1, once its previous tile is drained
+          const int qb = i & 1;
+          if (i >= 2 &&
+              !(ok = mbar_wait_warp(bar(Tr::B_DQ_FREE + qb), ((i >> 1) - 1) & 1, w, kBSiteDqFree)))
+            break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ss(leader, tmem + Tr::TM_DQ + qb * BM, desc_advance(k_mn, kk * 16 * 128),
+                    desc_advance(ds_mn, kk * 16 * 128), kIdescDQ, kk > 0 ? 1u : 0u);
+          umma_commit(leader, bar(Tr::B_DQ_FULL + qb));
+        }
+        if (more) {
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                                    kBSiteQFull)))
+            break;
+          tc_fence_after();
+          issue_first(i + 1);
+        }
+      }
+      umma_commit(leader, bar(Tr::B_KV_DONE));
+      umma_commit(leader, bar(Tr::B_DRAIN));
+      mbar_drain(bar(Tr::B_DRAIN), 0, p.limit_ns);
+    }
+    __syncwarp();
+  }  // warp 11 has no role
+  } else {
+    regs_grow();  // both compute warpgroups
+    // ----------------------------- compute warps 0-7: P^T, dS^T, dQ drain
+    const int quad = warp & 3, hf = warp >> 2;
+    const int r = quad * 32 + lane;  // key row (S^T, dP^T), d row (dQ^T)
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool key_valid = kt * BN + r < p.N;
+    const float c = p.sl2;
+    const uint32_t box = sSTG + warp * Tr::BOX_BYTES;
+    uint8_t* gbox = gSTG + warp * Tr::BOX_BYTES;
+    bool ok = true;
+
+    // dQ^T tile i: TMEM -> this warp's swizzled fp32 staging box (32 queries x
+    // 32 d) -> TMA reduce-add into the accumulator, issued by lane 0.
+    auto drain_dq = [&](int i) -> bool {
+      const int qb = i & 1;
+      bool good = mbar_wait(bar(Tr::B_DQ_FULL + qb), (i >> 1) & 1, w, kBSiteDqFull);
+      if (!__all_sync(0xffffffffu, good)) return false;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tl + Tr::TM_DQ + qb * BM + hf * 32, v);
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_DQ_FREE + qb));
+      if (lane == 0) bulk_wait_read_all();  // the previous reduce has read the box
+      __syncwarp();
+      // v[j] = dQ[query 32 hf + j][d = 32 quad + lane]; box row j holds query j
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        *reinterpret_cast<float*>(gbox + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) +
+                                  (lane & 3) * 4) = __uint_as_float(v[j]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && *abort_flag == 0) {
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM + hf * 32);
+        tma_reduce_add_2d(&tmacc, box, quad * 32, row);
+        bulk_commit();
+      }
+      return true;
+    };
+
+    for (int i = 0; i < n_qt; ++i) {
+      const int qs = i % QST;
+      // ---- P^T = 2^(c S^T - LSE2) for this warp's 32 query columns
+      ok = mbar_wait(bar(Tr::B_S_FULL), i & 1, w, kBSiteSFull);
+      ok = ok && mbar_wait(bar(Tr::B_Q_FULL + qs), (i / QST) & 1, w, kBSiteQFullSm);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float4* l4 = reinterpret_cast<const float4*>(sL + qs * BM + hf * 32);
+      const float4* d4 = reinterpret_cast<const float4*>(sDD + qs * BM + hf * 32);
+      float pr[32];
+      {
+        uint32_t sr[32];
+        tmem_ld32(tl + Tr::TM_S + hf * 32, sr);
+        tmem_wait_ld();
+        reg_fence(sr);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 L = l4[j4];
+          pr[4 * j4] = ex2(fmaf(__uint_as_float(sr[4 * j4]), c, -L.x));
+          pr[4 * j4 + 1] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 1]), c, -L.y));
+          pr[4 * j4 + 2] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 2]), c, -L.z));
+          pr[4 * j4 + 3] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 3]), c, -L.w));
+        }
+        if (!key_valid) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pr[j] = 0.f;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = Elem<T>::pack(pr[2 * j], pr[2 * j + 1]);
+        tmem_st16(tl + Tr::TM_S + hf * 32, pk);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_P_READY));
+      // ---- dS^T = P^T o (dP^T - D) for the same columns
+      ok = mbar_wait(bar(Tr::B_DP_FULL), i & 1, w, kBSiteDpFull);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      uint32_t ds16[16];
+      {
+        uint32_t dr[32];
+        tmem_ld32(tl + Tr::TM_DP + hf * 32, dr);
+        tmem_wait_ld();
+        reg_fence(dr);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 Dv = d4[j4];
+          ds16[2 * j4] = Elem<T>::pack(pr[4 * j4] * (__uint_as_float(dr[4 * j4]) - Dv.x),
+                                       pr[4 * j4 + 1] * (__uint_as_float(dr[4 * j4 + 1]) - Dv.y));
+          ds16[2 * j4 + 1] =
+              Elem<T>::pack(pr[4 * j4 + 2] * (__uint_as_float(dr[4 * j4 + 2]) - Dv.z),
+                            pr[4 * j4 + 3] * (__uint_as_float(dr[4 * j4 + 3]) - Dv.w));
+        }
+      }
+      tmem_st16(tl + Tr::TM_DP + hf * 32, ds16);
+      // dS^T row r (key), queries [32 hf, 32 hf + 32): 16-byte chunks 4 hf .. 4 hf + 3
+      // of the 128-byte-swizzled row
+      uint8_t* ds_row = gDS + r * 128;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4*>(ds_row + (((4 * hf + u) ^ (r & 7)) * 16)) =
+            make_uint4(ds16[4 * u], ds16[4 * u + 1], ds16[4 * u + 2], ds16[4 * u + 3]);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_DS_READY));
+      // ---- dQ of the previous tile
+      if (i > 0 && !(ok = drain_dq(i - 1))) break;
+    }
+    if (ok && n_qt > 0) ok = drain_dq(n_qt - 1);
+    if (lane == 0) bulk_wait_all();
+    // ---- epilogue: dV and scale * dK, key row r, d columns [64 hf, 64 hf + 64)
+    if (ok) ok = mbar_wait(bar(Tr::B_KV_DONE), 0, w, kBSiteKvDone);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const int key = kt * BN + r;
+      const size_t off = (((size_t)b * p.N + key) * p.H + h) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int col = hf * (D / 2) + cc * 32;
+        uint32_t a[32], k2[32];
+        tmem_ld32(tl + Tr::TM_DV + col, a);
+        tmem_ld32(tl + Tr::TM_DK + col, k2);
+        tmem_wait_ld();
+        reg_fence(a);
+        reg_fence(k2);
+        uint4 va[4], vk[4];
+        uint32_t* pa = reinterpret_cast<uint32_t*>(va);
+        uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
+          pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
+                                 __uint_as_float(k2[2 * j + 1]) * p.scale);
+        }
+        if (key_valid) {
+          uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dv) + off + col);
+          uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dk) + off + col);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            dvp[j] = va[j];
+            dkp[j] = vk[j];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Tr::TMEM_COLS);
+  }
+}
+
 // D_i = sum_x dO_ix O_ix; base-2 LSE; zero the dQ accumulator.  One warp per
 // padded row (b, h, i); rows past N get D = 0 and LSE = +inf (so P = 0 there).
 template <class T, int D>
@@ -535,25 +935,25 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
   *reinterpret_cast<uint4*>(dq + idx) = out;
 }
 
+// The three launches of one backward pass with scratch at ws (ws_bytes from
+// bwd_scratch_bytes): pre-pass, main kernel, dQ conversion.
 template <class T, class Tr>
-static int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
-                   cudaStream_t stream) {
+static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                                   const CUtensorMap, const CUtensorMap, const BwdParams),
+                      void* ws, const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                      int H, int N, float scale, cudaStream_t stream, bool timed) {
   constexpr int D = Tr::D;
   const bool bf16 = Elem<T>::kFmt == 1;
-  CUtensorMap tmq, tmk, tmv, tmdo;
+  CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
   int rc;
   if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
   if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
   if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
   if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
-
   const int n_qt = (N + Tr::BM - 1) / Tr::BM;
   const int Npad = n_qt * Tr::BM;
   const size_t rows = (size_t)B * H * Npad;
-  void* ws = nullptr;
-  const size_t ws_bytes = rows * D * sizeof(float) + 2 * rows * sizeof(float);
-  if ((rc = scratch_alloc(&ws, ws_bytes, stream)) != FA_OK) return rc;
   BwdParams p{};
   p.dq_acc = static_cast<float*>(ws);
   float* lse2 = p.dq_acc + rows * D;
@@ -571,43 +971,52 @@ static int run_bwd(const void* q, const void* k, const void* v, const void* o, c
   p.scale = scale;
   p.limit_ns = 4000000000ull;
   p.status = device_status_ptr();
-
-  CUtensorMap tmacc;
-  if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::BM)) != FA_OK) {
-    scratch_free(ws, stream);
+  if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::ACC_BOX_ROWS)) != FA_OK)
     return rc;
-  }
+  if ((rc = check_launch_regs((const void*)kern)) != FA_OK) return rc;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
+      cudaSuccess)
+    return launch_status(cudaGetLastError());
 
+  // The pre-pass rewrites every scratch word the pass reads (it zeroes the
+  // accumulator), so earlier contents of the scratch never leak in.
   fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
       Npad);
-  rc = launch_status(cudaGetLastError());
   note_launches(1);
-  if (rc == FA_OK) {
-    auto kern = fa_bwd_kernel<T, Tr>;
-    if ((rc = check_launch_regs((const void*)kern)) != FA_OK) {
-      // refused: the register split would not fit this build's allocation
-    } else if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Tr::SMEM_BYTES) != cudaSuccess) {
-      rc = launch_status(cudaGetLastError());
-    } else {
-      dim3 grid((N + Tr::BN - 1) / Tr::BN, H, B);
-      cudaEvent_t ev0, ev1;
-      take_kernel_events(true, &ev0, &ev1);
-      if (ev0) cudaEventRecord(ev0, stream);
-      kern<<<grid, 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
-      rc = launch_status(cudaGetLastError());
-      if (ev1) cudaEventRecord(ev1, stream);
-      note_launches(1);
-    }
-  }
-  if (rc == FA_OK) {
-    const long long total = (long long)B * N * H * D;
-    fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
-        p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
-    rc = launch_status(cudaGetLastError());
-    note_launches(1);
-  }
+  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (timed) take_kernel_events(true, &ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, stream);
+  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo,
+                                                                              tmacc, p);
+  rc = launch_status(cudaGetLastError());
+  if (ev1) cudaEventRecord(ev1, stream);
+  note_launches(1);
+  if (rc != FA_OK) return rc;
+  const long long total = (long long)B * N * H * D;
+  fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
+      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
+  note_launches(1);
+  return launch_status(cudaGetLastError());
+}
+
+template <class Tr>
+static size_t bwd_scratch_bytes(int B, int H, int N) {
+  const size_t rows = (size_t)B * H * ((N + Tr::BM - 1) / Tr::BM) * Tr::BM;
+  return rows * Tr::D * sizeof(float) + 2 * rows * sizeof(float);
+}
+
+template <class T, class Tr>
+static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                                const CUtensorMap, const CUtensorMap, const BwdParams),
+                   const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
+                   cudaStream_t stream) {
+  void* ws = nullptr;
+  int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N), stream);
+  if (rc != FA_OK) return rc;
+  rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, stream, true);
   scratch_free(ws, stream);
   return rc;
 }
@@ -621,7 +1030,11 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
   if (rc != FA_OK) return rc;
   switch (d) {
     case 64:
-      return run_bwd<T, BwdTraits64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, stream);
+      return run_bwd<T, BwdTraits64>(fa_bwd_kernel<T, BwdTraits64>, q, k, v, o, dout, lse, dq, dk,
+                                     dv, B, H, N, scale, stream);
+    case 128:
+      return run_bwd<T, BwdTq128>(fa_bwd_tq_kernel<T, BwdTq128>, q, k, v, o, dout, lse, dq, dk, dv,
+                                  B, H, N, scale, stream);
     default:
       return FA_ERR_HEADDIM;
   }
@@ -670,61 +1083,12 @@ template <class T, class Tr>
 static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, const void* o,
                                  const void* dout, const float* lse, void* dq, void* dk, void* dv,
                                  int B, int H, int N, float scale, cudaStream_t stream) {
-  constexpr int D = Tr::D;
-  const int n_qt = (N + Tr::BM - 1) / Tr::BM;
-  const int Npad = n_qt * Tr::BM;
-  const size_t rows = (size_t)B * H * Npad;
-  const size_t ws_bytes = rows * D * sizeof(float) + 2 * rows * sizeof(float);
-  if (ws_bytes > kFixedScratchBytes) return FA_ERR_SCRATCH;
+  if (bwd_scratch_bytes<Tr>(B, H, N) > kFixedScratchBytes) return FA_ERR_SCRATCH;
   void* ws = nullptr;
   int rc = fixed_scratch_address(&ws);
   if (rc != FA_OK) return rc;
-
-  const bool bf16 = Elem<T>::kFmt == 1;
-  CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
-  BwdParams p{};
-  p.dq_acc = static_cast<float*>(ws);
-  float* lse2 = p.dq_acc + rows * D;
-  float* dvec = lse2 + rows;
-  p.lse2 = lse2;
-  p.dvec = dvec;
-  p.dk = dk;
-  p.dv = dv;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.Npad = Npad;
-  p.n_qt = n_qt;
-  p.sl2 = scale * kLog2e;
-  p.scale = scale;
-  p.limit_ns = 4000000000ull;
-  p.status = device_status_ptr();
-  if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::BM)) != FA_OK) return rc;
-
-  // The pre-pass rewrites every scratch word this call reads (it zeroes the
-  // accumulator), so the previous call's contents never leak into this one.
-  fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
-      Npad);
-  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
-  auto kern = fa_bwd_kernel<T, Tr>;
-  if ((rc = check_launch_regs((const void*)kern)) != FA_OK) return rc;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES) !=
-      cudaSuccess)
-    return launch_status(cudaGetLastError());
-  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv,
-                                                                               tmdo, tmacc, p);
-  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
-  const long long total = (long long)B * N * H * D;
-  fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
-      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
-  if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
-  note_launches(3);
-  return FA_OK;
+  return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr>, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N,
+                           scale, stream, false);
 }
 
 }  // namespace fa

@@ -958,9 +958,12 @@ static int choose_splits(long long base_units, int n_kvt, int sm_count) {
 // give every SM the same number of (unit, K/V tile) steps instead.  Units are
 // then cut into pieces across neighbouring blocks and merged in the kernel,
 // so it is kept for units long enough (>= 16 K/V tiles) that the extra
-// Q loads and merges stay small, and for at least 4 steps a block.
+// Q loads and merges stay small, and for more than one wave of units (with
+// fewer units than SMs nearly every unit would be cut, and measured on B200
+// the merges then cost more than the idle SMs: 128 units of 32 tiles ran
+// 79 us balanced against 74 us round-robin).
 static bool use_balanced(long long units, int n_kvt, int sm_count) {
-  if (n_kvt < 16 || units * n_kvt < 4ll * sm_count || units * n_kvt >= (1ll << 31)) return false;
+  if (n_kvt < 16 || units <= sm_count || units * n_kvt >= (1ll << 31)) return false;
   const long long waves = (units + sm_count - 1) / sm_count;
   return (double)units / (double)(waves * sm_count) < 0.95;
 }

@@ -64,6 +64,23 @@ def test_fp16(fa, N):
     check_grads(fa, 1, N, 3, 64, "fp16", 600 + N)
 
 
+@pytest.mark.parametrize("N", [1, 17, 63, 64, 65, 127, 128, 129, 300, 640])
+def test_head_dim_128_bf16(fa, N):
+    # d = 128 runs the transposed-dQ kernel (64-query inner tiles)
+    check_grads(fa, 2, N, 2, 128, "bf16", 800 + N)
+
+
+@pytest.mark.parametrize("N", [1, 100, 257])
+def test_head_dim_128_fp16(fa, N):
+    check_grads(fa, 1, N, 3, 128, "fp16", 900 + N)
+
+
+def test_head_dim_128_many_tiles(fa):
+    # 16 key tiles per head, 32 query tiles each: both dQ^T buffers and every
+    # Q/dO stage are reused many times over
+    check_grads(fa, 1, 2048, 4, 128, "bf16", 950)
+
+
 def test_several_heads_and_batches(fa):
     check_grads(fa, 3, 200, 5, 64, "bf16", 701)
 
@@ -82,9 +99,10 @@ def test_training_workload_sampled_heads(fa):
         assert torch.isfinite(t.float()).all()
 
 
-def test_deterministic_dk_dv(fa):
+@pytest.mark.parametrize("d", [64, 128])
+def test_deterministic_dk_dv(fa, d):
     # dK and dV are owned by one block each (no atomics): bitwise repeatable.
-    q, k, v, dout = attn_inputs.draw(1, 700, 2, 64, "bf16", 702, 4, device="cuda")
+    q, k, v, dout = attn_inputs.draw(1, 700, 2, d, "bf16", 702, 4, device="cuda")
     a = run_bwd(fa, q, k, v, dout, 0.125)
     b = run_bwd(fa, q, k, v, dout, 0.125)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])

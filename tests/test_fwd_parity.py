@@ -72,12 +72,12 @@ def test_split_kv_path(fa):
     check_full(fa, 1, 1900, 1, 256, "bf16", 303)
 
 
-@pytest.mark.parametrize("B,N,H,d,dtype", [(1, 2000, 10, 64, "bf16"), (1, 2000, 10, 128, "fp16"),
-                                             (1, 4096, 5, 64, "bf16")])
+@pytest.mark.parametrize("B,N,H,d,dtype", [(1, 2000, 20, 64, "bf16"), (1, 2000, 20, 128, "fp16"),
+                                             (1, 4096, 10, 64, "bf16")])
 def test_balanced_schedule(fa, B, N, H, d, dtype):
-    # 80 units of 256 query rows on 148 SMs: every block takes an equal range
-    # of (unit, K/V tile) steps, so units are cut in two or three pieces on
-    # neighbouring blocks and merged in the kernel by their log-sum-exps
+    # 160 units of 256 query rows on 148 SMs: every block takes an equal range
+    # of (unit, K/V tile) steps, so units are cut in pieces on neighbouring
+    # blocks and merged in the kernel by their log-sum-exps
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert fa.fa_fwd_plan(B, H, N, d, sms)["balanced"] == 1
     check_full(fa, B, N, H, d, dtype, 310 + d + N)

@@ -18,7 +18,7 @@ SHAPES = [
     # (B, H, N, d): the workloads, the N sweep, ragged tails, few and many units
     (1, 2, 400, 64), (32, 4, 400, 64), (1, 1, 6400, 256), (1, 8, 8192, 128),
     (1, 8, 1024, 64), (1, 8, 2048, 64), (1, 8, 4096, 64), (1, 8, 8192, 64), (4, 8, 4096, 64),
-    (1, 10, 2000, 64), (1, 3, 8192, 64), (2, 3, 5000, 128), (1, 1, 1, 64), (3, 1, 129, 128),
+    (1, 10, 2000, 64), (1, 20, 2000, 64), (1, 10, 4096, 64), (1, 3, 8192, 64), (2, 3, 5000, 128), (1, 1, 1, 64), (3, 1, 129, 128),
     (1, 7, 4097, 64), (2, 16, 4096, 128), (1, 1, 100000, 64), (8, 16, 2048, 64),
 ]
 SMS = [148, 132, 7, 1]
