@@ -10,8 +10,8 @@
 //   dQ  += scale dS K   (fp32, reduced into global memory across K/V tiles)
 //
 // Three kernels:
-//   fa_bwd_pre_kernel   D, base-2 LSE (padded to whole Q tiles) and a zeroed
-//                       fp32 dQ accumulator
+//   fa_bwd_pre_kernel   D, minus the base-2 LSE (padded to whole Q tiles) and
+//                       a zeroed fp32 dQ accumulator
 //   fa_bwd_kernel       one block per (K/V tile of 128 keys, head, batch); its
 //                       loop walks the Q tiles of 128 queries
 //   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to 16 bits
@@ -55,7 +55,7 @@ struct BwdTraits64 {
   static constexpr int OFF_DO = OFF_Q + QST * QT_BYTES;
   static constexpr int OFF_DS = OFF_DO + QST * QT_BYTES;
   static constexpr int OFF_STG = OFF_DS + 2 * DS_BYTES;
-  static constexpr int OFF_L = OFF_STG + STAGE_BYTES;  // base-2 LSE per stage
+  static constexpr int OFF_L = OFF_STG + STAGE_BYTES;  // minus the base-2 LSE, per stage
   static constexpr int OFF_DD = OFF_L + QST * BM * 4;  // D per stage
   static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
@@ -74,7 +74,7 @@ struct BwdTraits64 {
 };
 
 struct BwdParams {
-  const float* lse2;  // [B, H, Npad] base-2 LSE, +inf past N
+  const float* lse2;  // [B, H, Npad] minus the base-2 LSE, -inf past N
   const float* dvec;  // [B, H, Npad] D, 0 past N
   float* dq_acc;      // [B, H, Npad, D] fp32
   void* dk;           // [B, N, H, D]
@@ -365,15 +365,17 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         reg_fence(sr[0]);
         reg_fence(sr[1]);
+        const uint64_t c2 = f32x2(c, c);
 #pragma unroll
         for (int j4 = 0; j4 < HC / 4; ++j4) {
-          const float4 L = l4[j4];
-          const float Ls[4] = {L.x, L.y, L.z, L.w};
+          const float4 L = l4[j4];  // minus the base-2 LSE of four queries
+          const int j = 4 * j4;
+          fma2(pr[j], pr[j + 1], __uint_as_float(sr[j / 32][j % 32]),
+               __uint_as_float(sr[j / 32][j % 32 + 1]), c2, f32x2(L.x, L.y));
+          fma2(pr[j + 2], pr[j + 3], __uint_as_float(sr[j / 32][j % 32 + 2]),
+               __uint_as_float(sr[j / 32][j % 32 + 3]), c2, f32x2(L.z, L.w));
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * j4 + e;
-            pr[j] = ex2(fmaf(__uint_as_float(sr[j / 32][j % 32]), c, -Ls[e]));
-          }
+          for (int e = 0; e < 4; ++e) pr[j + e] = ex2(pr[j + e]);
         }
         if (!key_valid) {
 #pragma unroll
@@ -405,13 +407,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int j4 = 0; j4 < HC / 4; ++j4) {
           const float4 Dv = d4[j4];
-          const float Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+          const int j = 4 * j4;
           float ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * j4 + e;
-            ds[e] = pr[j] * (__uint_as_float(dr[j / 32][j % 32]) - Ds[e]);
-          }
+          ds[0] = pr[j] * (__uint_as_float(dr[j / 32][j % 32]) - Dv.x);
+          ds[1] = pr[j + 1] * (__uint_as_float(dr[j / 32][j % 32 + 1]) - Dv.y);
+          ds[2] = pr[j + 2] * (__uint_as_float(dr[j / 32][j % 32 + 2]) - Dv.z);
+          ds[3] = pr[j + 3] * (__uint_as_float(dr[j / 32][j % 32 + 3]) - Dv.w);
           dk16[2 * j4] = Elem<T>::pack(ds[0], ds[1]);
           dk16[2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
         }
@@ -508,7 +509,7 @@ struct BwdTqTraits {
   static constexpr int OFF_DO = OFF_Q + QST * QT_BYTES;
   static constexpr int OFF_DS = OFF_DO + QST * QT_BYTES;
   static constexpr int OFF_STG = OFF_DS + DS_BYTES;
-  static constexpr int OFF_L = OFF_STG + 8 * BOX_BYTES;  // base-2 LSE per stage
+  static constexpr int OFF_L = OFF_STG + 8 * BOX_BYTES;  // minus the base-2 LSE, per stage
   static constexpr int OFF_DD = OFF_L + QST * BM * 4;    // D per stage
   static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
@@ -771,13 +772,16 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32(tl + Tr::TM_S + hf * 32, sr);
         tmem_wait_ld();
         reg_fence(sr);
+        const uint64_t c2 = f32x2(c, c);
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
-          const float4 L = l4[j4];
-          pr[4 * j4] = ex2(fmaf(__uint_as_float(sr[4 * j4]), c, -L.x));
-          pr[4 * j4 + 1] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 1]), c, -L.y));
-          pr[4 * j4 + 2] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 2]), c, -L.z));
-          pr[4 * j4 + 3] = ex2(fmaf(__uint_as_float(sr[4 * j4 + 3]), c, -L.w));
+          const float4 L = l4[j4];  // minus the base-2 LSE of four queries
+          fma2(pr[4 * j4], pr[4 * j4 + 1], __uint_as_float(sr[4 * j4]),
+               __uint_as_float(sr[4 * j4 + 1]), c2, f32x2(L.x, L.y));
+          fma2(pr[4 * j4 + 2], pr[4 * j4 + 3], __uint_as_float(sr[4 * j4 + 2]),
+               __uint_as_float(sr[4 * j4 + 3]), c2, f32x2(L.z, L.w));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pr[4 * j4 + e] = ex2(pr[4 * j4 + e]);
         }
         if (!key_valid) {
 #pragma unroll
@@ -804,11 +808,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const float4 Dv = d4[j4];
-          ds16[2 * j4] = Elem<T>::pack(pr[4 * j4] * (__uint_as_float(dr[4 * j4]) - Dv.x),
-                                       pr[4 * j4 + 1] * (__uint_as_float(dr[4 * j4 + 1]) - Dv.y));
-          ds16[2 * j4 + 1] =
-              Elem<T>::pack(pr[4 * j4 + 2] * (__uint_as_float(dr[4 * j4 + 2]) - Dv.z),
-                            pr[4 * j4 + 3] * (__uint_as_float(dr[4 * j4 + 3]) - Dv.w));
+          float ds[4];
+          sub_mul2(ds[0], ds[1], __uint_as_float(dr[4 * j4]), __uint_as_float(dr[4 * j4 + 1]),
+                   Dv.x, Dv.y, pr[4 * j4], pr[4 * j4 + 1]);
+          sub_mul2(ds[2], ds[3], __uint_as_float(dr[4 * j4 + 2]), __uint_as_float(dr[4 * j4 + 3]),
+                   Dv.z, Dv.w, pr[4 * j4 + 2], pr[4 * j4 + 3]);
+          ds16[2 * j4] = Elem<T>::pack(ds[0], ds[1]);
+          ds16[2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
         }
       }
       tmem_st16(tl + Tr::TM_DP + hf * 32, ds16);
@@ -873,8 +879,9 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// D_i = sum_x dO_ix O_ix; base-2 LSE; zero the dQ accumulator.  One warp per
-// padded row (b, h, i); rows past N get D = 0 and LSE = +inf (so P = 0 there).
+// D_i = sum_x dO_ix O_ix; minus the base-2 LSE; zero the dQ accumulator.  One
+// warp per padded row (b, h, i); rows past N get D = 0 and -LSE = -inf (so
+// P = 0 there).
 template <class T, int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o,
                                                          const T* __restrict__ dout,
@@ -908,7 +915,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
   for (int j = 0; j < PER; ++j) arow[j] = 0.f;
   if (lane == 0) {
     dvec[row] = acc;
-    lse2[row] = (i < N) ? lse[((size_t)b * H + h) * N + i] * kLog2e : INFINITY;
+    lse2[row] = (i < N) ? -(lse[((size_t)b * H + h) * N + i] * kLog2e) : -INFINITY;
   }
 }
 
@@ -1049,7 +1056,7 @@ template int bwd_launch<__half>(const void*, const void*, const void*, const voi
 
 // ------------------------------------------------------------------------
 // Fixed-scratch backward (fa_bwd_noalloc).  Same kernels as run_bwd, but the
-// scratch (dQ accumulator, base-2 LSE, D) lives in a file-scope device array
+// scratch (dQ accumulator, minus the base-2 LSE, D) lives in a file-scope device array
 // instead of a stream-ordered allocation, for callers that cannot allocate.
 // Host code cannot pass g_fixed_scratch itself to a kernel (in host code the
 // name denotes a host-side stand-in); its device address is looked up once

@@ -318,6 +318,53 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// Three-input max / min (one instruction for two new values of a running
+// reduction).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32x2 arithmetic (one instruction for two lanes of work, each lane
+// rounded exactly as the scalar operation).  A pair (lo, hi) travels as one
+// 64-bit operand; f32x2(v, v) broadcasts.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+// (x0, x1) = (s0 * c.lo + n.lo, s1 * c.hi + n.hi)
+__device__ __forceinline__ void fma2(float& x0, float& x1, float s0, float s1, uint64_t c,
+                                     uint64_t n) {
+  asm("{\n\t.reg .b64 a, r;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 r, a, %4, %5;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(x0), "=f"(x1)
+      : "f"(s0), "f"(s1), "l"(c), "l"(n));
+}
+// (a0, a1) += (b0, b1)
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
+// (r0, r1) = ((a0 - b0) * m0, (a1 - b1) * m1): packed subtract, then multiply
+__device__ __forceinline__ void sub_mul2(float& r0, float& r1, float a0, float a1, float b0,
+                                         float b1, float m0, float m1) {
+  asm("{\n\t.reg .b64 a, b, m, t;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mov.b64 m, {%6, %7};\n\tsub.rn.f32x2 t, a, b;\n\tmul.rn.f32x2 t, t, m;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(m0), "f"(m1));
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -142,7 +142,7 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
 
 // Timeout sites reported in the status word.
 enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull,
-       kSiteSFull, kSiteODone, kSiteEpi, kSitePeer };
+       kSiteSFull, kSiteODone, kSiteEpi, kSitePeer, kSiteSFree };
 
 // Growth of the running max (base 2) tolerated before O is rescaled.
 constexpr float kRescaleThreshold = 8.0f;
@@ -157,32 +157,44 @@ template <class T, int BN>
 __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], int valid, float c,
                                               float& m, float& l, uint32_t (&pk)[BN / 2]) {
   auto S = [&](int j) { return __uint_as_float(r[j / 32][j % 32]); };
-  // row max of s*c (the min of s when c < 0), 8 independent chains
-  float part[8];
   const bool full = valid >= BN;
   const bool neg = c < 0.f;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) part[q] = neg ? INFINITY : -INFINITY;
+  // row max of s*c (the min of s when c < 0): 8 independent chains, two new
+  // columns per three-input max
+  float mx;
   if (full) {
+    float part[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) part[q] = S(q);
     if (!neg) {
 #pragma unroll
-      for (int j = 0; j < BN; ++j) part[j & 7] = fmaxf(part[j & 7], S(j));
+      for (int j = 8; j < BN; j += 16)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) part[q] = max3f(part[q], S(j + q), S(j + 8 + q));
+      mx = max3f(max3f(part[0], part[1], part[2]), max3f(part[3], part[4], part[5]),
+                 fmaxf(part[6], part[7]));
     } else {
 #pragma unroll
-      for (int j = 0; j < BN; ++j) part[j & 7] = fminf(part[j & 7], S(j));
+      for (int j = 8; j < BN; j += 16)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) part[q] = min3f(part[q], S(j + q), S(j + 8 + q));
+      mx = min3f(min3f(part[0], part[1], part[2]), min3f(part[3], part[4], part[5]),
+                 fminf(part[6], part[7]));
     }
   } else {
+    float part[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) part[q] = neg ? INFINITY : -INFINITY;
 #pragma unroll
     for (int j = 0; j < BN; ++j)
       if (j < valid) part[j & 7] = neg ? fminf(part[j & 7], S(j)) : fmaxf(part[j & 7], S(j));
+    if (!neg)
+      mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
+                 fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
+    else
+      mx = fminf(fminf(fminf(part[0], part[1]), fminf(part[2], part[3])),
+                 fminf(fminf(part[4], part[5]), fminf(part[6], part[7])));
   }
-  float mx;
-  if (!neg)
-    mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
-               fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
-  else
-    mx = fminf(fminf(fminf(part[0], part[1]), fminf(part[2], part[3])),
-               fminf(fminf(part[4], part[5]), fminf(part[6], part[7])));
   const float mc = mx * c;  // max of s*c over the valid columns
   float alpha = 1.f;
   if (mc > m + kRescaleThreshold) {
@@ -190,18 +202,29 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
     m = mc;
   }
   const float neg_m = -m;
-  float sum[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) sum[q] = 0.f;
+  float rs;
   if (full) {
+    // x = s*c - m two columns per packed FMA; four packed running sums
+    const uint64_t c2 = f32x2(c, c), n2 = f32x2(neg_m, neg_m);
+    float sum[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum[q] = 0.f;
 #pragma unroll
     for (int j = 0; j < BN / 2; ++j) {
-      const float p0 = ex2(fmaf(S(2 * j), c, neg_m));
-      const float p1 = ex2(fmaf(S(2 * j + 1), c, neg_m));
-      sum[j & 7] += p0 + p1;
+      float x0, x1;
+      fma2(x0, x1, S(2 * j), S(2 * j + 1), c2, n2);
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      add2(sum[2 * (j & 3)], sum[2 * (j & 3) + 1], p0, p1);
       pk[j] = Elem<T>::pack(p0, p1);
     }
+    add2(sum[0], sum[1], sum[4], sum[5]);
+    add2(sum[2], sum[3], sum[6], sum[7]);
+    add2(sum[0], sum[1], sum[2], sum[3]);
+    rs = sum[0] + sum[1];
   } else {
+    float sum[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum[q] = 0.f;
 #pragma unroll
     for (int j = 0; j < BN / 2; ++j) {
       const float p0 = (2 * j < valid) ? ex2(fmaf(S(2 * j), c, neg_m)) : 0.f;
@@ -209,8 +232,8 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
       sum[j & 7] += p0 + p1;
       pk[j] = Elem<T>::pack(p0, p1);
     }
+    rs = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
   }
-  const float rs = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
   l = l * alpha + rs;
   return alpha;
 }
@@ -397,12 +420,19 @@ struct FwdPPTraits {
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
                        B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
                        B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
-                       B_O_DONE = B_P_FULL + 2, B_DRAIN = B_O_DONE + 2, NUM_BARS = B_DRAIN + 1;
+                       B_O_DONE = B_P_FULL + 2, B_S_FREE = B_O_DONE + 2,
+                       B_DRAIN = B_S_FREE + 2, NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr uint32_t TM_O = 2 * BN;
+  // P in its own tensor-memory columns when they fit (d = 64: S 2 x 128, P
+  // 2 x 64, O 2 x 64 = 512): Q K^T of the next K/V tile may then overwrite S
+  // as soon as the softmax warps have read it, before P.V has consumed P.
+  // Otherwise (d = 128) P is written over the first BN/2 columns of its S.
+  static constexpr bool SEP_P = 2 * BN + 2 * (BN / 2) + 2 * D <= 512;
+  static constexpr uint32_t TM_P = 2 * BN;                      // used when SEP_P
+  static constexpr uint32_t TM_O = SEP_P ? 3 * BN : 2 * BN;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(2 * BN + 2 * D <= 512, "tensor memory budget");
+  static_assert(TM_O + 2 * D <= 512, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -440,6 +470,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(Tr::B_S_FULL + s), 1);
       mbar_init(bar(Tr::B_P_FULL + s), 128);
       mbar_init(bar(Tr::B_O_DONE + s), 1);
+      mbar_init(bar(Tr::B_S_FREE + s), 128);
     }
     mbar_init(bar(Tr::B_DRAIN), 1);
     fence_mbar_init();
@@ -532,12 +563,63 @@ __global__ void __launch_bounds__(384, 1)
       // O_t (+)= P_t V for the V stage of counter vc
       auto issue_pv = [&](int t, bool first) {
         const uint64_t vd = desc_advance(v_desc0, (vc % VST) * Tr::KV_BYTES);
+        const uint32_t pa = Tr::SEP_P ? Tr::TM_P + t * (BN / 2) : t * BN;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + t * BN + kk * 8,
+          umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
                   desc_advance(vd, kk * 16 * 128), kIdescPV, (!first || kk > 0) ? 1u : 0u);
       };
       UnitIter it(p, blockIdx.x);
+      if constexpr (Tr::SEP_P) {
+        // S_0, S_1 of the next K/V tile are issued as soon as both softmax
+        // warpgroups have read the current ones (S_FREE), ahead of P.V; the
+        // tensor cores then compute the next scores while the exponentials of
+        // the current tile run, and each warpgroup can go straight on to its
+        // next tile.  Per K/V tile: Q0 K^T, Q1 K^T (next tile), P0 V, P1 V.
+        uint32_t sq = 0;  // S tiles issued per Q tile
+        auto issue_s_pair = [&]() -> bool {
+          if (!mbar_wait_warp(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))
+            return false;
+#pragma unroll 1
+          for (int t = 0; t < 2; ++t) {
+            if (sq > 0 && !mbar_wait_warp(bar(Tr::B_S_FREE + t), (sq - 1) & 1u, w, kSiteSFree))
+              return false;
+            tc_fence_after();
+            issue_qk(t);
+            umma_commit(leader, bar(Tr::B_S_FULL + t));
+          }
+          umma_commit(leader, bar(Tr::B_K_EMPTY + kc % KST));
+          ++kc;
+          ++sq;
+          return true;
+        };
+        for (Unit un; ok && it.next(p, un);) {
+          const int n = un.t1 - un.t0;
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
+          if (!(ok = issue_s_pair())) break;
+          if (n == 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
+          for (int j = 0; j < n; ++j, ++g) {
+            if (j + 1 < n) {
+              if (!(ok = issue_s_pair())) break;
+              if (j + 2 == n) umma_commit(leader, bar(Tr::B_Q_EMPTY));
+            }
+            if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 0), g & 1u, w, kSitePFull))) break;
+            if (!(ok = mbar_wait_warp(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
+              break;
+            tc_fence_after();
+            issue_pv(0, j == 0);
+            umma_commit(leader, bar(Tr::B_O_DONE + 0));
+            if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
+            tc_fence_after();
+            issue_pv(1, j == 0);
+            umma_commit(leader, bar(Tr::B_O_DONE + 1));
+            umma_commit(leader, bar(Tr::B_V_EMPTY + vc % VST));
+            ++vc;
+          }
+          if (!ok) break;
+          ++uc;
+        }
+      } else
       for (Unit un; ok && it.next(p, un);) {
         const int n = un.t1 - un.t0;
         if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
@@ -597,6 +679,7 @@ __global__ void __launch_bounds__(384, 1)
     const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = tl + wg * BN;
+    const uint32_t p_col = tl + Tr::TM_P + wg * (BN / 2);  // used when SEP_P
     const uint32_t o_col = tl + Tr::TM_O + wg * D;
     const float c = p.sl2;
     uint32_t g = 0;
@@ -615,18 +698,39 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
+        if constexpr (Tr::SEP_P) {
+          // S is in registers: the next tile's Q K^T may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(Tr::B_S_FREE + wg));
+        }
         uint32_t pk[BN / 2];
         const float alpha = softmax_step<T, BN>(r, p.N - (un.t0 + j) * BN, c, m, l, pk);
+        if constexpr (Tr::SEP_P) {
+          // P has one buffer per Q tile: the previous P.V (the previous tile of
+          // this unit, or the last of the previous unit, already waited for by
+          // its epilogue) must have read it, and have landed in O before O is
+          // rescaled
+          if (g > 0) {
+            ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteODone);
+            if (!(ok = __all_sync(0xffffffffu, ok))) break;
+            tc_fence_after();
+          }
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q) tmem_st16(s_col + q * 16, &pk[q * 16]);
-        tmem_wait_st();
-        if (j > 0) {
-          // the previous P.V into this O must have landed before O is touched
-          // or the next P.V is issued (every phase is waited once, in order)
-          ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteODone);
-          if (!(ok = __all_sync(0xffffffffu, ok))) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
+          for (int q = 0; q < BN / 32; ++q) tmem_st16(p_col + q * 16, &pk[q * 16]);
+          tmem_wait_st();
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
+        } else {
+#pragma unroll
+          for (int q = 0; q < BN / 32; ++q) tmem_st16(s_col + q * 16, &pk[q * 16]);
+          tmem_wait_st();
+          if (j > 0) {
+            // the previous P.V into this O must have landed before O is touched
+            // or the next P.V is issued (every phase is waited once, in order)
+            ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteODone);
+            if (!(ok = __all_sync(0xffffffffu, ok))) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
+          }
         }
         tc_fence_before();
         mbar_arrive(bar(Tr::B_P_FULL + wg));
