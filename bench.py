@@ -46,8 +46,6 @@ L2_FLUSH_BYTES = 512 << 20
 TRAFFIC = {
     ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.76384e6 + 23.8016e6,
                                                     "src": "8032130a965a3d77"},
-    ("fa_fwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.387712e6 + 1.182976e6,
-                                                    "src": "8032130a965a3d77"},
 }
 
 
@@ -133,6 +131,15 @@ def max_over_ranks(x: float, dist=None, device="cpu") -> float:
 def job_tflops(flop_per_step: float, ms_per_step: float, world: int) -> float:
     """Whole-job throughput: every rank processes flop_per_step in ms_per_step."""
     return world * flop_per_step / (ms_per_step * 1e-3) / 1e12
+
+
+def main_kernel_names(fa, w: attn_inputs.Workload, props) -> tuple:
+    """Names of the forward and backward main kernels the library launches for
+    this workload (the ones the kernel events bracket)."""
+    plan = fa.fa_fwd_plan(w.B, w.H, w.N, w.d, props.multi_processor_count)
+    fwd = "fa_fwd_pp_kernel" if plan["kernel"] == 1 else "fa_fwd_kernel"
+    bwd = "fa_bwd_kernel" if w.d == 64 else "fa_bwd_tq_kernel"
+    return fwd, bwd
 
 
 def cpu_oracle_sample(w: attn_inputs.Workload, rows: int, heads: int):
@@ -294,10 +301,11 @@ def main():
 
     # ----------------------------------------- roofline of the dominant kernel
     pk, pk_src = peaks()
+    fwd_name, bwd_name = main_kernel_names(fa, w, torch.cuda.get_device_properties(dev))
     if train:
-        dom, dom_ms, dom_flop = "fa_bwd_kernel", statistics.mean(bwd_ms), w.bwd_flop
+        dom, dom_ms, dom_flop = bwd_name, statistics.mean(bwd_ms), w.bwd_flop
     else:
-        dom, dom_ms, dom_flop = "fa_fwd_kernel", statistics.mean(fwd_ms), w.fwd_flop
+        dom, dom_ms, dom_flop = fwd_name, statistics.mean(fwd_ms), w.fwd_flop
     achieved = dom_flop / (dom_ms * 1e-3) / 1e12
     tr = TRAFFIC.get((dom, w.name))
     traffic = tr["bytes"] if tr and tr["src"] == kernel_source_hash() else None
@@ -306,10 +314,10 @@ def main():
                 "kernel": dom, "kernel_ms": dom_ms,
                 "peak_source": f"bf16_tflops (burst) of {pk_src} MEASURED_PEAKS.json",
                 "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
-    kernels = {"fa_fwd_kernel": {"ms": statistics.mean(fwd_ms),
-                                 "tflops": w.fwd_flop / (statistics.mean(fwd_ms) * 1e-3) / 1e12}}
+    kernels = {fwd_name: {"ms": statistics.mean(fwd_ms),
+                          "tflops": w.fwd_flop / (statistics.mean(fwd_ms) * 1e-3) / 1e12}}
     if train:
-        kernels["fa_bwd_kernel"] = {"ms": statistics.mean(bwd_ms), "tflops": achieved}
+        kernels[bwd_name] = {"ms": statistics.mean(bwd_ms), "tflops": achieved}
     for kv in kernels.values():
         kv["frac"] = kv["tflops"] / pk["bf16_tflops"]
 

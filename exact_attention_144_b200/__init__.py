@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.fa_set_kernel_events.restype = i
     lib.fa_kernel_launches.restype = ctypes.c_ulonglong
     lib.fa_last_cuda_error.restype = i
+    lib.fa_selftest_exp2.argtypes = [vp, vp, i, vp]
+    lib.fa_selftest_exp2.restype = i
     lib.fa_fwd_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(FwdPlan)]
     lib.fa_fwd_plan.restype = i
     lib.fa_fwd_plan_pieces.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int), i]
@@ -271,6 +273,18 @@ def fa_selftest_bounded_wait(limit_us: int = 20000) -> int:
     if rc != FA_OK:
         raise FAError("fa_selftest_bounded_wait", rc)
     return int(out.value)
+
+
+def fa_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x (float32 CUDA tensor) by the softmax's FMA-pipe exponential."""
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.float32
+            and x.is_contiguous()):
+        raise TypeError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    rc = _load().fa_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_selftest_exp2", rc)
+    return y
 
 
 def _event_handle(ev):

@@ -266,6 +266,17 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned long 
   __syncthreads();
 }
 
+// y = 2^x by ex2_poly2 (the FMA-pipe exponential of the softmax), two per thread
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : x[i];
+  float ya, yb;
+  ex2_poly2(ya, yb, a, b);
+  y[i] = ya;
+  if (i + 1 < n) y[i + 1] = yb;
+}
+
 }  // namespace fa
 
 // =================================================================== C ABI
@@ -374,6 +385,18 @@ FA_EXPORT int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long
     return FA_ERR_LAUNCH;
   }
   return fa_get_device_status(status_out, 1);
+}
+
+FA_EXPORT int fa_selftest_exp2(const float* x, float* y, int n, cudaStream_t stream) {
+  if (x == nullptr || y == nullptr) return FA_ERR_NULL;
+  if (n < 1) return FA_ERR_SHAPE;
+  fa::DeviceInfo dev;
+  int rc = fa::current_device(&dev);
+  if (rc != FA_OK) return rc;
+  const int pairs = (n + 1) / 2;
+  fa::selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  fa::note_launches(1);
+  return fa::launch_status(cudaGetLastError());
 }
 
 FA_EXPORT int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,

@@ -365,6 +365,36 @@ __device__ __forceinline__ void sub_mul2(float& r0, float& r1, float a0, float a
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(m0), "f"(m1));
 }
 
+// 2^x0, 2^x1 on the FMA pipe instead of MUFU, for offloading part of the
+// softmax exponentials.  Method: round-to-nearest range reduction x = n + f,
+// |f| <= 1/2, by adding 1.5 * 2^23 (the integer n lands in the low mantissa
+// bits of the sum); a degree-3 polynomial for 2^f whose coefficients were
+// fitted here by least squares on the relative error at Chebyshev nodes of
+// [-1/2, 1/2] (max relative error 7.5e-5 evaluated in fp32, far below the
+// 16-bit rounding of P); n is then added to the exponent field.  x is clamped
+// at -125 so that the result stays a normal number (2^-125 is far below every
+// p that matters: the row maximum gives p >= 2^-8).  Valid for x <= 127.
+__device__ __forceinline__ void ex2_poly2(float& y0, float& y1, float x0, float x1) {
+  const uint64_t magic = f32x2(12582912.f, 12582912.f);
+  const uint64_t c3 = f32x2(0.0551716648f, 0.0551716648f), c2 = f32x2(0.242611125f, 0.242611125f),
+                 c1 = f32x2(0.693260968f, 0.693260968f), c0 = f32x2(0.999928057f, 0.999928057f);
+  const uint64_t x = f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  uint64_t t, pv;
+  asm("{\n\t.reg .b64 n, f;\n\t"
+      "add.rn.f32x2 %0, %2, %3;\n\t"      // t = x + 1.5 * 2^23
+      "sub.rn.f32x2 n, %0, %3;\n\t"       // n = round(x)
+      "sub.rn.f32x2 f, %2, n;\n\t"        // f = x - n
+      "fma.rn.f32x2 %1, %4, f, %5;\n\t"
+      "fma.rn.f32x2 %1, %1, f, %6;\n\t"
+      "fma.rn.f32x2 %1, %1, f, %7;\n\t}"
+      : "=&l"(t), "=&l"(pv)
+      : "l"(x), "l"(magic), "l"(c3), "l"(c2), "l"(c1), "l"(c0));
+  const uint32_t tl = (uint32_t)t, th = (uint32_t)(t >> 32);
+  const uint32_t pl = (uint32_t)pv, ph = (uint32_t)(pv >> 32);
+  y0 = __uint_as_float(pl + (tl << 23));
+  y1 = __uint_as_float(ph + (th << 23));
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -147,13 +147,20 @@ enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteP
 // Growth of the running max (base 2) tolerated before O is rescaled.
 constexpr float kRescaleThreshold = 8.0f;
 
+
 // ---------------------------------------------------------------------------
 // One softmax step for the row a thread owns.  r holds the row's BN raw scores
 // (fp32 bits, unscaled); columns >= valid are keys past N.  c = scale*log2(e).
 // Updates the reference max m (base 2) and the running sum l, returns the
 // factor alpha that O must be multiplied by (1 when the reference max is
 // kept), and packs P = 2^(s*c - m) as 16-bit pairs into pk.
-template <class T, int BN>
+// EMU: of every 8 column pairs of a full tile, this many take their
+// exponentials on the FMA pipe (ex2_poly2) instead of MUFU.  It pays where one
+// softmax warp at a time keeps MUFU busy (the d = 128 ping-pong: 274 -> 266 us
+// on the long-sequence workload); where two warps per SM sub-partition run
+// their softmax together (d = 64) the extra instructions cost more than MUFU
+// time saved (225 -> 241 us), so there it is 0.
+template <class T, int BN, int EMU = 0>
 __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], int valid, float c,
                                               float& m, float& l, uint32_t (&pk)[BN / 2]) {
   auto S = [&](int j) { return __uint_as_float(r[j / 32][j % 32]); };
@@ -211,9 +218,14 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
     for (int q = 0; q < 8; ++q) sum[q] = 0.f;
 #pragma unroll
     for (int j = 0; j < BN / 2; ++j) {
-      float x0, x1;
+      float x0, x1, p0, p1;
       fma2(x0, x1, S(2 * j), S(2 * j + 1), c2, n2);
-      const float p0 = ex2(x0), p1 = ex2(x1);
+      if ((j & 7) >= 8 - EMU) {
+        ex2_poly2(p0, p1, x0, x1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
       add2(sum[2 * (j & 3)], sum[2 * (j & 3) + 1], p0, p1);
       pk[j] = Elem<T>::pack(p0, p1);
     }
@@ -429,6 +441,9 @@ struct FwdPPTraits {
   // as soon as the softmax warps have read it, before P.V has consumed P.
   // Otherwise (d = 128) P is written over the first BN/2 columns of its S.
   static constexpr bool SEP_P = 2 * BN + 2 * (BN / 2) + 2 * D <= 512;
+  // exponentials on the FMA pipe per 8 column pairs (see softmax_step): the
+  // d = 128 warpgroups take turns, the d = 64 ones run together
+  static constexpr int EMU = SEP_P ? 0 : 2;
   static constexpr uint32_t TM_P = 2 * BN;                      // used when SEP_P
   static constexpr uint32_t TM_O = SEP_P ? 3 * BN : 2 * BN;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -704,7 +719,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(bar(Tr::B_S_FREE + wg));
         }
         uint32_t pk[BN / 2];
-        const float alpha = softmax_step<T, BN>(r, p.N - (un.t0 + j) * BN, c, m, l, pk);
+        const float alpha = softmax_step<T, BN, Tr::EMU>(r, p.N - (un.t0 + j) * BN, c, m, l, pk);
         if constexpr (Tr::SEP_P) {
           // P has one buffer per Q tile: the previous P.V (the previous tile of
           // this unit, or the last of the previous unit, already waited for by

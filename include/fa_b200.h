@@ -188,6 +188,16 @@ int fa_get_device_status(unsigned long long *status_out, int clear);
 int fa_selftest_bounded_wait(unsigned int limit_us, unsigned long long *status_out);
 
 /*
+ * Diagnostic: y[i] = 2^x[i] for n device floats (n >= 1), computed by the
+ * FMA-pipe exponential that the forward softmax uses for part of each row's
+ * columns instead of the hardware ex2 (range reduction x = n + f, |f| <= 1/2,
+ * and a degree-3 polynomial for 2^f; relative error below 1e-4 for
+ * -125 <= x <= 127; inputs below -125 give about 2^-125).  Enqueued on
+ * `stream`; returns FA_OK, FA_ERR_NULL, FA_ERR_SHAPE or a launch error.
+ */
+int fa_selftest_exp2(const float *x, float *y, int n, cudaStream_t stream);
+
+/*
  * Instrumentation for benchmarks.  Arms CUDA events that the library records
  * on the launching stream immediately before and immediately after the main
  * kernel (fa_fwd_kernel / fa_bwd_kernel) of the next forward / backward call.
