@@ -66,6 +66,10 @@ WORKLOADS = {
 }
 for _n in (1024, 2048, 4096, 8192):
     WORKLOADS[f"sweep{_n}"] = Workload(f"c4_sweep_n{_n}_h8_d64", 1, _n, 8, 64, "bf16", 1000 + _n)
+# Not one of the pages' configurations: the long-sequence shape with a
+# backward, to measure and test the d = 128 backward at full size.
+WORKLOADS["c4train"] = Workload("c4_train_n8192_h8_d128", 1, 8192, 8, 128, "bf16", 1006,
+                                backward=True, note="long-sequence shape, forward + backward")
 
 
 def draw(B: int, N: int, H: int, d: int, dtype: str, seed: int, count: int = 3,
