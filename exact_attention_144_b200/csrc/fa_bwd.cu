@@ -48,7 +48,7 @@ struct BwdTraits64 {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int QT_BYTES = BM * D * 2;
   static constexpr int DS_BYTES = BN * BM * 2;       // dS tile, 16-bit
-  static constexpr int STAGE_BYTES = BM * D * 4;     // dQ tile, fp32
+  static constexpr int STAGE_BYTES = BM * D * 4;     // dQ tile, fp32: 8 warps x 4 KiB boxes
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
@@ -69,7 +69,8 @@ struct BwdTraits64 {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int ACC_BOX_ROWS = BM;  // dQ reduce box: 32 d columns x 128 queries
+  static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries (one warp's)
+  static constexpr int EMU = 0;  // exponentials on the FMA pipe per 8 column pairs of P^T
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -309,43 +310,38 @@ __global__ void __launch_bounds__(384, 1)
     const int r = quad * 32 + lane;  // key row (S^T, dP^T) and query row (dQ)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const bool key_valid = kt * BN + r < p.N;
-    const bool issuer = lane == 0 && quad == 0;  // one thread per half issues its reduce
     const float c = p.sl2;
     bool ok = true;
 
-    // dQ tile i: TMEM -> swizzled fp32 staging box hf -> TMA reduce-add
-    // Every thread of a half reaches both named barriers even when a wait
-    // gave up, so no warp is left waiting on them.
+    // dQ tile i: TMEM -> this warp's swizzled fp32 staging box (its 32 query
+    // rows x 32 d columns) -> TMA reduce-add issued by its lane 0.  Each warp
+    // only waits for its own previous reduce: no barrier across warps.
+    uint8_t* gbox = gSTG + warp * 4096;
     auto drain_dq = [&](int i) -> bool {
       bool good = mbar_wait(bar(Tr::B_DQ_FULL), i & 1, w, kBSiteDqFull);
-      good = __all_sync(0xffffffffu, good);
+      if (!__all_sync(0xffffffffu, good)) return false;
       uint32_t v[32];
-      if (good) {
-        tc_fence_after();
-        tmem_ld32(tl + Tr::TM_DQ + hf * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        tc_fence_before();
-        mbar_arrive(bar(Tr::B_DQ_FREE));
-      }
-      if (issuer) bulk_wait_read_all();  // the previous reduce has read the staging box
-      named_bar_sync(1 + hf, 128);
-      if (good) {
-        uint8_t* box = gSTG + hf * (BM * 128);
+      tc_fence_after();
+      tmem_ld32(tl + Tr::TM_DQ + hf * 32, v);
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(bar(Tr::B_DQ_FREE));
+      if (lane == 0) bulk_wait_read_all();  // the previous reduce has read the box
+      __syncwarp();
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) =
-              make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                          __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
-        fence_proxy_async_smem();
-      }
-      named_bar_sync(1 + hf, 128);
-      if (issuer && good && *abort_flag == 0) {
-        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM);
-        tma_reduce_add_2d(&tmacc, sSTG + hf * (BM * 128), hf * 32, row);
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<float4*>(gbox + lane * 128 + ((u ^ (lane & 7)) * 16)) =
+            make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                        __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && *abort_flag == 0) {
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM + quad * 32);
+        tma_reduce_add_2d(&tmacc, sSTG + warp * 4096, hf * 32, row);
         bulk_commit();
       }
-      return good;
+      return true;
     };
 
     for (int i = 0; i < n_qt; ++i) {
@@ -374,8 +370,19 @@ __global__ void __launch_bounds__(384, 1)
                __uint_as_float(sr[j / 32][j % 32 + 1]), c2, f32x2(L.x, L.y));
           fma2(pr[j + 2], pr[j + 3], __uint_as_float(sr[j / 32][j % 32 + 2]),
                __uint_as_float(sr[j / 32][j % 32 + 3]), c2, f32x2(L.z, L.w));
-#pragma unroll
-          for (int e = 0; e < 4; ++e) pr[j + e] = ex2(pr[j + e]);
+          // of every 8 column pairs, EMU take the FMA-pipe exponential
+          if (((j / 2) & 7) >= 8 - Tr::EMU) {
+            ex2_poly2(pr[j], pr[j + 1], pr[j], pr[j + 1]);
+          } else {
+            pr[j] = ex2(pr[j]);
+            pr[j + 1] = ex2(pr[j + 1]);
+          }
+          if ((((j + 2) / 2) & 7) >= 8 - Tr::EMU) {
+            ex2_poly2(pr[j + 2], pr[j + 3], pr[j + 2], pr[j + 3]);
+          } else {
+            pr[j + 2] = ex2(pr[j + 2]);
+            pr[j + 3] = ex2(pr[j + 3]);
+          }
         }
         if (!key_valid) {
 #pragma unroll
@@ -397,24 +404,23 @@ __global__ void __launch_bounds__(384, 1)
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
       uint32_t dk16[HC / 2];
-      {
-        uint32_t dr[2][32];
-        tmem_ld32(tl + Tr::TM_DP + hf * HC, dr[0]);
-        tmem_ld32(tl + Tr::TM_DP + hf * HC + 32, dr[1]);
-        tmem_wait_ld();
-        reg_fence(dr[0]);
-        reg_fence(dr[1]);
 #pragma unroll
-        for (int j4 = 0; j4 < HC / 4; ++j4) {
-          const float4 Dv = d4[j4];
-          const int j = 4 * j4;
+      for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time: fewer live registers
+        uint32_t dr[32];
+        tmem_ld32(tl + Tr::TM_DP + hf * HC + hh * 32, dr);
+        tmem_wait_ld();
+        reg_fence(dr);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 Dv = d4[hh * 8 + j4];
+          const int j = 32 * hh + 4 * j4;
           float ds[4];
-          ds[0] = pr[j] * (__uint_as_float(dr[j / 32][j % 32]) - Dv.x);
-          ds[1] = pr[j + 1] * (__uint_as_float(dr[j / 32][j % 32 + 1]) - Dv.y);
-          ds[2] = pr[j + 2] * (__uint_as_float(dr[j / 32][j % 32 + 2]) - Dv.z);
-          ds[3] = pr[j + 3] * (__uint_as_float(dr[j / 32][j % 32 + 3]) - Dv.w);
-          dk16[2 * j4] = Elem<T>::pack(ds[0], ds[1]);
-          dk16[2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
+          sub_mul2(ds[0], ds[1], __uint_as_float(dr[4 * j4]), __uint_as_float(dr[4 * j4 + 1]),
+                   Dv.x, Dv.y, pr[j], pr[j + 1]);
+          sub_mul2(ds[2], ds[3], __uint_as_float(dr[4 * j4 + 2]), __uint_as_float(dr[4 * j4 + 3]),
+                   Dv.z, Dv.w, pr[j + 2], pr[j + 3]);
+          dk16[16 * hh + 2 * j4] = Elem<T>::pack(ds[0], ds[1]);
+          dk16[16 * hh + 2 * j4 + 1] = Elem<T>::pack(ds[2], ds[3]);
         }
       }
       tmem_st16(tl + Tr::TM_DP + hf * HC, &dk16[0]);
@@ -433,7 +439,7 @@ __global__ void __launch_bounds__(384, 1)
       if (i > 0 && !(ok = drain_dq(i - 1))) break;
     }
     if (ok && n_qt > 0) ok = drain_dq(n_qt - 1);
-    if (issuer) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
     // ---- epilogue: dV and scale * dK, this warp's key rows and 32 of the d columns
     if (ok) ok = mbar_wait(bar(Tr::B_KV_DONE), 0, w, kBSiteKvDone);
     if (__all_sync(0xffffffffu, ok)) {
