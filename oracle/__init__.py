@@ -79,14 +79,14 @@ class Oracle:
         dp = ctypes.POINTER(ctypes.c_double)
         ip = ctypes.POINTER(ctypes.c_int)
         i, f = ctypes.c_int, ctypes.c_double
-        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f]
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f, i]
         lib.oracle_attn_fwd_two_pass.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f]
         lib.oracle_attn_fwd_online.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f, i, i]
-        lib.oracle_attn_fwd_rows.argtypes = [dp, dp, dp, ip, i, dp, dp, i, i, i, i, f]
-        lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, f]
-        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f]
-        lib.oracle_attn_bwd_rows.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f, i, i]
-        lib.oracle_attn_dscores.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f]
+        lib.oracle_attn_fwd_rows.argtypes = [dp, dp, dp, ip, i, dp, dp, i, i, i, i, f, i]
+        lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, f, i]
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f, i]
+        lib.oracle_attn_bwd_rows.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f, i, i, i]
+        lib.oracle_attn_dscores.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f, i]
         lib.oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
 
@@ -94,8 +94,9 @@ class Oracle:
         """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all host cores)."""
         return int(self.lib.oracle_num_threads())
 
-    def attn_fwd(self, q, k, v, scale):
-        """O = softmax(scale Q K^T) V and LSE (natural log) by the definition.
+    def attn_fwd(self, q, k, v, scale, causal=False):
+        """O = softmax(scale Q K^T) V and LSE (natural log) by the definition;
+        with causal, row i sees keys j <= i only.
 
         q, k, v: [B, N, H, d] arrays (any float dtype, widened to fp64).
         Returns o [B, N, H, d] fp64 and lse [B, H, N] fp64.
@@ -104,10 +105,11 @@ class Oracle:
         B, N, H, d = _shape(q)
         o = np.empty_like(q)
         lse = np.empty((B, H, N), dtype=np.float64)
-        self.lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale))
+        self.lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                 float(scale), int(bool(causal)))
         return o, lse
 
-    def attn_fwd_rows(self, q, k, v, scale, rows):
+    def attn_fwd_rows(self, q, k, v, scale, rows, causal=False):
         """Forward pass for selected (b, h, i) rows; returns o [R, d], lse [R]."""
         q, k, v = _c(q), _c(k), _c(v)
         B, N, H, d = _shape(q)
@@ -117,7 +119,8 @@ class Oracle:
         lse = np.empty((R,), dtype=np.float64)
         self.lib.oracle_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v),
                                       rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), R,
-                                      _ptr(o), _ptr(lse), B, H, N, d, float(scale))
+                                      _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                      int(bool(causal)))
         return o, lse
 
     def attn_fwd_two_pass(self, q, k, v, scale):
@@ -138,24 +141,25 @@ class Oracle:
                                         float(scale), int(block_q), int(block_kv))
         return o, lse
 
-    def attn_probs(self, q, k, scale):
+    def attn_probs(self, q, k, scale, causal=False):
         """P = softmax(scale Q K^T) as [B, H, N, N] (small N only)."""
         q, k = _c(q), _c(k)
         B, N, H, d = _shape(q)
         p = np.empty((B, H, N, N), dtype=np.float64)
-        self.lib.oracle_attn_probs(_ptr(q), _ptr(k), _ptr(p), B, H, N, d, float(scale))
+        self.lib.oracle_attn_probs(_ptr(q), _ptr(k), _ptr(p), B, H, N, d, float(scale),
+                                   int(bool(causal)))
         return p
 
-    def attn_bwd(self, q, k, v, dout, scale):
+    def attn_bwd(self, q, k, v, dout, scale, causal=False):
         """dQ, dK, dV of L = sum(O * dO) by recompute; each [B, N, H, d] fp64."""
         q, k, v, dout = _c(q), _c(k), _c(v), _c(dout)
         B, N, H, d = _shape(q)
         dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
         self.lib.oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                                 B, H, N, d, float(scale))
+                                 B, H, N, d, float(scale), int(bool(causal)))
         return dq, dk, dv
 
-    def attn_bwd_rows(self, q, k, v, dout, scale, row_begin, row_end):
+    def attn_bwd_rows(self, q, k, v, dout, scale, row_begin, row_end, causal=False):
         """Backward pass restricted to query rows [row_begin, row_end): dq rows
         in the range are exact; dk, dv are those rows' contributions.  Rows of
         dq outside the range are returned as zeros."""
@@ -166,16 +170,16 @@ class Oracle:
         dq, dk, dv = np.zeros_like(q), np.empty_like(q), np.empty_like(q)
         self.lib.oracle_attn_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
                                       _ptr(dv), B, H, N, d, float(scale), int(row_begin),
-                                      int(row_end))
+                                      int(row_end), int(bool(causal)))
         return dq, dk, dv
 
-    def attn_dscores(self, q, k, v, dout, scale):
+    def attn_dscores(self, q, k, v, dout, scale, causal=False):
         """dS = P * (dP - D) as [B, H, N, N] (small N only)."""
         q, k, v, dout = _c(q), _c(k), _c(v), _c(dout)
         B, N, H, d = _shape(q)
         ds = np.empty((B, H, N, N), dtype=np.float64)
         self.lib.oracle_attn_dscores(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(ds),
-                                     B, H, N, d, float(scale))
+                                     B, H, N, d, float(scale), int(bool(causal)))
         return ds
 
 
@@ -191,12 +195,12 @@ def num_threads():
     return default().num_threads()
 
 
-def attn_fwd(q, k, v, scale):
-    return default().attn_fwd(q, k, v, scale)
+def attn_fwd(q, k, v, scale, causal=False):
+    return default().attn_fwd(q, k, v, scale, causal)
 
 
-def attn_fwd_rows(q, k, v, scale, rows):
-    return default().attn_fwd_rows(q, k, v, scale, rows)
+def attn_fwd_rows(q, k, v, scale, rows, causal=False):
+    return default().attn_fwd_rows(q, k, v, scale, rows, causal)
 
 
 def attn_fwd_two_pass(q, k, v, scale):
@@ -207,17 +211,17 @@ def attn_fwd_online(q, k, v, scale, block_q, block_kv):
     return default().attn_fwd_online(q, k, v, scale, block_q, block_kv)
 
 
-def attn_probs(q, k, scale):
-    return default().attn_probs(q, k, scale)
+def attn_probs(q, k, scale, causal=False):
+    return default().attn_probs(q, k, scale, causal)
 
 
-def attn_bwd(q, k, v, dout, scale):
-    return default().attn_bwd(q, k, v, dout, scale)
+def attn_bwd(q, k, v, dout, scale, causal=False):
+    return default().attn_bwd(q, k, v, dout, scale, causal)
 
 
-def attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end):
-    return default().attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end)
+def attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end, causal=False):
+    return default().attn_bwd_rows(q, k, v, dout, scale, row_begin, row_end, causal)
 
 
-def attn_dscores(q, k, v, dout, scale):
-    return default().attn_dscores(q, k, v, dout, scale)
+def attn_dscores(q, k, v, dout, scale, causal=False):
+    return default().attn_dscores(q, k, v, dout, scale, causal)

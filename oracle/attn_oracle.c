@@ -15,6 +15,10 @@
  *   The LLM explainer page, section 6.2 (recompute strategy): backward by
  *   recomputing S and P; the gradients are the textbook chain rule through
  *   softmax, which that passage presupposes but does not print.
+ *   The LLM explainer page, section 7.1: the causal mask of GPT-style models,
+ *   which hides every future position from a query: with `causal` set, row i
+ *   attends to keys j <= i only (P_ij = 0 for j > i).  Every public function
+ *   takes `causal` as its last argument (0: all keys).
  *
  * Layout: q, k, v, o, dO, dq, dk, dv are [B, N, H, d] row-major fp64;
  * lse is [B, H, N] fp64, natural log.  All loops are plain and sequential
@@ -44,38 +48,42 @@ int oracle_num_threads(void)
 /*
  * Row i of the probability matrix, by the definition (YOLO11 page, 1.2):
  *   S_ij = scale * sum_x q_ix k_jx,  m_i = max_j S_ij,
- *   l_i = sum_j exp(S_ij - m_i),     P_ij = exp(S_ij - m_i) / l_i.
+ *   l_i = sum_j exp(S_ij - m_i),     P_ij = exp(S_ij - m_i) / l_i,
+ * over the keys the row sees: j < N, or j <= i with the causal mask (LLM
+ * explainer page, 7.1); P_ij = 0 for the hidden keys.
  * Writes P_i. into p[0..N) and returns m_i, l_i.
  */
 static void row_probs(const double *q, const double *k, int b, int h, int i,
-                      int N, int H, int d, double scale, double *p,
+                      int N, int H, int d, double scale, int causal, double *p,
                       double *m_out, double *l_out)
 {
+    const int nk = causal ? i + 1 : N;  /* keys visible to row i */
     const double *qi = q + at(b, i, h, 0, N, H, d);
-    for (int j = 0; j < N; ++j) {
+    for (int j = 0; j < nk; ++j) {
         const double *kj = k + at(b, j, h, 0, N, H, d);
         double dot = 0.0;
         for (int x = 0; x < d; ++x) dot += qi[x] * kj[x];
         p[j] = scale * dot;
     }
     double m = p[0];
-    for (int j = 1; j < N; ++j) if (p[j] > m) m = p[j];
+    for (int j = 1; j < nk; ++j) if (p[j] > m) m = p[j];
     double l = 0.0;
-    for (int j = 0; j < N; ++j) l += exp(p[j] - m);
-    for (int j = 0; j < N; ++j) p[j] = exp(p[j] - m) / l;
+    for (int j = 0; j < nk; ++j) l += exp(p[j] - m);
+    for (int j = 0; j < nk; ++j) p[j] = exp(p[j] - m) / l;
+    for (int j = nk; j < N; ++j) p[j] = 0.0;
     *m_out = m;
     *l_out = l;
 }
 
 /* P for every (b, h): probs is [B, H, N, N].  Small N only (tests). */
 void oracle_attn_probs(const double *q, const double *k, double *probs,
-                       int B, int H, int N, int d, double scale)
+                       int B, int H, int N, int d, double scale, int causal)
 {
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h)
             for (int i = 0; i < N; ++i) {
                 double m, l;
-                row_probs(q, k, b, h, i, N, H, d, scale,
+                row_probs(q, k, b, h, i, N, H, d, scale, causal,
                           probs + (((size_t)b * H + h) * N + i) * (size_t)N, &m, &l);
             }
 }
@@ -83,10 +91,10 @@ void oracle_attn_probs(const double *q, const double *k, double *probs,
 /* One output row: O_i = sum_j P_ij V_j, LSE_i = m_i + ln l_i. */
 static void fwd_row(const double *q, const double *k, const double *v,
                     int b, int h, int i, int N, int H, int d, double scale,
-                    double *p, double *o_row, double *lse_out)
+                    int causal, double *p, double *o_row, double *lse_out)
 {
     double m, l;
-    row_probs(q, k, b, h, i, N, H, d, scale, p, &m, &l);
+    row_probs(q, k, b, h, i, N, H, d, scale, causal, p, &m, &l);
     for (int x = 0; x < d; ++x) o_row[x] = 0.0;
     for (int j = 0; j < N; ++j) {
         const double *vj = v + at(b, j, h, 0, N, H, d);
@@ -98,7 +106,7 @@ static void fwd_row(const double *q, const double *k, const double *v,
 /* Forward pass by the definition, every row. */
 void oracle_attn_fwd(const double *q, const double *k, const double *v,
                      double *o, double *lse, int B, int H, int N, int d,
-                     double scale)
+                     double scale, int causal)
 {
     long long rows = (long long)B * H * N;
 #pragma omp parallel
@@ -109,7 +117,7 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
             int i = (int)(r % N);
             int h = (int)((r / N) % H);
             int b = (int)(r / ((long long)N * H));
-            fwd_row(q, k, v, b, h, i, N, H, d, scale, p,
+            fwd_row(q, k, v, b, h, i, N, H, d, scale, causal, p,
                     o + at(b, i, h, 0, N, H, d),
                     lse + ((size_t)b * H + h) * N + i);
         }
@@ -124,7 +132,7 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
 void oracle_attn_fwd_rows(const double *q, const double *k, const double *v,
                           const int *rows, int nrows, double *o_rows,
                           double *lse_rows, int B, int H, int N, int d,
-                          double scale)
+                          double scale, int causal)
 {
     (void)B;
 #pragma omp parallel
@@ -133,7 +141,7 @@ void oracle_attn_fwd_rows(const double *q, const double *k, const double *v,
 #pragma omp for schedule(dynamic, 1)
         for (int r = 0; r < nrows; ++r)
             fwd_row(q, k, v, rows[3 * r], rows[3 * r + 1], rows[3 * r + 2], N,
-                    H, d, scale, p, o_rows + (size_t)r * d, lse_rows + r);
+                    H, d, scale, causal, p, o_rows + (size_t)r * d, lse_rows + r);
         free(p);
     }
 }
@@ -255,7 +263,7 @@ void oracle_attn_fwd_online(const double *q, const double *k, const double *v,
 void oracle_attn_bwd_rows(const double *q, const double *k, const double *v,
                           const double *dout, double *dq, double *dk, double *dv,
                           int B, int H, int N, int d, double scale,
-                          int row_begin, int row_end)
+                          int row_begin, int row_end, int causal)
 {
     int heads = B * H;
 #pragma omp parallel
@@ -272,7 +280,7 @@ void oracle_attn_bwd_rows(const double *q, const double *k, const double *v,
                 }
             for (int i = row_begin; i < row_end; ++i) {
                 double m, l;
-                row_probs(q, k, b, h, i, N, H, d, scale, p, &m, &l);
+                row_probs(q, k, b, h, i, N, H, d, scale, causal, p, &m, &l);
                 const double *doi = dout + at(b, i, h, 0, N, H, d);
                 const double *qi = q + at(b, i, h, 0, N, H, d);
                 double Di = 0.0;
@@ -306,15 +314,15 @@ void oracle_attn_bwd_rows(const double *q, const double *k, const double *v,
 /* Backward pass over every query row (see oracle_attn_bwd_rows). */
 void oracle_attn_bwd(const double *q, const double *k, const double *v,
                      const double *dout, double *dq, double *dk, double *dv,
-                     int B, int H, int N, int d, double scale)
+                     int B, int H, int N, int d, double scale, int causal)
 {
-    oracle_attn_bwd_rows(q, k, v, dout, dq, dk, dv, B, H, N, d, scale, 0, N);
+    oracle_attn_bwd_rows(q, k, v, dout, dq, dk, dv, B, H, N, d, scale, 0, N, causal);
 }
 
 /* dS for every (b, h): ds is [B, H, N, N] (tests of the row-sum identity). */
 void oracle_attn_dscores(const double *q, const double *k, const double *v,
                          const double *dout, double *ds, int B, int H, int N,
-                         int d, double scale)
+                         int d, double scale, int causal)
 {
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     double *dp = (double *)malloc(sizeof(double) * (size_t)N);
@@ -322,7 +330,7 @@ void oracle_attn_dscores(const double *q, const double *k, const double *v,
         for (int h = 0; h < H; ++h)
             for (int i = 0; i < N; ++i) {
                 double m, l;
-                row_probs(q, k, b, h, i, N, H, d, scale, p, &m, &l);
+                row_probs(q, k, b, h, i, N, H, d, scale, causal, p, &m, &l);
                 const double *doi = dout + at(b, i, h, 0, N, H, d);
                 double Di = 0.0;
                 for (int j = 0; j < N; ++j) {

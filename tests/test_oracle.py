@@ -196,8 +196,8 @@ def check_online_recurrence_equals_definition_to_rounding(orc, block_q, block_kv
 
 # ---------------------------------------------------------------- backward
 
-def _loss(orc, q, k, v, dout, scale):
-    o, _ = orc.attn_fwd(q, k, v, scale)
+def _loss(orc, q, k, v, dout, scale, causal=False):
+    o, _ = orc.attn_fwd(q, k, v, scale, causal)
     return float(np.sum(o * dout))
 
 
@@ -286,7 +286,73 @@ def test_page_printed_shapes():
 
 # Every check above, in order; tests/test_oracle_mutants.py reruns the same
 # list against oracle copies with planted mistakes.
-CHECKS = [check_probability_rows_sum_to_one, check_zero_queries_give_mean_of_values, check_single_key_gives_its_value, check_constant_values_give_that_value, check_hand_worked_one_dimensional_case, check_shift_of_every_key_leaves_output_and_shifts_lse, check_permutations, check_one_hot_dominance_at_large_scale, check_heads_and_batches_are_independent, check_rows_entry_point_matches_full_forward, check_definition_matches_two_pass_form, check_online_recurrence_bit_equal_with_one_kv_block, check_online_recurrence_bit_equal_when_max_is_in_first_block, check_online_recurrence_equals_definition_to_rounding, check_backward_matches_central_finite_differences, check_score_gradient_rows_sum_to_zero, check_backward_closed_forms, check_backward_row_ranges_partition_the_full_backward]
+# ------------------------------------------------------------ causal mask
+# LLM explainer page, section 7.1: the causal mask hides every future position
+# from a query.  Row i sees keys j <= i.
+
+def check_causal_first_row_is_first_value(orc):
+    # row 0 sees only key 0: O_0 = V_0, LSE_0 = scale q_0 . k_0
+    B, N, H, d = 2, 9, 2, 5
+    q, k, v = rnd((B, N, H, d), 60), rnd((B, N, H, d), 61), rnd((B, N, H, d), 62)
+    o, lse = orc.attn_fwd(q, k, v, 0.6, causal=True)
+    assert np.array_equal(o[:, 0], v[:, 0])
+    expect = 0.6 * np.einsum("bhx,bhx->bh", q[:, 0], k[:, 0])
+    assert np.max(np.abs(lse[:, :, 0] - expect)) <= 1e-14
+
+
+def check_causal_rows_equal_attention_over_their_prefix(orc):
+    # brute force: causal row i is ordinary attention of q_i over keys and
+    # values 0..i (a problem of i + 1 positions, computed without the mask)
+    B, N, H, d = 1, 12, 2, 4
+    q, k, v = rnd((B, N, H, d), 63), rnd((B, N, H, d), 64), rnd((B, N, H, d), 65)
+    o, lse = orc.attn_fwd(q, k, v, 0.8, causal=True)
+    for i in range(N):
+        op, lp = orc.attn_fwd(q[:, :i + 1], k[:, :i + 1], v[:, :i + 1], 0.8)
+        assert np.max(np.abs(o[:, i] - op[:, i])) <= 1e-14, i
+        assert np.max(np.abs(lse[:, :, i] - lp[:, :, i])) <= 1e-14, i
+    # the last row sees every key: it matches the unmasked forward
+    o_full, lse_full = orc.attn_fwd(q, k, v, 0.8)
+    assert np.max(np.abs(o[:, -1] - o_full[:, -1])) <= 1e-14
+
+
+def check_causal_probabilities_are_lower_triangular(orc):
+    q, k = rnd((1, 23, 2, 6), 66), rnd((1, 23, 2, 6), 67)
+    p = orc.attn_probs(q, k, 0.9, causal=True)
+    upper = np.triu(np.ones((23, 23), dtype=bool), 1)
+    assert np.all(p[..., upper] == 0.0)
+    assert np.all(p[..., ~upper] > 0.0)
+    assert np.max(np.abs(p.sum(-1) - 1.0)) <= 1e-12
+
+
+def check_causal_backward_matches_central_finite_differences(orc):
+    B, N, H, d = 1, 6, 2, 3
+    q, k, v = rnd((B, N, H, d), 68), rnd((B, N, H, d), 69), rnd((B, N, H, d), 70)
+    dout = rnd((B, N, H, d), 71)
+    scale = 0.7
+    dq, dk, dv = orc.attn_bwd(q, k, v, dout, scale, causal=True)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (_loss(orc, args_p["q"], args_p["k"], args_p["v"], dout, scale, True)
+                       - _loss(orc, args_m["q"], args_m["k"], args_m["v"], dout, scale, True)) / (2 * h)
+        err = np.max(np.abs(fd - g))
+        assert err <= 1e-6 * max(1.0, np.max(np.abs(g))), (name, err)
+    # the last key is seen by the last query only: dV_{N-1} = P_{N-1,N-1} dO_{N-1}
+    p = orc.attn_probs(q, k, scale, causal=True)
+    expect = p[0, :, N - 1, N - 1][:, None] * dout[0, N - 1]
+    assert np.max(np.abs(dv[0, N - 1] - expect)) <= 1e-14
+
+
+CHECKS = [check_probability_rows_sum_to_one, check_zero_queries_give_mean_of_values, check_single_key_gives_its_value, check_constant_values_give_that_value, check_hand_worked_one_dimensional_case, check_shift_of_every_key_leaves_output_and_shifts_lse, check_permutations, check_one_hot_dominance_at_large_scale, check_heads_and_batches_are_independent, check_rows_entry_point_matches_full_forward, check_definition_matches_two_pass_form, check_online_recurrence_bit_equal_with_one_kv_block, check_online_recurrence_bit_equal_when_max_is_in_first_block, check_online_recurrence_equals_definition_to_rounding, check_backward_matches_central_finite_differences, check_score_gradient_rows_sum_to_zero, check_backward_closed_forms, check_backward_row_ranges_partition_the_full_backward, check_causal_first_row_is_first_value, check_causal_rows_equal_attention_over_their_prefix, check_causal_probabilities_are_lower_triangular, check_causal_backward_matches_central_finite_differences]
 
 def test_probability_rows_sum_to_one():
     check_probability_rows_sum_to_one(ORC)
@@ -362,3 +428,19 @@ def test_backward_closed_forms():
 
 def test_backward_row_ranges_partition_the_full_backward():
     check_backward_row_ranges_partition_the_full_backward(ORC)
+
+
+def test_causal_first_row_is_first_value():
+    check_causal_first_row_is_first_value(ORC)
+
+
+def test_causal_rows_equal_attention_over_their_prefix():
+    check_causal_rows_equal_attention_over_their_prefix(ORC)
+
+
+def test_causal_probabilities_are_lower_triangular():
+    check_causal_probabilities_are_lower_triangular(ORC)
+
+
+def test_causal_backward_matches_central_finite_differences():
+    check_causal_backward_matches_central_finite_differences(ORC)

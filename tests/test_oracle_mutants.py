@@ -43,6 +43,13 @@ MUTANTS = [
     ("online max never updated", "oracle_attn_fwd_online", "m[r] = m_new;", "(void)m_new;"),
     ("dS table without D", "oracle_attn_dscores",
      "row[j] = p[j] * (dp[j] - Di);", "row[j] = p[j] * dp[j];"),
+    ("causal mask lets one future key through", "row_probs",
+     "const int nk = causal ? i + 1 : N;", "const int nk = causal ? (i + 2 < N ? i + 2 : N) : N;"),
+    ("causal mask hides the diagonal", "row_probs",
+     "const int nk = causal ? i + 1 : N;", "const int nk = causal ? (i > 0 ? i : 1) : N;"),
+    ("causal mask ignored by the backward", "oracle_attn_bwd_rows",
+     "row_probs(q, k, b, h, i, N, H, d, scale, causal, p, &m, &l);",
+     "row_probs(q, k, b, h, i, N, H, d, scale, 0, p, &m, &l);"),
 ]
 
 # One representative argument set for each parametrised pin.
