@@ -54,7 +54,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, f, vp]
     lib.fa_bwd_f16.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes
-    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc"):
+    lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_bwd_ex.argtypes = [vp] * 9 + [i, i, i, i, f, i, ctypes.c_uint, vp]
+    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc", "fa_fwd_ex",
+              "fa_bwd_ex"):
         getattr(lib, n).restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -73,6 +76,11 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_plan.restype = i
     lib.fa_fwd_plan_pieces.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int), i]
     lib.fa_fwd_plan_pieces.restype = i
+    lib.fa_fwd_plan_ex.argtypes = [i, i, i, i, ctypes.c_uint, i, ctypes.POINTER(FwdPlan)]
+    lib.fa_fwd_plan_ex.restype = i
+    lib.fa_fwd_plan_pieces_ex.argtypes = [i, i, i, i, ctypes.c_uint, i, i,
+                                          ctypes.POINTER(ctypes.c_int), i]
+    lib.fa_fwd_plan_pieces_ex.restype = i
     _lib = lib
     return lib
 
@@ -81,6 +89,10 @@ FA_OK = 0
 FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_ALIGN = -1, -2, -3, -4
 FA_ERR_LAUNCH, FA_ERR_NOMEM, FA_ERR_DEVICE, FA_ERR_SCALE = -5, -6, -7, -8
 FA_ERR_SCRATCH = -9
+FA_ERR_FLAGS, FA_ERR_DTYPE = -10, -11
+FA_BF16, FA_FP16 = 0, 1
+FA_FLAG_CAUSAL = 1
+_DTYPE_CODE = {torch.bfloat16: FA_BF16, torch.float16: FA_FP16}
 
 
 class FAError(RuntimeError):
@@ -137,7 +149,7 @@ def _check_bnhd(name: str, t: torch.Tensor, dtype: torch.dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def _fwd(entry: str, dtype, q, k, v, o, lse, scale, stream):
+def _fwd(entry: str, dtype, q, k, v, o, lse, scale, stream, flags: int = 0):
     _check_bnhd("q", q, dtype)
     if q.dim() != 4:
         raise ValueError("q must be [B, N, H, d]")
@@ -152,14 +164,19 @@ def _fwd(entry: str, dtype, q, k, v, o, lse, scale, stream):
     _check_bnhd("lse", lse, torch.float32, (B, H, N))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
-                              float(scale), _stream(stream))
+    if flags:
+        rc = _load().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                               float(scale), _DTYPE_CODE[dtype], int(flags), _stream(stream))
+        entry = "fa_fwd_ex"
+    else:
+        rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                  float(scale), _stream(stream))
     if rc != FA_OK:
         raise FAError(entry, rc)
     return o, lse
 
 
-def _bwd(entry: str, dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream):
+def _bwd(entry: str, dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream, flags: int = 0):
     _check_bnhd("q", q, dtype)
     if q.dim() != 4:
         raise ValueError("q must be [B, N, H, d]")
@@ -174,9 +191,15 @@ def _bwd(entry: str, dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream):
         _check_bnhd(name, t, dtype, q.shape)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
-                              _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
-                              _stream(stream))
+    if flags:
+        rc = _load().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                               _DTYPE_CODE[dtype], int(flags), _stream(stream))
+        entry = "fa_bwd_ex"
+    else:
+        rc = getattr(_load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                  _stream(stream))
     if rc != FA_OK:
         raise FAError(entry, rc)
     return dq, dk, dv
@@ -218,40 +241,65 @@ _FWD = {torch.bfloat16: fa_fwd, torch.float16: fa_fwd_f16}
 _BWD = {torch.bfloat16: fa_bwd, torch.float16: fa_bwd_f16}
 
 
-def forward(q, k, v, scale=None, o=None, lse=None, stream=None):
-    """fa_fwd or fa_fwd_f16, chosen by q's element type."""
+def fa_fwd_ex(q, k, v, o=None, lse=None, scale=None, flags=0, stream=None):
+    """Forward with flags (FA_FLAG_CAUSAL); element type from q (bf16 / fp16)."""
+    if q.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported element type {q.dtype}")
+    entry = "fa_fwd" if q.dtype == torch.bfloat16 else "fa_fwd_f16"
+    if flags == 0:
+        return _fwd(entry, q.dtype, q, k, v, o, lse, scale, stream)
+    return _fwd(entry, q.dtype, q, k, v, o, lse, scale, stream, flags)
+
+
+def fa_bwd_ex(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, flags=0, stream=None):
+    """Backward with flags (FA_FLAG_CAUSAL: o and lse from the causal forward)."""
+    if q.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported element type {q.dtype}")
+    entry = "fa_bwd" if q.dtype == torch.bfloat16 else "fa_bwd_f16"
+    return _bwd(entry, q.dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream, flags)
+
+
+def forward(q, k, v, scale=None, o=None, lse=None, stream=None, causal=False):
+    """fa_fwd or fa_fwd_f16 (fa_fwd_ex when causal), chosen by q's element type."""
     if q.dtype not in _FWD:
         raise TypeError(f"unsupported element type {q.dtype}")
+    if causal:
+        return fa_fwd_ex(q, k, v, o=o, lse=lse, scale=scale, flags=FA_FLAG_CAUSAL, stream=stream)
     return _FWD[q.dtype](q, k, v, o=o, lse=lse, scale=scale, stream=stream)
 
 
-def backward(q, k, v, o, dout, lse, scale=None, dq=None, dk=None, dv=None, stream=None):
-    """fa_bwd or fa_bwd_f16, chosen by q's element type."""
+def backward(q, k, v, o, dout, lse, scale=None, dq=None, dk=None, dv=None, stream=None,
+             causal=False):
+    """fa_bwd or fa_bwd_f16 (fa_bwd_ex when causal), chosen by q's element type."""
     if q.dtype not in _BWD:
         raise TypeError(f"unsupported element type {q.dtype}")
+    if causal:
+        return fa_bwd_ex(q, k, v, o, dout, lse, dq=dq, dk=dk, dv=dv, scale=scale,
+                         flags=FA_FLAG_CAUSAL, stream=stream)
     return _BWD[q.dtype](q, k, v, o, dout, lse, dq=dq, dk=dk, dv=dv, scale=scale, stream=stream)
 
 
-def fa_fwd_plan(B: int, H: int, N: int, d: int, sm_count: int) -> dict:
+def fa_fwd_plan(B: int, H: int, N: int, d: int, sm_count: int, flags: int = 0) -> dict:
     """The forward's work decomposition for a device with sm_count SMs (host
     logic only; needs no GPU)."""
     plan = FwdPlan()
-    rc = _load().fa_fwd_plan(B, H, N, d, sm_count, ctypes.byref(plan))
+    rc = _load().fa_fwd_plan_ex(B, H, N, d, flags, sm_count, ctypes.byref(plan))
     if rc != FA_OK:
         raise FAError("fa_fwd_plan", rc)
     return plan.as_dict()
 
 
-def fa_fwd_plan_pieces(B: int, H: int, N: int, d: int, sm_count: int, block: int) -> list:
+def fa_fwd_plan_pieces(B: int, H: int, N: int, d: int, sm_count: int, block: int,
+                       flags: int = 0) -> list:
     """The pieces one forward block processes, as (unit, first K/V tile, end
     K/V tile, kind, first peer, peer count) tuples; kind 0 = whole result,
     1 = partial rows, 2 = merge with the peers' partial rows."""
     lib_ = _load()
-    n = lib_.fa_fwd_plan_pieces(B, H, N, d, sm_count, block, None, 0)
+    n = lib_.fa_fwd_plan_pieces_ex(B, H, N, d, flags, sm_count, block, None, 0)
     if n < 0:
         raise FAError("fa_fwd_plan_pieces", n)
     buf = (ctypes.c_int * (6 * max(n, 1)))()
-    got = lib_.fa_fwd_plan_pieces(B, H, N, d, sm_count, block, buf, n)
+    got = lib_.fa_fwd_plan_pieces_ex(B, H, N, d, flags, sm_count, block, buf, n)
     if got != n:
         raise FAError("fa_fwd_plan_pieces", got if got < 0 else FA_ERR_SHAPE)
     return [tuple(buf[6 * i:6 * i + 6]) for i in range(n)]

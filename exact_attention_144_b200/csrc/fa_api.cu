@@ -221,21 +221,23 @@ static int check_ptrs(std::initializer_list<const void*> ptrs) {
 
 template <class T>
 static int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int H, int N, int d, float scale, cudaStream_t stream) {
+                     int H, int N, int d, float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, lse});
   if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
-  if (rc == FA_OK) rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, stream);
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc == FA_OK) rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
   return rc;
 }
 
 template <class T>
 static int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                     float scale, cudaStream_t stream) {
+                     float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
   if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc == FA_OK)
-    rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, stream);
+    rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, flags, stream);
   return rc;
 }
 
@@ -287,31 +289,56 @@ extern "C" {
 
 FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, cudaStream_t stream) {
-  return fa::fwd_entry<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, stream);
+  return fa::fwd_entry<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, 0u, stream);
 }
 
 FA_EXPORT int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int N, int d, float scale, cudaStream_t stream) {
-  return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, stream);
+  return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, 0u, stream);
+}
+
+FA_EXPORT int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int N, int d, float scale, int dtype, unsigned flags,
+                        cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::fwd_entry<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
+  if (dtype == FA_FP16)
+    return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
+  return FA_ERR_DTYPE;
 }
 
 FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
            const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
            cudaStream_t stream) {
-  return fa::bwd_entry<__nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale,
+  return fa::bwd_entry<__nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, 0u,
                                       stream);
 }
 
 FA_EXPORT int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                float scale, cudaStream_t stream) {
-  return fa::bwd_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, stream);
+  return fa::bwd_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, 0u, stream);
 }
 
-FA_EXPORT int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t* plan) {
+FA_EXPORT int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                        int H, int N, int d, float scale, int dtype, unsigned flags,
+                        cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::bwd_entry<__nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale,
+                                        flags, stream);
+  if (dtype == FA_FP16)
+    return fa::bwd_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, flags,
+                                 stream);
+  return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_fwd_plan_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
+                             fa_fwd_plan_t* plan) {
   if (plan == nullptr) return FA_ERR_NULL;
+  if ((flags & ~fa::kKnownFlags) != 0) return FA_ERR_FLAGS;
   fa::FwdSchedule s;
-  const int rc = fa::plan_fwd(B, H, N, d, sm_count, &s);
+  const int rc = fa::plan_fwd(B, H, N, d, flags, sm_count, &s);
   if (rc != FA_OK) return rc;
   plan->kernel = s.pair;
   plan->unit_rows = s.unit_rows;
@@ -325,14 +352,24 @@ FA_EXPORT int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_
   return FA_OK;
 }
 
-FA_EXPORT int fa_fwd_plan_pieces(int B, int H, int N, int d, int sm_count, int block,
-                                 int* pieces, int max_pieces) {
+FA_EXPORT int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t* plan) {
+  return fa_fwd_plan_ex(B, H, N, d, 0u, sm_count, plan);
+}
+
+FA_EXPORT int fa_fwd_plan_pieces_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
+                                    int block, int* pieces, int max_pieces) {
   if (pieces == nullptr && max_pieces > 0) return FA_ERR_NULL;
+  if ((flags & ~fa::kKnownFlags) != 0) return FA_ERR_FLAGS;
   fa::FwdSchedule s;
-  const int rc = fa::plan_fwd(B, H, N, d, sm_count, &s);
+  const int rc = fa::plan_fwd(B, H, N, d, flags, sm_count, &s);
   if (rc != FA_OK) return rc;
   if (block < 0 || block >= s.grid) return FA_ERR_SHAPE;
   return fa::fwd_block_pieces(s, block, pieces, max_pieces < 0 ? 0 : max_pieces);
+}
+
+FA_EXPORT int fa_fwd_plan_pieces(int B, int H, int N, int d, int sm_count, int block,
+                                 int* pieces, int max_pieces) {
+  return fa_fwd_plan_pieces_ex(B, H, N, d, 0u, sm_count, block, pieces, max_pieces);
 }
 
 FA_EXPORT const char* fa_status_string(int status) {
@@ -347,6 +384,8 @@ FA_EXPORT const char* fa_status_string(int status) {
     case FA_ERR_DEVICE: return "current device is not compute capability 10.0 (B200)";
     case FA_ERR_SCALE: return "scale is NaN or infinite";
     case FA_ERR_SCRATCH: return "problem needs more scratch than the fixed no-alloc buffer (64 MiB) holds";
+    case FA_ERR_FLAGS: return "unknown flag bits";
+    case FA_ERR_DTYPE: return "unknown element type";
     default: return "unknown status";
   }
 }

@@ -125,7 +125,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <class T, class Tr>
+template <class T, class Tr, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n_qt = p.n_qt;
+  // causal: query tiles wholly before this key tile see none of its keys
+  const int i0 = CAUSAL ? (kt * BN) / BM : 0;
+  const int n_qt = p.n_qt - i0;  // query tiles this block visits; tile i is global tile i0 + i
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -196,10 +198,12 @@ __global__ void __launch_bounds__(384, 1)
           break;
         const uint32_t fb = bar(Tr::B_Q_FULL + qs);
         mbar_expect_tx(leader, fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
-        tma_load_4d(leader, sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, i * BM, b);
-        tma_load_4d(leader, sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, i * BM, b);
-        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
-        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
+        tma_load_4d(leader, sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, (i0 + i) * BM, b);
+        tma_load_4d(leader, sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, (i0 + i) * BM, b);
+        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)(i0 + i) * BM,
+                  BM * 4, fb);
+        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)(i0 + i) * BM,
+                  BM * 4, fb);
         ++issued;
       }
       mbar_drain(bar(Tr::B_KV_FULL), 0, p.limit_ns);
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && *abort_flag == 0) {
-        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM + quad * 32);
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)(i0 + i) * BM + quad * 32);
         tma_reduce_add_2d(&tmacc, sSTG + warp * 4096, hf * 32, row);
         bulk_commit();
       }
@@ -384,9 +388,15 @@ __global__ void __launch_bounds__(384, 1)
             pr[j + 3] = ex2(pr[j + 3]);
           }
         }
-        if (!key_valid) {
+        // P = 0 for keys past N, and with the causal mask for the columns
+        // whose query comes before this key (query - key < 0: the first
+        // `hidden` of this warp's columns)
+        int hidden = key_valid ? 0 : HC;
+        if (CAUSAL) hidden = max(hidden, min(HC, (kt * BN + r) - ((i0 + i) * BM + hf * HC)));
+        if (hidden > 0) {
 #pragma unroll
-          for (int j = 0; j < HC; ++j) pr[j] = 0.f;
+          for (int j = 0; j < HC; ++j)
+            if (j < hidden) pr[j] = 0.f;
         }
         uint32_t pk[HC / 2];
 #pragma unroll
@@ -538,7 +548,7 @@ struct BwdTqTraits {
 
 using BwdTq128 = BwdTqTraits<128, 3>;
 
-template <class T, class Tr>
+template <class T, class Tr, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_tq_kernel(const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk,
@@ -563,7 +573,9 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n_qt = p.n_qt;
+  // causal: query tiles wholly before this key tile see none of its keys
+  const int i0 = CAUSAL ? (kt * BN) / BM : 0;
+  const int n_qt = p.n_qt - i0;  // query tiles this block visits; tile i is global tile i0 + i
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -622,12 +634,15 @@ __global__ void __launch_bounds__(384, 1)
         mbar_expect_tx(leader, fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
 #pragma unroll
         for (int c = 0; c < KCH; ++c) {
-          tma_load_4d(leader, sQ + qs * Tr::QT_BYTES + c * (BM * 128), &tmq, fb, c * 64, h, i * BM, b);
-          tma_load_4d(leader, sDO + qs * Tr::QT_BYTES + c * (BM * 128), &tmdo, fb, c * 64, h, i * BM,
-                      b);
+          tma_load_4d(leader, sQ + qs * Tr::QT_BYTES + c * (BM * 128), &tmq, fb, c * 64, h,
+                      (i0 + i) * BM, b);
+          tma_load_4d(leader, sDO + qs * Tr::QT_BYTES + c * (BM * 128), &tmdo, fb, c * 64, h,
+                      (i0 + i) * BM, b);
         }
-        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)i * BM, BM * 4, fb);
-        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)i * BM, BM * 4, fb);
+        bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)(i0 + i) * BM,
+                  BM * 4, fb);
+        bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)(i0 + i) * BM,
+                  BM * 4, fb);
         ++issued;
       }
       mbar_drain(bar(Tr::B_KV_FULL), 0, p.limit_ns);
@@ -756,7 +771,7 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && *abort_flag == 0) {
-        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)i * BM + hf * 32);
+        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)(i0 + i) * BM + hf * 32);
         tma_reduce_add_2d(&tmacc, box, quad * 32, row);
         bulk_commit();
       }
@@ -789,9 +804,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) pr[4 * j4 + e] = ex2(pr[4 * j4 + e]);
         }
-        if (!key_valid) {
+        int hidden = key_valid ? 0 : 32;  // as in fa_bwd_kernel
+        if (CAUSAL) hidden = max(hidden, min(32, (kt * BN + r) - ((i0 + i) * BM + hf * 32)));
+        if (hidden > 0) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) pr[j] = 0.f;
+          for (int j = 0; j < 32; ++j)
+            if (j < hidden) pr[j] = 0.f;
         }
         uint32_t pk[16];
 #pragma unroll
@@ -955,7 +973,7 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
                                    const CUtensorMap, const CUtensorMap, const BwdParams),
                       void* ws, const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                      int H, int N, float scale, cudaStream_t stream, bool timed) {
+                      int H, int N, float scale, unsigned flags, cudaStream_t stream, bool timed) {
   constexpr int D = Tr::D;
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
@@ -1025,11 +1043,12 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
                                 const CUtensorMap, const CUtensorMap, const BwdParams),
                    const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
-                   cudaStream_t stream) {
+                   unsigned flags, cudaStream_t stream) {
   void* ws = nullptr;
   int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N), stream);
   if (rc != FA_OK) return rc;
-  rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, stream, true);
+  rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags, stream,
+                         true);
   scratch_free(ws, stream);
   return rc;
 }
@@ -1037,17 +1056,21 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-               float scale, cudaStream_t stream) {
+               float scale, unsigned flags, cudaStream_t stream) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
   switch (d) {
     case 64:
-      return run_bwd<T, BwdTraits64>(fa_bwd_kernel<T, BwdTraits64>, q, k, v, o, dout, lse, dq, dk,
-                                     dv, B, H, N, scale, stream);
+      return run_bwd<T, BwdTraits64>((flags & 1u) ? fa_bwd_kernel<T, BwdTraits64, true>
+                                                  : fa_bwd_kernel<T, BwdTraits64, false>,
+                                     q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags,
+                                     stream);
     case 128:
-      return run_bwd<T, BwdTq128>(fa_bwd_tq_kernel<T, BwdTq128>, q, k, v, o, dout, lse, dq, dk, dv,
-                                  B, H, N, scale, stream);
+      return run_bwd<T, BwdTq128>((flags & 1u) ? fa_bwd_tq_kernel<T, BwdTq128, true>
+                                               : fa_bwd_tq_kernel<T, BwdTq128, false>,
+                                  q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags,
+                                  stream);
     default:
       return FA_ERR_HEADDIM;
   }
@@ -1055,10 +1078,10 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
 
 template int bwd_launch<__nv_bfloat16>(const void*, const void*, const void*, const void*,
                                        const void*, const float*, void*, void*, void*, int, int,
-                                       int, int, float, cudaStream_t);
+                                       int, int, float, unsigned, cudaStream_t);
 template int bwd_launch<__half>(const void*, const void*, const void*, const void*, const void*,
                                 const float*, void*, void*, void*, int, int, int, int, float,
-                                cudaStream_t);
+                                unsigned, cudaStream_t);
 
 // ------------------------------------------------------------------------
 // Fixed-scratch backward (fa_bwd_noalloc).  Same kernels as run_bwd, but the
@@ -1100,8 +1123,8 @@ static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, co
   void* ws = nullptr;
   int rc = fixed_scratch_address(&ws);
   if (rc != FA_OK) return rc;
-  return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr>, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N,
-                           scale, stream, false);
+  return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr, false>, ws, q, k, v, o, dout, lse, dq, dk, dv, B,
+                           H, N, scale, 0u, stream, false);
 }
 
 }  // namespace fa

@@ -63,6 +63,21 @@ __host__ __device__ __forceinline__ int range_begin(const FwdSchedule& s, int c)
 __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s) {
   Unit x;
   x.u = u;
+  x.kind = kStoreWhole;
+  x.peer0 = x.npeer = 0;
+  if (s.causal) {
+    // longest first: every head's last Q unit, then every head's second last,
+    // ...; a unit needs the K/V tiles up to its last query row
+    const int bh = u % (s.B * s.H), qi = u / (s.B * s.H);
+    x.qt = s.n_qt - 1 - qi;
+    x.sp = 0;
+    x.h = bh % s.H;
+    x.b = bh / s.H;
+    x.t0 = 0;
+    const int rows_end = imin(s.N, (x.qt + 1) * s.unit_rows);
+    x.t1 = (rows_end + s.bn - 1) / s.bn;
+    return x;
+  }
   x.qt = u % s.n_qt;
   int r = u / s.n_qt;
   x.sp = r % s.n_split;
@@ -71,14 +86,16 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
   x.b = r / s.H;
   x.t0 = x.sp * s.kvt_per_split;
   x.t1 = imin(x.t0 + s.kvt_per_split, s.n_kvt);
-  x.kind = kStoreWhole;
-  x.peer0 = x.npeer = 0;
   return x;
 }
 
 // The units (or pieces of units) block `blk` processes, in order.  Every role
 // of the block walks its own copy and sees the same sequence.
 //   plain:    units blk, blk + grid, blk + 2 grid, ...
+//   causal:   units in waves of grid, each wave walked in the opposite
+//             direction of the one before (units come longest first, so a
+//             block that took a long unit in one wave takes a short one in
+//             the next)
 //   balanced: the steps [range_begin(blk), range_begin(blk + 1)) cut at unit
 //             boundaries.  Only a block's first piece can start inside a unit
 //             (kStorePartial); the piece holding K/V tile 0 of a unit cut in
@@ -90,12 +107,23 @@ struct UnitIter {
     if (s.n_iter > 0) {
       i = range_begin(s, blk);
       end = range_begin(s, blk + 1);
+    } else if (s.causal) {
+      i = 0;  // wave
+      end = s.n_units;
     } else {
       i = blk;
       end = s.n_units;
     }
   }
   __host__ __device__ __forceinline__ bool next(const FwdSchedule& s, Unit& x) {
+    if (s.n_iter == 0 && s.causal) {
+      // a unit past the end in one wave means none in later waves either
+      const int u = i * s.grid + ((i & 1) ? s.grid - 1 - blk : blk);
+      if (u >= end) return false;
+      x = decode_unit(u, s);
+      ++i;
+      return true;
+    }
     if (i >= end) return false;
     if (s.n_iter == 0) {
       x = decode_unit(i, s);
@@ -719,7 +747,12 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(bar(Tr::B_S_FREE + wg));
         }
         uint32_t pk[BN / 2];
-        const float alpha = softmax_step<T, BN, Tr::EMU>(r, p.N - (un.t0 + j) * BN, c, m, l, pk);
+        // key columns this row sees in K/V tile t: below N, and with the
+        // causal mask up to the row's own position
+        const int t = un.t0 + j;
+        int valid = p.N - t * BN;
+        if (p.causal) valid = imin(valid, (2 * un.qt + wg) * BM + row - t * BN + 1);
+        const float alpha = softmax_step<T, BN, Tr::EMU>(r, valid, c, m, l, pk);
         if constexpr (Tr::SEP_P) {
           // P has one buffer per Q tile: the previous P.V (the previous tile of
           // this unit, or the last of the previous unit, already waited for by
@@ -990,7 +1023,10 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
         uint32_t pk[BN / 2];
-        const float alpha = softmax_step<T, BN>(r, p.N - (un.t0 + i) * BN, c, m, l, pk);
+        const int t = un.t0 + i;
+        int valid = p.N - t * BN;
+        if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
+        const float alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
 #pragma unroll
         for (int q = 0; q < BN / 32; ++q) tmem_st16(scol + q * 16, &pk[q * 16]);
         tmem_wait_st();
@@ -1087,7 +1123,7 @@ static bool use_balanced(long long units, int n_kvt, int sm_count) {
   return (double)units / (double)(waves * sm_count) < 0.95;
 }
 
-int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s) {
+int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedule* s) {
   if (B < 1 || H < 1 || N < 1 || sm_count < 1) return FA_ERR_SHAPE;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
   FwdSchedule x{};
@@ -1095,6 +1131,7 @@ int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s) {
   x.H = H;
   x.N = N;
   x.d = d;
+  x.causal = (flags & 1u) ? 1 : 0;
   // Two Q tiles per unit once a head has more than one tile's worth of rows;
   // a single tile per unit for short sequences and for d = 256 (whose O
   // accumulator leaves tensor memory room for only one Q tile).
@@ -1105,12 +1142,14 @@ int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s) {
   x.n_kvt = (N + x.bn - 1) / x.bn;
   const long long base_units = (long long)B * H * x.n_qt;
   if (base_units >= (1ll << 31)) return FA_ERR_SHAPE;
-  int n_split = choose_splits(base_units, x.n_kvt, sm_count);
+  // causal units differ in length: they are neither split nor cut, and run
+  // longest first (decode_unit)
+  int n_split = x.causal ? 1 : choose_splits(base_units, x.n_kvt, sm_count);
   x.kvt_per_split = (x.n_kvt + n_split - 1) / n_split;
   x.n_split = (x.n_kvt + x.kvt_per_split - 1) / x.kvt_per_split;  // no empty split
   x.n_units = (int)(base_units * x.n_split);
   const bool balanced =
-      x.pair && x.n_split == 1 && use_balanced(base_units, x.n_kvt, sm_count);
+      !x.causal && x.pair && x.n_split == 1 && use_balanced(base_units, x.n_kvt, sm_count);
   x.grid = balanced ? sm_count : (x.n_units < sm_count ? x.n_units : sm_count);
   if (balanced) {
     x.n_iter = (int)(base_units * x.n_kvt);
@@ -1244,12 +1283,12 @@ static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void
 
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, cudaStream_t stream) {
+               int N, int d, float scale, unsigned flags, cudaStream_t stream) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
   FwdSchedule s;
-  if ((rc = plan_fwd(B, H, N, d, dev.sm_count, &s)) != FA_OK) return rc;
+  if ((rc = plan_fwd(B, H, N, d, flags, dev.sm_count, &s)) != FA_OK) return rc;
   switch (d) {
     case 64:
       return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, stream)
@@ -1265,8 +1304,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
 }
 
 template int fwd_launch<__nv_bfloat16>(const void*, const void*, const void*, void*, float*, int,
-                                       int, int, int, float, cudaStream_t);
+                                       int, int, int, float, unsigned, cudaStream_t);
 template int fwd_launch<__half>(const void*, const void*, const void*, void*, float*, int, int,
-                                int, int, float, cudaStream_t);
+                                int, int, float, unsigned, cudaStream_t);
 
 }  // namespace fa

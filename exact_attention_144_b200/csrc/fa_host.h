@@ -63,12 +63,16 @@ int check_bwd_args(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale);
 
+// Flags of the *_ex entry points that the library knows (FA_FLAG_* bits).
+constexpr unsigned kKnownFlags = 1u;  // FA_FLAG_CAUSAL
+
 // Work decomposition of one forward call (fa_fwd.cu).  A unit is unit_rows
 // query rows of one (batch, head), possibly limited to one share of the K/V
 // tiles (split mode); blocks walk units round-robin, or in the balanced
 // schedule each block takes a contiguous range of (unit, K/V tile) steps.
 struct FwdSchedule {
   int B, H, N, d;
+  int causal;         // 1: row i sees keys j <= i (units ordered longest first)
   int pair;           // 1: fa_fwd_pp_kernel (two 128-row Q tiles a unit), 0: fa_fwd_kernel
   int unit_rows;      // 256 (pair) or 128
   int bn;             // K/V tile rows
@@ -84,7 +88,7 @@ struct FwdSchedule {
 
 // Fills *s for a forward call on a device with sm_count SMs (pure host logic).
 // FA_OK, or FA_ERR_SHAPE / FA_ERR_HEADDIM for shapes the forward rejects.
-int plan_fwd(int B, int H, int N, int d, int sm_count, FwdSchedule* s);
+int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedule* s);
 
 // Scratch bytes the forward needs for schedule s (split partials, or the
 // balanced schedule's partial-row slots and flags).
@@ -99,10 +103,10 @@ int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 // Launchers (argument validation is done by the callers in fa_api.cu).
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, cudaStream_t stream);
+               int N, int d, float scale, unsigned flags, cudaStream_t stream);
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-               float scale, cudaStream_t stream);
+               float scale, unsigned flags, cudaStream_t stream);
 
 }  // namespace fa

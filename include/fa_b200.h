@@ -65,9 +65,23 @@ enum fa_status {
     FA_ERR_NOMEM = -6,       /* scratch allocation failed                       */
     FA_ERR_DEVICE = -7,      /* current device is not compute capability 10.0   */
     FA_ERR_SCALE = -8,       /* scale is NaN or infinite                        */
-    FA_ERR_SCRATCH = -9      /* fa_bwd_noalloc: the problem needs more scratch than
+    FA_ERR_SCRATCH = -9,     /* fa_bwd_noalloc: the problem needs more scratch than
                                 its fixed buffer holds                           */
+    FA_ERR_FLAGS = -10,      /* *_ex: unknown flag bits                          */
+    FA_ERR_DTYPE = -11       /* *_ex: unknown element type                       */
 };
+
+/* Element types of the *_ex entry points. */
+enum fa_dtype { FA_BF16 = 0, FA_FP16 = 1 };
+
+/*
+ * Flags of the *_ex entry points.
+ * FA_FLAG_CAUSAL: the causal mask of autoregressive models (LLM explainer
+ *   page, section 7.1): query row i attends to key rows j <= i only (the
+ *   same position index in Q and K/V), i.e. S_ij = -inf for j > i before the
+ *   softmax; the LSE and the gradients are those of the masked problem.
+ */
+enum fa_flag { FA_FLAG_CAUSAL = 1u };
 
 /*
  * Forward pass, bf16.  Writes o [B,N,H,d] and lse [B,H,N].
@@ -79,6 +93,16 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 /* Forward pass, fp16; otherwise identical to fa_fwd. */
 int fa_fwd_f16(const void *q, const void *k, const void *v, void *o, float *lse,
                int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/*
+ * Forward pass with an element type (FA_BF16 / FA_FP16) and flags
+ * (FA_FLAG_*; 0 gives exactly fa_fwd / fa_fwd_f16).  Arguments, layout and
+ * errors as fa_fwd, plus FA_ERR_DTYPE and FA_ERR_FLAGS.  With FA_FLAG_CAUSAL
+ * the K/V tiles wholly above a Q tile's diagonal are skipped.
+ */
+int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+              int B, int H, int N, int d, float scale, int dtype, unsigned flags,
+              cudaStream_t stream);
 
 /*
  * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
@@ -96,6 +120,16 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
 int fa_bwd_f16(const void *q, const void *k, const void *v, const void *o,
                const void *dout, const float *lse, void *dq, void *dk, void *dv,
                int B, int H, int N, int d, float scale, cudaStream_t stream);
+
+/*
+ * Backward pass with an element type and flags, as fa_fwd_ex.  With
+ * FA_FLAG_CAUSAL, o and lse must come from the causal forward (fa_fwd_ex
+ * with the same flag); query tiles wholly before a key tile are skipped.
+ */
+int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+              const void *dout, const float *lse, void *dq, void *dk, void *dv,
+              int B, int H, int N, int d, float scale, int dtype, unsigned flags,
+              cudaStream_t stream);
 
 /*
  * Backward pass, bf16, for callers that cannot allocate device memory.
@@ -155,6 +189,12 @@ typedef struct fa_fwd_plan {
  */
 int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t *plan);
 
+/* fa_fwd_plan for fa_fwd_ex with the given flags (FA_ERR_FLAGS on unknown bits).
+ * Causal units cover only the K/V tiles up to their diagonal, are never cut
+ * or split, and are walked longest first. */
+int fa_fwd_plan_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
+                   fa_fwd_plan_t *plan);
+
 /*
  * The pieces block `block` (0 <= block < plan.grid) processes, in order,
  * 6 ints each: unit index, first K/V tile, end K/V tile, store kind
@@ -166,6 +206,10 @@ int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_t *plan);
  */
 int fa_fwd_plan_pieces(int B, int H, int N, int d, int sm_count, int block, int *pieces,
                        int max_pieces);
+
+/* fa_fwd_plan_pieces for fa_fwd_ex with the given flags. */
+int fa_fwd_plan_pieces_ex(int B, int H, int N, int d, unsigned flags, int sm_count, int block,
+                          int *pieces, int max_pieces);
 
 /* Static description of a status code.  Never NULL. */
 const char *fa_status_string(int status);

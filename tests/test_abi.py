@@ -122,3 +122,18 @@ def test_product_package_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_ex_entry_points_reject_bad_flags_and_types():
+    import ctypes
+    import exact_attention_144_b200 as fa
+    lib = fa.lib()
+    buf = (ctypes.c_char * 4096)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    args = [p] * 5 + [1, 1, 8, 64, ctypes.c_float(0.125)]
+    assert lib.fa_fwd_ex(*args, 0, 2, None) == fa.FA_ERR_FLAGS
+    assert lib.fa_fwd_ex(*args, 7, 0, None) == fa.FA_ERR_DTYPE
+    bargs = [p] * 9 + [1, 1, 8, 64, ctypes.c_float(0.125)]
+    assert lib.fa_bwd_ex(*bargs, 0, 0x80, None) == fa.FA_ERR_FLAGS
+    assert lib.fa_bwd_ex(*bargs, -1, 1, None) == fa.FA_ERR_DTYPE
+    assert fa.fa_status_string(fa.FA_ERR_FLAGS) == "unknown flag bits"

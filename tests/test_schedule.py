@@ -122,3 +122,46 @@ def test_plan_rejects_bad_arguments():
     assert e.value.status == fa.FA_ERR_HEADDIM
     with pytest.raises(fa.FAError):
         fa.fa_fwd_plan_pieces(1, 1, 64, 64, 148, 5)  # block past the grid
+
+
+# ------------------------------------------------------------------ causal
+CAUSAL = 1
+
+
+@pytest.mark.parametrize("sms", [148, 7, 1])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_causal_units_cover_up_to_their_diagonal(shape, sms):
+    # with the causal mask a unit of query rows [a, b) needs exactly the K/V
+    # tiles holding keys 0 .. b-1; every unit runs once, whole, on one block
+    B, H, N, d = shape
+    plan = fa.fa_fwd_plan(B, H, N, d, sms, CAUSAL)
+    assert plan["balanced"] == 0 and plan["n_split"] == 1 and plan["scratch_bytes"] == 0
+    ur, bn = plan["unit_rows"], plan["kv_tile_rows"]
+    n_qt = -(-N // ur)
+    assert plan["n_units"] == B * H * n_qt
+    seen = {}
+    for blk in range(plan["grid"]):
+        for (u, t0, t1, kind, peer0, npeer) in fa.fa_fwd_plan_pieces(B, H, N, d, sms, blk, CAUSAL):
+            assert kind == 0 and u not in seen
+            seen[u] = (t0, t1)
+    assert sorted(seen) == list(range(plan["n_units"]))
+    for u, (t0, t1) in seen.items():
+        qt = n_qt - 1 - u // (B * H)  # longest units first
+        assert (t0, t1) == (0, -(-min(N, (qt + 1) * ur) // bn)), (u, qt, t0, t1)
+
+
+def test_causal_waves_balance_the_load():
+    # 256 units of 2..64 K/V tiles on 148 blocks: alternating the direction of
+    # each wave keeps every block within 8 tiles of the mean
+    B, H, N, d = 1, 8, 8192, 128
+    plan = fa.fa_fwd_plan(B, H, N, d, 148, CAUSAL)
+    loads = [sum(t1 - t0 for (_, t0, t1, *_r) in fa.fa_fwd_plan_pieces(B, H, N, d, 148, b, CAUSAL))
+             for b in range(plan["grid"])]
+    assert sum(loads) == B * H * sum(2 * qt + 2 for qt in range(32))
+    assert max(loads) - sum(loads) / len(loads) <= 8
+
+
+def test_unknown_flags_are_rejected():
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_fwd_plan(1, 1, 64, 64, 148, 2)
+    assert e.value.status == fa.FA_ERR_FLAGS
