@@ -56,8 +56,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes
     lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
     lib.fa_bwd_ex.argtypes = [vp] * 9 + [i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_bwd_qkvpacked.argtypes = [vp] * 5 + [i, i, i, i, f, i, ctypes.c_uint, vp]
     for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc", "fa_fwd_ex",
-              "fa_bwd_ex"):
+              "fa_bwd_ex", "fa_fwd_qkvpacked", "fa_bwd_qkvpacked"):
         getattr(lib, n).restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -259,6 +261,51 @@ def fa_bwd_ex(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, scale=None, flag
     return _bwd(entry, q.dtype, q, k, v, o, dout, lse, dq, dk, dv, scale, stream, flags)
 
 
+def _check_packed(qkv):
+    if not isinstance(qkv, torch.Tensor) or not qkv.is_cuda or not qkv.is_contiguous():
+        raise ValueError("qkv must be a contiguous CUDA tensor")
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError("qkv must be [B, N, 3, H, d]")
+    if qkv.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported element type {qkv.dtype}")
+    B, N, _, H, d = qkv.shape
+    return B, N, H, d
+
+
+def fa_fwd_qkvpacked(qkv, o=None, lse=None, scale=None, flags=0, stream=None):
+    """Forward on a packed [B, N, 3, H, d] tensor; returns (o [B,N,H,d], lse)."""
+    B, N, H, d = _check_packed(qkv)
+    o = torch.empty((B, N, H, d), dtype=qkv.dtype, device=qkv.device) if o is None else o
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=qkv.device) if lse is None else lse
+    _check_bnhd("o", o, qkv.dtype, (B, N, H, d))
+    _check_bnhd("lse", lse, torch.float32, (B, H, N))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = _load().fa_fwd_qkvpacked(_ptr(qkv), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                  _DTYPE_CODE[qkv.dtype], int(flags), _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_qkvpacked", rc)
+    return o, lse
+
+
+def fa_bwd_qkvpacked(qkv, o, dout, lse, dqkv=None, scale=None, flags=0, stream=None):
+    """Backward on a packed tensor; returns dqkv [B, N, 3, H, d] (dQ, dK, dV)."""
+    B, N, H, d = _check_packed(qkv)
+    for name, t in (("o", o), ("dout", dout)):
+        _check_bnhd(name, t, qkv.dtype, (B, N, H, d))
+    _check_bnhd("lse", lse, torch.float32, (B, H, N))
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    if tuple(dqkv.shape) != tuple(qkv.shape) or dqkv.dtype != qkv.dtype or \
+            not dqkv.is_contiguous():
+        raise ValueError("dqkv must match qkv")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = _load().fa_bwd_qkvpacked(_ptr(qkv), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dqkv), B, H, N,
+                                  d, float(scale), _DTYPE_CODE[qkv.dtype], int(flags),
+                                  _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_bwd_qkvpacked", rc)
+    return dqkv
+
+
 def forward(q, k, v, scale=None, o=None, lse=None, stream=None, causal=False):
     """fa_fwd or fa_fwd_f16 (fa_fwd_ex when causal), chosen by q's element type."""
     if q.dtype not in _FWD:
@@ -354,3 +401,38 @@ def fa_set_kernel_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop
 def fa_kernel_launches() -> int:
     """Kernel launches this library has issued since it was loaded."""
     return int(_load().fa_kernel_launches())
+
+
+class _Attention(torch.autograd.Function):
+    """Autograd glue over the C entry points: the forward saves only O and the
+    LSE (the recompute strategy), the backward calls fa_bwd(_ex) with them."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal):
+        o, lse = forward(q, k, v, scale=scale, causal=causal)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.scale, ctx.causal = scale, causal
+        return o, lse
+
+    @staticmethod
+    def backward(ctx, do, dlse):
+        if dlse is not None and bool(torch.any(dlse != 0)):
+            raise NotImplementedError("gradients through the LSE output are not supported")
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, scale=ctx.scale,
+                              causal=ctx.causal)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, scale=None, causal=False, return_lse=False):
+    """Exact attention O = softmax(scale Q K^T [causal mask]) V with autograd.
+
+    q, k, v: contiguous [B, N, H, d] CUDA tensors of bfloat16 or float16;
+    scale defaults to 1/sqrt(d).  Returns O (and the fp32 LSE [B, H, N] when
+    return_lse).  The backward recomputes P from O and the LSE in the
+    library's kernels; no N x N matrix is ever stored.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    o, lse = _Attention.apply(q, k, v, float(scale), bool(causal))
+    return (o, lse) if return_lse else o

@@ -170,13 +170,13 @@ static EncodeTiledFn encode_fn() {
 }
 
 int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d,
-                   int box_rows) {
+                   int box_rows, long long tok_stride) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return FA_ERR_LAUNCH;
   // dims innermost first: element within head, head, token, batch
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
-                                 (cuuint64_t)N * H * d * 2};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)tok_stride * 2,
+                                 (cuuint64_t)N * tok_stride * 2};
   const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
@@ -225,7 +225,8 @@ static int fwd_entry(const void* q, const void* k, const void* v, void* o, float
   int rc = check_ptrs({q, k, v, o, lse});
   if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
-  if (rc == FA_OK) rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
+  if (rc == FA_OK)
+    rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, flags, (long long)H * d, stream);
   return rc;
 }
 
@@ -237,8 +238,41 @@ static int bwd_entry(const void* q, const void* k, const void* v, const void* o,
   if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc == FA_OK)
-    rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, flags, stream);
+    rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, flags,
+                       (long long)H * d, (long long)H * d, stream);
   return rc;
+}
+
+// Packed Q, K, V: qkv is [B, N, 3, H, d]; Q, K, V are its slices 0, 1, 2
+// (token stride 3*H*d), and dqkv the same for the gradients.
+template <class T>
+static int fwd_packed_entry(const void* qkv, void* o, float* lse, int B, int H, int N, int d,
+                            float scale, unsigned flags, cudaStream_t stream) {
+  int rc = check_ptrs({qkv, o, lse});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK && (long long)B * N * 3 * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc != FA_OK) return rc;
+  const T* base = static_cast<const T*>(qkv);
+  const long long hd = (long long)H * d;
+  return fwd_launch<T>(base, base + hd, base + 2 * hd, o, lse, B, H, N, d, scale, flags, 3 * hd,
+                       stream);
+}
+
+template <class T>
+static int bwd_packed_entry(const void* qkv, const void* o, const void* dout, const float* lse,
+                            void* dqkv, int B, int H, int N, int d, float scale, unsigned flags,
+                            cudaStream_t stream) {
+  int rc = check_ptrs({qkv, o, dout, lse, dqkv});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK && (long long)B * N * 3 * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc != FA_OK) return rc;
+  const T* base = static_cast<const T*>(qkv);
+  T* g = static_cast<T*>(dqkv);
+  const long long hd = (long long)H * d;
+  return bwd_launch<T>(base, base + hd, base + 2 * hd, o, dout, lse, g, g + hd, g + 2 * hd, B, H,
+                       N, d, scale, flags, 3 * hd, 3 * hd, stream);
 }
 
 int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -304,6 +338,26 @@ FA_EXPORT int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
     return fa::fwd_entry<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
   if (dtype == FA_FP16)
     return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
+  return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, int N, int d,
+                               float scale, int dtype, unsigned flags, cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::fwd_packed_entry<__nv_bfloat16>(qkv, o, lse, B, H, N, d, scale, flags, stream);
+  if (dtype == FA_FP16)
+    return fa::fwd_packed_entry<__half>(qkv, o, lse, B, H, N, d, scale, flags, stream);
+  return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_bwd_qkvpacked(const void* qkv, const void* o, const void* dout, const float* lse,
+                               void* dqkv, int B, int H, int N, int d, float scale, int dtype,
+                               unsigned flags, cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::bwd_packed_entry<__nv_bfloat16>(qkv, o, dout, lse, dqkv, B, H, N, d, scale, flags,
+                                               stream);
+  if (dtype == FA_FP16)
+    return fa::bwd_packed_entry<__half>(qkv, o, dout, lse, dqkv, B, H, N, d, scale, flags, stream);
   return FA_ERR_DTYPE;
 }
 

@@ -81,6 +81,7 @@ struct BwdParams {
   void* dk;           // [B, N, H, D]
   void* dv;
   int B, H, N, Npad, n_qt;
+  long long tok_g;    // token stride of dk, dv (elements): H*D, or 3*H*D when packed
   float sl2;          // scale * log2(e)
   float scale;
   unsigned long long limit_ns;
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = (((size_t)b * p.N + key) * p.H + h) * D + hf * 32;
+      const size_t off = ((size_t)b * p.N + key) * p.tok_g + (size_t)h * D + hf * 32;
       uint32_t a[32], k2[32];
       tmem_ld32(tl + Tr::TM_DV + hf * 32, a);
       tmem_ld32(tl + Tr::TM_DK + hf * 32, k2);
@@ -863,7 +864,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = (((size_t)b * p.N + key) * p.H + h) * D;
+      const size_t off = ((size_t)b * p.N + key) * p.tok_g + (size_t)h * D;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
         const int col = hf * (D / 2) + cc * 32;
@@ -943,11 +944,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
   }
 }
 
-// dQ = scale * accumulator, rounded; 8 elements per thread.
+// dQ = scale * accumulator, rounded; 8 elements per thread.  dq rows are
+// tok_g elements apart (H*D, or 3*H*D inside a packed dQKV).
 template <class T, int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dq_acc,
                                                         T* __restrict__ dq, int B, int H, int N,
-                                                        int Npad, float scale) {
+                                                        int Npad, float scale, long long tok_g) {
   const long long idx = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
   const long long total = (long long)B * N * H * D;
   if (idx >= total) return;
@@ -963,7 +965,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
   out.y = Elem<T>::pack(a.z * scale, a.w * scale);
   out.z = Elem<T>::pack(c.x * scale, c.y * scale);
   out.w = Elem<T>::pack(c.z * scale, c.w * scale);
-  *reinterpret_cast<uint4*>(dq + idx) = out;
+  *reinterpret_cast<uint4*>(dq + ((size_t)b * N + n) * tok_g + (size_t)h * D + x) = out;
 }
 
 // The three launches of one backward pass with scratch at ws (ws_bytes from
@@ -973,15 +975,17 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
                                    const CUtensorMap, const CUtensorMap, const BwdParams),
                       void* ws, const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                      int H, int N, float scale, unsigned flags, cudaStream_t stream, bool timed) {
+                      int H, int N, float scale, long long tok_in, long long tok_g,
+                      cudaStream_t stream, bool timed) {
   constexpr int D = Tr::D;
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM, (long long)H * D)) != FA_OK)
+    return rc;
   const int n_qt = (N + Tr::BM - 1) / Tr::BM;
   const int Npad = n_qt * Tr::BM;
   const size_t rows = (size_t)B * H * Npad;
@@ -998,6 +1002,7 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   p.N = N;
   p.Npad = Npad;
   p.n_qt = n_qt;
+  p.tok_g = tok_g;
   p.sl2 = scale * kLog2e;
   p.scale = scale;
   p.limit_ns = 4000000000ull;
@@ -1027,7 +1032,7 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   if (rc != FA_OK) return rc;
   const long long total = (long long)B * N * H * D;
   fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
-      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale);
+      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale, tok_g);
   note_launches(1);
   return launch_status(cudaGetLastError());
 }
@@ -1043,12 +1048,12 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
                                 const CUtensorMap, const CUtensorMap, const BwdParams),
                    const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
-                   unsigned flags, cudaStream_t stream) {
+                   long long tok_in, long long tok_g, cudaStream_t stream) {
   void* ws = nullptr;
   int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N), stream);
   if (rc != FA_OK) return rc;
-  rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags, stream,
-                         true);
+  rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in, tok_g,
+                         stream, true);
   scratch_free(ws, stream);
   return rc;
 }
@@ -1056,7 +1061,8 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-               float scale, unsigned flags, cudaStream_t stream) {
+               float scale, unsigned flags, long long tok_in, long long tok_g,
+               cudaStream_t stream) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
@@ -1064,13 +1070,13 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
     case 64:
       return run_bwd<T, BwdTraits64>((flags & 1u) ? fa_bwd_kernel<T, BwdTraits64, true>
                                                   : fa_bwd_kernel<T, BwdTraits64, false>,
-                                     q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags,
-                                     stream);
+                                     q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
+                                     tok_g, stream);
     case 128:
       return run_bwd<T, BwdTq128>((flags & 1u) ? fa_bwd_tq_kernel<T, BwdTq128, true>
                                                : fa_bwd_tq_kernel<T, BwdTq128, false>,
-                                  q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, flags,
-                                  stream);
+                                  q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
+                                  tok_g, stream);
     default:
       return FA_ERR_HEADDIM;
   }
@@ -1078,10 +1084,11 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
 
 template int bwd_launch<__nv_bfloat16>(const void*, const void*, const void*, const void*,
                                        const void*, const float*, void*, void*, void*, int, int,
-                                       int, int, float, unsigned, cudaStream_t);
+                                       int, int, float, unsigned, long long, long long,
+                                       cudaStream_t);
 template int bwd_launch<__half>(const void*, const void*, const void*, const void*, const void*,
                                 const float*, void*, void*, void*, int, int, int, int, float,
-                                unsigned, cudaStream_t);
+                                unsigned, long long, long long, cudaStream_t);
 
 // ------------------------------------------------------------------------
 // Fixed-scratch backward (fa_bwd_noalloc).  Same kernels as run_bwd, but the
@@ -1124,7 +1131,7 @@ static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, co
   int rc = fixed_scratch_address(&ws);
   if (rc != FA_OK) return rc;
   return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr, false>, ws, q, k, v, o, dout, lse, dq, dk, dv, B,
-                           H, N, scale, 0u, stream, false);
+                           H, N, scale, (long long)H * Tr::D, (long long)H * Tr::D, stream, false);
 }
 
 }  // namespace fa

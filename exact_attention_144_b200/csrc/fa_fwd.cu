@@ -1189,13 +1189,14 @@ int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces) {
 
 template <class T, int D, int BN, int THREADS, int SMEM, bool SPLIT_REGS, class Kernel>
 static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const void* k,
-                      const void* v, void* o, float* lse, float scale, cudaStream_t stream) {
+                      const void* v, void* o, float* lse, float scale, long long tok_in,
+                      cudaStream_t stream) {
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, s.B, s.N, s.H, D, 128)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, s.B, s.N, s.H, D, BN)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, s.B, s.N, s.H, D, BN)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, s.B, s.N, s.H, D, 128, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, s.B, s.N, s.H, D, BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, s.B, s.N, s.H, D, BN, tok_in)) != FA_OK) return rc;
 
   FwdParams p{};
   static_cast<FwdSchedule&>(p) = s;
@@ -1267,23 +1268,23 @@ static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const vo
 
 template <class T, class Tr>
 static int run_single(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
-                      float* lse, float scale, cudaStream_t stream) {
+                      float* lse, float scale, long long tok_in, cudaStream_t stream) {
   static_assert(Tr::BM == 128, "unit rows");
   return launch_fwd<T, Tr::D, Tr::BN, 224, Tr::SMEM_BYTES, false>(fa_fwd_kernel<T, Tr>, s, q, k,
-                                                                   v, o, lse, scale, stream);
+                                                                   v, o, lse, scale, tok_in, stream);
 }
 
 template <class T, class Tr>
 static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
-                  float* lse, float scale, cudaStream_t stream) {
+                  float* lse, float scale, long long tok_in, cudaStream_t stream) {
   static_assert(2 * Tr::BM == 256, "unit rows");
   return launch_fwd<T, Tr::D, Tr::BN, 384, Tr::SMEM_BYTES, true>(fa_fwd_pp_kernel<T, Tr>, s, q, k,
-                                                                 v, o, lse, scale, stream);
+                                                                 v, o, lse, scale, tok_in, stream);
 }
 
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, unsigned flags, cudaStream_t stream) {
+               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
@@ -1291,21 +1292,23 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = plan_fwd(B, H, N, d, flags, dev.sm_count, &s)) != FA_OK) return rc;
   switch (d) {
     case 64:
-      return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, stream)
-                    : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale, stream);
+      return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, tok_in, stream)
+                    : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale, tok_in,
+                                                               stream);
     case 128:
-      return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, stream)
-                    : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale, stream);
+      return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream)
+                    : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale, tok_in,
+                                                                stream);
     case 256:
-      return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, stream);
+      return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream);
     default:
       return FA_ERR_HEADDIM;
   }
 }
 
 template int fwd_launch<__nv_bfloat16>(const void*, const void*, const void*, void*, float*, int,
-                                       int, int, int, float, unsigned, cudaStream_t);
+                                       int, int, int, float, unsigned, long long, cudaStream_t);
 template int fwd_launch<__half>(const void*, const void*, const void*, void*, float*, int, int,
-                                int, int, float, unsigned, cudaStream_t);
+                                int, int, float, unsigned, long long, cudaStream_t);
 
 }  // namespace fa

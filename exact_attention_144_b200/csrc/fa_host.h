@@ -50,8 +50,10 @@ unsigned long long* device_status_ptr();
 // Tensor map over a contiguous [B, N, H, d] 16-bit tensor for TMA tile loads
 // of `box_rows` tokens x 64 elements of one head (128 bytes, 128-byte swizzle).
 // Rows past N are filled with zeros by the hardware.
+// tok_stride: elements from one token to the next (H*d for [B,N,H,d]; 3*H*d
+// for one of Q, K, V inside a packed [B,N,3,H,d] tensor).
 int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d,
-                   int box_rows);
+                   int box_rows, long long tok_stride);
 
 // Tensor map over a contiguous [rows, cols] fp32 matrix for TMA tiles of
 // box_rows x box_cols (box_cols * 4 = 128 bytes, 128-byte swizzle).
@@ -101,12 +103,15 @@ size_t fwd_scratch_bytes(const FwdSchedule& s);
 int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 
 // Launchers (argument validation is done by the callers in fa_api.cu).
+// tok_in: token stride of q, k, v (elements); tok_g: of dq, dk, dv.  o, lse,
+// dout are always contiguous [B,N,H,d] / [B,H,N].
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, unsigned flags, cudaStream_t stream);
+               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream);
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-               float scale, unsigned flags, cudaStream_t stream);
+               float scale, unsigned flags, long long tok_in, long long tok_g,
+               cudaStream_t stream);
 
 }  // namespace fa

@@ -132,6 +132,22 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
               cudaStream_t stream);
 
 /*
+ * Packed Q, K, V (the YOLOv12 image page's flash_attn_qkvpacked_func input):
+ * qkv is one contiguous [B, N, 3, H, d] device array of the element type
+ * `dtype` whose slices 0, 1, 2 along the third axis are Q, K, V (token stride
+ * 3*H*d).  fa_fwd_qkvpacked writes o [B,N,H,d] and lse [B,H,N] exactly as
+ * fa_fwd_ex on the three slices would; fa_bwd_qkvpacked takes o, dout
+ * [B,N,H,d] and lse and overwrites dqkv, a [B, N, 3, H, d] array holding dQ,
+ * dK, dV in the same slices.  Flags, errors and d as fa_fwd_ex / fa_bwd_ex;
+ * each of qkv and dqkv must hold fewer than 2^31 elements.
+ */
+int fa_fwd_qkvpacked(const void *qkv, void *o, float *lse, int B, int H, int N, int d,
+                     float scale, int dtype, unsigned flags, cudaStream_t stream);
+int fa_bwd_qkvpacked(const void *qkv, const void *o, const void *dout, const float *lse,
+                     void *dqkv, int B, int H, int N, int d, float scale, int dtype,
+                     unsigned flags, cudaStream_t stream);
+
+/*
  * Backward pass, bf16, for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it exists for hosts
  * such as plugin runtimes with their own static memory plan, code that runs
