@@ -58,8 +58,14 @@ def _load() -> ctypes.CDLL:
     lib.fa_bwd_ex.argtypes = [vp] * 9 + [i, i, i, i, f, i, ctypes.c_uint, vp]
     lib.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
     lib.fa_bwd_qkvpacked.argtypes = [vp] * 5 + [i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_fwd_varlen.argtypes = [vp] * 6 + [i, i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_bwd_varlen.argtypes = [vp] * 10 + [i, i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_varlen_bounds.argtypes = [ctypes.POINTER(ctypes.c_int), i, i, i,
+                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.fa_varlen_bounds.restype = i
     for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc", "fa_fwd_ex",
-              "fa_bwd_ex", "fa_fwd_qkvpacked", "fa_bwd_qkvpacked"):
+              "fa_bwd_ex", "fa_fwd_qkvpacked", "fa_bwd_qkvpacked", "fa_fwd_varlen",
+              "fa_bwd_varlen"):
         getattr(lib, n).restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -304,6 +310,72 @@ def fa_bwd_qkvpacked(qkv, o, dout, lse, dqkv=None, scale=None, flags=0, stream=N
     if rc != FA_OK:
         raise FAError("fa_bwd_qkvpacked", rc)
     return dqkv
+
+
+def _check_varlen(q, cu_seqlens, max_seqlen):
+    if q.dim() != 3:
+        raise ValueError("varlen q must be [total, H, d]")
+    if not (isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda and
+            cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and
+            cu_seqlens.is_contiguous() and cu_seqlens.numel() >= 2):
+        raise ValueError("cu_seqlens must be a contiguous int32 CUDA tensor of B + 1 entries")
+    if q.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported element type {q.dtype}")
+    total, H, d = q.shape
+    return cu_seqlens.numel() - 1, total, H, d, int(max_seqlen)
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, o=None, lse=None, scale=None, flags=0,
+                  stream=None):
+    """Forward over B sequences packed along the token axis: q, k, v are
+    [total, H, d], cu_seqlens (int32, B + 1) their starts.  Returns (o [total,
+    H, d], lse [H, total])."""
+    B, total, H, d, ms = _check_varlen(q, cu_seqlens, max_seqlen)
+    for name, t in (("k", k), ("v", v)):
+        _check_bnhd(name, t, q.dtype, q.shape)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((H, total), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_bnhd("o", o, q.dtype, q.shape)
+    _check_bnhd("lse", lse, torch.float32, (H, total))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = _load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B,
+                               total, ms, H, d, float(scale), _DTYPE_CODE[q.dtype], int(flags),
+                               _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_varlen", rc)
+    return o, lse
+
+
+def fa_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens, max_seqlen, dq=None, dk=None, dv=None,
+                  scale=None, flags=0, stream=None):
+    """Backward of fa_fwd_varlen; returns (dq, dk, dv), each [total, H, d]."""
+    B, total, H, d, ms = _check_varlen(q, cu_seqlens, max_seqlen)
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_bnhd(name, t, q.dtype, q.shape)
+    _check_bnhd("lse", lse, torch.float32, (H, total))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bnhd(name, t, q.dtype, q.shape)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = _load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), B, total, ms, H, d,
+                               float(scale), _DTYPE_CODE[q.dtype], int(flags), _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_bwd_varlen", rc)
+    return dq, dk, dv
+
+
+def fa_varlen_bounds(cu_seqlens, b: int, max_seqlen: int, total: int) -> tuple:
+    """(first token, length) the varlen kernels use for sequence b, from a
+    host list of cu_seqlens (the clamping rule, evaluated on the host)."""
+    arr = (ctypes.c_int * len(cu_seqlens))(*cu_seqlens)
+    t0, n = ctypes.c_int(0), ctypes.c_int(0)
+    rc = _load().fa_varlen_bounds(arr, b, max_seqlen, total, ctypes.byref(t0), ctypes.byref(n))
+    if rc != FA_OK:
+        raise FAError("fa_varlen_bounds", rc)
+    return t0.value, n.value
 
 
 def forward(q, k, v, scale=None, o=None, lse=None, stream=None, causal=False):

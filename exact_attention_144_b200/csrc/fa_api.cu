@@ -275,6 +275,44 @@ static int bwd_packed_entry(const void* qkv, const void* o, const void* dout, co
                        N, d, scale, flags, 3 * hd, 3 * hd, stream);
 }
 
+// Variable-length batch: B sequences packed along one token axis of `total`
+// tokens ([total, H, d] tensors, lse [H, total]); cu_seqlens (device, B + 1
+// entries) holds each sequence's first token, max_seqlen bounds their lengths.
+static int check_varlen(const int* cu, int B, int total, int max_seqlen, int H, int d,
+                        float scale, bool bwd) {
+  if (cu == nullptr) return FA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return FA_ERR_ALIGN;
+  if (total < 1 || max_seqlen < 1) return FA_ERR_SHAPE;
+  int rc = check_common(B, H, max_seqlen, d, scale, bwd);
+  if (rc == FA_OK && (long long)total * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
+  return rc;
+}
+
+template <class T>
+static int fwd_varlen_entry(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu, int B, int total, int max_seqlen, int H, int d,
+                            float scale, unsigned flags, cudaStream_t stream) {
+  int rc = check_ptrs({q, k, v, o, lse});
+  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale, false);
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc != FA_OK) return rc;
+  return fwd_launch<T>(q, k, v, o, lse, B, H, max_seqlen, d, scale, flags, (long long)H * d,
+                       stream, cu, total);
+}
+
+template <class T>
+static int bwd_varlen_entry(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            const int* cu, int B, int total, int max_seqlen, int H, int d,
+                            float scale, unsigned flags, cudaStream_t stream) {
+  int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
+  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale, true);
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc != FA_OK) return rc;
+  return bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, max_seqlen, d, scale, flags,
+                       (long long)H * d, (long long)H * d, stream, cu, total);
+}
+
 int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale) {
@@ -359,6 +397,40 @@ FA_EXPORT int fa_bwd_qkvpacked(const void* qkv, const void* o, const void* dout,
   if (dtype == FA_FP16)
     return fa::bwd_packed_entry<__half>(qkv, o, dout, lse, dqkv, B, H, N, d, scale, flags, stream);
   return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens, int B, int total, int max_seqlen, int H, int d,
+                            float scale, int dtype, unsigned flags, cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::fwd_varlen_entry<__nv_bfloat16>(q, k, v, o, lse, cu_seqlens, B, total, max_seqlen,
+                                               H, d, scale, flags, stream);
+  if (dtype == FA_FP16)
+    return fa::fwd_varlen_entry<__half>(q, k, v, o, lse, cu_seqlens, B, total, max_seqlen, H, d,
+                                        scale, flags, stream);
+  return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            const int* cu_seqlens, int B, int total, int max_seqlen, int H, int d,
+                            float scale, int dtype, unsigned flags, cudaStream_t stream) {
+  if (dtype == FA_BF16)
+    return fa::bwd_varlen_entry<__nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens, B,
+                                               total, max_seqlen, H, d, scale, flags, stream);
+  if (dtype == FA_FP16)
+    return fa::bwd_varlen_entry<__half>(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens, B, total,
+                                        max_seqlen, H, d, scale, flags, stream);
+  return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_varlen_bounds(const int* cu_seqlens_host, int b, int max_seqlen, int total,
+                               int* tok0, int* len) {
+  if (cu_seqlens_host == nullptr || tok0 == nullptr || len == nullptr) return FA_ERR_NULL;
+  if (b < 0 || max_seqlen < 1 || total < 1) return FA_ERR_SHAPE;
+  int tb = 0;
+  fa::seq_bounds(cu_seqlens_host, b, max_seqlen, total, tb, *tok0, *len);
+  return FA_OK;
 }
 
 FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

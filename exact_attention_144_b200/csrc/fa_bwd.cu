@@ -80,8 +80,10 @@ struct BwdParams {
   float* dq_acc;      // [B, H, Npad, D] fp32
   void* dk;           // [B, N, H, D]
   void* dv;
-  int B, H, N, Npad, n_qt;
+  int B, H, N, Npad, n_qt;  // varlen: B sequences, N = max_seqlen
   long long tok_g;    // token stride of dk, dv (elements): H*D, or 3*H*D when packed
+  const int* cu;      // varlen: device [B+1] sequence starts on the token axis; else null
+  int total;          // tokens a batch entry holds in memory: N, or all tokens (varlen)
   float sl2;          // scale * log2(e)
   float scale;
   unsigned long long limit_ns;
@@ -126,7 +128,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <class T, class Tr, bool CAUSAL>
+template <class T, class Tr, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -150,9 +152,14 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
+  // tok0 + len); a key tile past a shorter sequence's end has no work
+  int tb, tok0, len;
+  seq_bounds(VARLEN ? p.cu : nullptr, b, p.N, p.total, tb, tok0, len);
+  if (kt * BN >= len) return;  // block-uniform, before any barrier or allocation
   // causal: query tiles wholly before this key tile see none of its keys
   const int i0 = CAUSAL ? (kt * BN) / BM : 0;
-  const int n_qt = p.n_qt - i0;  // query tiles this block visits; tile i is global tile i0 + i
+  const int n_qt = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - i0;  // tile i is global i0 + i
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -188,8 +195,8 @@ __global__ void __launch_bounds__(384, 1)
     {
       const bool leader = lane == 0;  // issues; all lanes run the loop
       mbar_expect_tx(leader, bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
-      tma_load_4d(leader, sK, &tmk, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
-      tma_load_4d(leader, sV, &tmv, bar(Tr::B_KV_FULL), 0, h, kt * BN, b);
+      tma_load_4d(leader, sK, &tmk, bar(Tr::B_KV_FULL), 0, h, tok0 + kt * BN, tb);
+      tma_load_4d(leader, sV, &tmv, bar(Tr::B_KV_FULL), 0, h, tok0 + kt * BN, tb);
       const size_t row0 = ((size_t)b * p.H + h) * p.Npad;
       int issued = 0;
       for (int i = 0; i < n_qt; ++i) {
@@ -199,8 +206,8 @@ __global__ void __launch_bounds__(384, 1)
           break;
         const uint32_t fb = bar(Tr::B_Q_FULL + qs);
         mbar_expect_tx(leader, fb, 2 * Tr::QT_BYTES + 2 * BM * 4);
-        tma_load_4d(leader, sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, (i0 + i) * BM, b);
-        tma_load_4d(leader, sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, (i0 + i) * BM, b);
+        tma_load_4d(leader, sQ + qs * Tr::QT_BYTES, &tmq, fb, 0, h, tok0 + (i0 + i) * BM, tb);
+        tma_load_4d(leader, sDO + qs * Tr::QT_BYTES, &tmdo, fb, 0, h, tok0 + (i0 + i) * BM, tb);
         bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)(i0 + i) * BM,
                   BM * 4, fb);
         bulk_load(leader, base + Tr::OFF_DD + qs * BM * 4, p.dvec + row0 + (size_t)(i0 + i) * BM,
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(384, 1)
     const int quad = warp & 3, hf = warp >> 2;
     const int r = quad * 32 + lane;  // key row (S^T, dP^T) and query row (dQ)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    const bool key_valid = kt * BN + r < p.N;
+    const bool key_valid = kt * BN + r < len;
     const float c = p.sl2;
     bool ok = true;
 
@@ -456,7 +463,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = ((size_t)b * p.N + key) * p.tok_g + (size_t)h * D + hf * 32;
+      const size_t off = ((size_t)tb * p.total + tok0 + key) * p.tok_g + (size_t)h * D + hf * 32;
       uint32_t a[32], k2[32];
       tmem_ld32(tl + Tr::TM_DV + hf * 32, a);
       tmem_ld32(tl + Tr::TM_DK + hf * 32, k2);
@@ -549,7 +556,7 @@ struct BwdTqTraits {
 
 using BwdTq128 = BwdTqTraits<128, 3>;
 
-template <class T, class Tr, bool CAUSAL>
+template <class T, class Tr, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_tq_kernel(const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk,
@@ -574,9 +581,14 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
+  // tok0 + len); a key tile past a shorter sequence's end has no work
+  int tb, tok0, len;
+  seq_bounds(VARLEN ? p.cu : nullptr, b, p.N, p.total, tb, tok0, len);
+  if (kt * BN >= len) return;  // block-uniform, before any barrier or allocation
   // causal: query tiles wholly before this key tile see none of its keys
   const int i0 = CAUSAL ? (kt * BN) / BM : 0;
-  const int n_qt = p.n_qt - i0;  // query tiles this block visits; tile i is global tile i0 + i
+  const int n_qt = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - i0;  // tile i is global i0 + i
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -621,8 +633,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_expect_tx(leader, bar(Tr::B_KV_FULL), 2 * Tr::KV_BYTES);
 #pragma unroll
       for (int c = 0; c < KCH; ++c) {
-        tma_load_4d(leader, sK + c * (BN * 128), &tmk, bar(Tr::B_KV_FULL), c * 64, h, kt * BN, b);
-        tma_load_4d(leader, sV + c * (BN * 128), &tmv, bar(Tr::B_KV_FULL), c * 64, h, kt * BN, b);
+        tma_load_4d(leader, sK + c * (BN * 128), &tmk, bar(Tr::B_KV_FULL), c * 64, h,
+                    tok0 + kt * BN, tb);
+        tma_load_4d(leader, sV + c * (BN * 128), &tmv, bar(Tr::B_KV_FULL), c * 64, h,
+                    tok0 + kt * BN, tb);
       }
       const size_t row0 = ((size_t)b * p.H + h) * p.Npad;
       int issued = 0;
@@ -636,9 +650,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < KCH; ++c) {
           tma_load_4d(leader, sQ + qs * Tr::QT_BYTES + c * (BM * 128), &tmq, fb, c * 64, h,
-                      (i0 + i) * BM, b);
+                      tok0 + (i0 + i) * BM, tb);
           tma_load_4d(leader, sDO + qs * Tr::QT_BYTES + c * (BM * 128), &tmdo, fb, c * 64, h,
-                      (i0 + i) * BM, b);
+                      tok0 + (i0 + i) * BM, tb);
         }
         bulk_load(leader, base + Tr::OFF_L + qs * BM * 4, p.lse2 + row0 + (size_t)(i0 + i) * BM,
                   BM * 4, fb);
@@ -743,7 +757,7 @@ __global__ void __launch_bounds__(384, 1)
     const int quad = warp & 3, hf = warp >> 2;
     const int r = quad * 32 + lane;  // key row (S^T, dP^T), d row (dQ^T)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    const bool key_valid = kt * BN + r < p.N;
+    const bool key_valid = kt * BN + r < len;
     const float c = p.sl2;
     const uint32_t box = sSTG + warp * Tr::BOX_BYTES;
     uint8_t* gbox = gSTG + warp * Tr::BOX_BYTES;
@@ -864,7 +878,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = ((size_t)b * p.N + key) * p.tok_g + (size_t)h * D;
+      const size_t off = ((size_t)tb * p.total + tok0 + key) * p.tok_g + (size_t)h * D;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
         const int col = hf * (D / 2) + cc * 32;
@@ -904,9 +918,10 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// D_i = sum_x dO_ix O_ix; minus the base-2 LSE; zero the dQ accumulator.  One
-// warp per padded row (b, h, i); rows past N get D = 0 and -LSE = -inf (so
-// P = 0 there).
+// D_i = sum_x dO_ix O_ix; minus the base-2 LSE; zero the dQ accumulator.
+// Accumulator rows are (b, h, i) with i < Npad for every sequence b; rows past
+// the sequence's length get D = 0 and -LSE = -inf (so P = 0 there).  D / 8
+// lanes take one row, 16 bytes of O and of dO each.
 template <class T, int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o,
                                                          const T* __restrict__ dout,
@@ -914,58 +929,71 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
                                                          float* __restrict__ lse2,
                                                          float* __restrict__ dvec,
                                                          float* __restrict__ dq_acc, int B, int H,
-                                                         int N, int Npad) {
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= (long long)B * H * Npad) return;
-  const int i = (int)(row % Npad);
-  const int h = (int)((row / Npad) % H);
-  const int b = (int)(row / ((long long)Npad * H));
-  constexpr int PER = D / 32;
+                                                         int N, int Npad, const int* cu,
+                                                         int total) {
+  constexpr int LPR = D / 8;     // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp
+  const int lane = threadIdx.x & 31, sub = lane % LPR;
+  const long long row = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
+  const bool in = row < (long long)B * H * Npad;
+  int i = 0, h = 0, tb = 0, tok0 = 0, len = 0;
   float acc = 0.f;
-  if (i < N) {
-    const T* orow = o + (((size_t)b * N + i) * H + h) * D + lane * PER;
-    const T* drow = dout + (((size_t)b * N + i) * H + h) * D + lane * PER;
+  if (in) {
+    i = (int)(row % Npad);
+    h = (int)((row / Npad) % H);
+    const int b = (int)(row / ((long long)Npad * H));
+    seq_bounds(cu, b, N, total, tb, tok0, len);
+    if (i < len) {
+      const size_t at = (((size_t)tb * total + tok0 + i) * H + h) * D + sub * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(o + at);
+      const uint4 c = *reinterpret_cast<const uint4*>(dout + at);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int j = 0; j < PER; j += 2) {
-      const float2 a = Elem<T>::unpack(*reinterpret_cast<const uint32_t*>(orow + j));
-      const float2 c = Elem<T>::unpack(*reinterpret_cast<const uint32_t*>(drow + j));
-      acc += a.x * c.x + a.y * c.y;
+      for (int j = 0; j < 4; ++j) {
+        const float2 x = Elem<T>::unpack(aw[j]), y = Elem<T>::unpack(cw[j]);
+        acc += x.x * y.x + x.y * y.y;
+      }
     }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  float* arow = dq_acc + (size_t)row * D + lane * PER;
-#pragma unroll
-  for (int j = 0; j < PER; ++j) arow[j] = 0.f;
-  if (lane == 0) {
-    dvec[row] = acc;
-    lse2[row] = (i < N) ? -(lse[((size_t)b * H + h) * N + i] * kLog2e) : -INFINITY;
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (in) {
+    float4* arow = reinterpret_cast<float4*>(dq_acc + (size_t)row * D + sub * 8);
+    arow[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    arow[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sub == 0) {
+      dvec[row] = acc;
+      lse2[row] = (i < len) ? -(lse[((size_t)tb * H + h) * total + tok0 + i] * kLog2e) : -INFINITY;
+    }
   }
 }
 
-// dQ = scale * accumulator, rounded; 8 elements per thread.  dq rows are
-// tok_g elements apart (H*D, or 3*H*D inside a packed dQKV).
+// dQ = scale * accumulator, rounded; 8 elements per thread, over the
+// accumulator rows (b, h, i < Npad), written for i below the sequence length.
+// dq rows are tok_g elements apart (H*D, or 3*H*D inside a packed dQKV).
 template <class T, int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dq_acc,
                                                         T* __restrict__ dq, int B, int H, int N,
-                                                        int Npad, float scale, long long tok_g) {
-  const long long idx = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
-  const long long total = (long long)B * N * H * D;
-  if (idx >= total) return;
-  const int x = (int)(idx % D);
-  const int h = (int)((idx / D) % H);
-  const int n = (int)((idx / ((long long)D * H)) % N);
-  const int b = (int)(idx / ((long long)D * H * N));
-  const float* src = dq_acc + (((size_t)b * H + h) * Npad + n) * D + x;
-  const float4 a = *reinterpret_cast<const float4*>(src);
-  const float4 c = *reinterpret_cast<const float4*>(src + 4);
+                                                        int Npad, float scale, long long tok_g,
+                                                        const int* cu, int total) {
+  const long long e = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
+  if (e >= (long long)B * H * Npad * D) return;
+  const long long row = e / D;
+  const int x = (int)(e % D);
+  const int i = (int)(row % Npad);
+  const int h = (int)((row / Npad) % H);
+  const int b = (int)(row / ((long long)Npad * H));
+  int tb, tok0, len;
+  seq_bounds(cu, b, N, total, tb, tok0, len);
+  if (i >= len) return;
+  const float4 a = *reinterpret_cast<const float4*>(dq_acc + e);
+  const float4 c = *reinterpret_cast<const float4*>(dq_acc + e + 4);
   uint4 out;
   out.x = Elem<T>::pack(a.x * scale, a.y * scale);
   out.y = Elem<T>::pack(a.z * scale, a.w * scale);
   out.z = Elem<T>::pack(c.x * scale, c.y * scale);
   out.w = Elem<T>::pack(c.z * scale, c.w * scale);
-  *reinterpret_cast<uint4*>(dq + ((size_t)b * N + n) * tok_g + (size_t)h * D + x) = out;
+  *reinterpret_cast<uint4*>(dq + ((size_t)tb * total + tok0 + i) * tok_g + (size_t)h * D + x) = out;
 }
 
 // The three launches of one backward pass with scratch at ws (ws_bytes from
@@ -976,15 +1004,18 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
                       void* ws, const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                       int H, int N, float scale, long long tok_in, long long tok_g,
-                      cudaStream_t stream, bool timed) {
+                      cudaStream_t stream, bool timed, const int* cu, int total) {
   constexpr int D = Tr::D;
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, B, N, H, D, Tr::BM, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, B, N, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, B, N, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, B, N, H, D, Tr::BM, (long long)H * D)) != FA_OK)
+  // memory view: B batch entries of N tokens, or one entry of all tokens (varlen)
+  if (cu == nullptr) total = N;
+  const int mB = cu ? 1 : B;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, mB, total, H, D, Tr::BM, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, mB, total, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, mB, total, H, D, Tr::BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmdo, dout, bf16, mB, total, H, D, Tr::BM, (long long)H * D)) != FA_OK)
     return rc;
   const int n_qt = (N + Tr::BM - 1) / Tr::BM;
   const int Npad = n_qt * Tr::BM;
@@ -1003,6 +1034,8 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   p.Npad = Npad;
   p.n_qt = n_qt;
   p.tok_g = tok_g;
+  p.cu = cu;
+  p.total = total;
   p.sl2 = scale * kLog2e;
   p.scale = scale;
   p.limit_ns = 4000000000ull;
@@ -1016,9 +1049,11 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
 
   // The pre-pass rewrites every scratch word the pass reads (it zeroes the
   // accumulator), so earlier contents of the scratch never leak in.
-  fa_bwd_pre_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H, N,
-      Npad);
+  constexpr int kPreRowsPerBlock = 8 * (32 / (D / 8));
+  fa_bwd_pre_kernel<T, D>
+      <<<(unsigned)((rows + kPreRowsPerBlock - 1) / kPreRowsPerBlock), 256, 0, stream>>>(
+          static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H,
+          N, Npad, cu, total);
   note_launches(1);
   if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
@@ -1030,9 +1065,9 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);
   if (rc != FA_OK) return rc;
-  const long long total = (long long)B * N * H * D;
-  fa_bwd_dq_kernel<T, D><<<(unsigned)((total / 8 + 255) / 256), 256, 0, stream>>>(
-      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale, tok_g);
+  const long long acc_elems = (long long)rows * D;
+  fa_bwd_dq_kernel<T, D><<<(unsigned)((acc_elems / 8 + 255) / 256), 256, 0, stream>>>(
+      p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale, tok_g, cu, total);
   note_launches(1);
   return launch_status(cudaGetLastError());
 }
@@ -1048,12 +1083,13 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
                                 const CUtensorMap, const CUtensorMap, const BwdParams),
                    const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
-                   long long tok_in, long long tok_g, cudaStream_t stream) {
+                   long long tok_in, long long tok_g, cudaStream_t stream, const int* cu,
+                   int total) {
   void* ws = nullptr;
   int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N), stream);
   if (rc != FA_OK) return rc;
   rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in, tok_g,
-                         stream, true);
+                         stream, true, cu, total);
   scratch_free(ws, stream);
   return rc;
 }
@@ -1062,21 +1098,27 @@ template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                float scale, unsigned flags, long long tok_in, long long tok_g,
-               cudaStream_t stream) {
+               cudaStream_t stream, const int* cu, int total) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
   switch (d) {
-    case 64:
-      return run_bwd<T, BwdTraits64>((flags & 1u) ? fa_bwd_kernel<T, BwdTraits64, true>
-                                                  : fa_bwd_kernel<T, BwdTraits64, false>,
-                                     q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
-                                     tok_g, stream);
-    case 128:
-      return run_bwd<T, BwdTq128>((flags & 1u) ? fa_bwd_tq_kernel<T, BwdTq128, true>
-                                               : fa_bwd_tq_kernel<T, BwdTq128, false>,
-                                  q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
-                                  tok_g, stream);
+    case 64: {
+      auto kern = (flags & 1u) ? (cu ? fa_bwd_kernel<T, BwdTraits64, true, true>
+                                     : fa_bwd_kernel<T, BwdTraits64, true, false>)
+                               : (cu ? fa_bwd_kernel<T, BwdTraits64, false, true>
+                                     : fa_bwd_kernel<T, BwdTraits64, false, false>);
+      return run_bwd<T, BwdTraits64>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale,
+                                     tok_in, tok_g, stream, cu, total);
+    }
+    case 128: {
+      auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq128, true, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq128, true, false>)
+                               : (cu ? fa_bwd_tq_kernel<T, BwdTq128, false, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq128, false, false>);
+      return run_bwd<T, BwdTq128>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
+                                  tok_g, stream, cu, total);
+    }
     default:
       return FA_ERR_HEADDIM;
   }
@@ -1085,10 +1127,10 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
 template int bwd_launch<__nv_bfloat16>(const void*, const void*, const void*, const void*,
                                        const void*, const float*, void*, void*, void*, int, int,
                                        int, int, float, unsigned, long long, long long,
-                                       cudaStream_t);
+                                       cudaStream_t, const int*, int);
 template int bwd_launch<__half>(const void*, const void*, const void*, const void*, const void*,
                                 const float*, void*, void*, void*, int, int, int, int, float,
-                                unsigned, long long, long long, cudaStream_t);
+                                unsigned, long long, long long, cudaStream_t, const int*, int);
 
 // ------------------------------------------------------------------------
 // Fixed-scratch backward (fa_bwd_noalloc).  Same kernels as run_bwd, but the
@@ -1130,8 +1172,9 @@ static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, co
   void* ws = nullptr;
   int rc = fixed_scratch_address(&ws);
   if (rc != FA_OK) return rc;
-  return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr, false>, ws, q, k, v, o, dout, lse, dq, dk, dv, B,
-                           H, N, scale, (long long)H * Tr::D, (long long)H * Tr::D, stream, false);
+  return launch_bwd<T, Tr>(fa_bwd_kernel<T, Tr, false, false>, ws, q, k, v, o, dout, lse, dq, dk, dv, B,
+                           H, N, scale, (long long)H * Tr::D, (long long)H * Tr::D, stream, false,
+                           nullptr, N);
 }
 
 }  // namespace fa

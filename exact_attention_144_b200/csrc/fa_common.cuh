@@ -395,6 +395,27 @@ __device__ __forceinline__ void ex2_poly2(float& y0, float& y1, float x0, float 
   y1 = __uint_as_float(ph + (th << 23));
 }
 
+// Where sequence b lies on the token axis.  Fixed length (cu null): batch
+// entry b, tokens [0, N).  Varlen: tokens [cu[b], cu[b+1]) of the one packed
+// batch entry, clamped into [0, total) and to at most N (max_seqlen) tokens,
+// so that no contents of cu can send an access out of bounds.
+__host__ __device__ __forceinline__ void seq_bounds(const int* cu, int b, int N, int total,
+                                                   int& tb, int& tok0, int& len) {
+  if (cu == nullptr) {
+    tb = b;
+    tok0 = 0;
+    len = N;
+    return;
+  }
+  int st = cu[b], en = cu[b + 1];
+  st = st < 0 ? 0 : (st > total ? total : st);
+  const int lim = (st + N < total) ? st + N : total;
+  en = en < st ? st : (en > lim ? lim : en);
+  tb = 0;
+  tok0 = st;
+  len = en - st;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

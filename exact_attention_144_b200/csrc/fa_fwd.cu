@@ -50,6 +50,9 @@ enum : int {
 struct Unit {
   int u;  // unit index
   int b, h, qt, sp, t0, t1;
+  int tb;    // batch coordinate of the unit's rows in memory (0 for a varlen batch)
+  int tok0;  // first token of the unit's sequence along the token axis (varlen)
+  int len;   // tokens in the unit's sequence
   int kind, peer0, npeer;
 };
 
@@ -60,6 +63,12 @@ __host__ __device__ __forceinline__ int range_begin(const FwdSchedule& s, int c)
   return c * s.iter_per + imin(c, s.iter_rem);
 }
 
+__host__ __device__ __forceinline__ void locate_seq(const FwdSchedule& s, int b, int& tb,
+                                                   int& tok0, int& len) {
+  seq_bounds(s.cu, b, s.N, s.total, tb, tok0, len);
+}
+
+// Unit u; t1 <= t0 when the unit holds no query row of its sequence (varlen).
 __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s) {
   Unit x;
   x.u = u;
@@ -73,9 +82,10 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
     x.sp = 0;
     x.h = bh % s.H;
     x.b = bh / s.H;
+    locate_seq(s, x.b, x.tb, x.tok0, x.len);
     x.t0 = 0;
-    const int rows_end = imin(s.N, (x.qt + 1) * s.unit_rows);
-    x.t1 = (rows_end + s.bn - 1) / s.bn;
+    const int rows_end = imin(x.len, (x.qt + 1) * s.unit_rows);
+    x.t1 = x.qt * s.unit_rows < x.len ? (rows_end + s.bn - 1) / s.bn : 0;
     return x;
   }
   x.qt = u % s.n_qt;
@@ -84,8 +94,10 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
   r /= s.n_split;
   x.h = r % s.H;
   x.b = r / s.H;
+  locate_seq(s, x.b, x.tb, x.tok0, x.len);
   x.t0 = x.sp * s.kvt_per_split;
-  x.t1 = imin(x.t0 + s.kvt_per_split, s.n_kvt);
+  x.t1 = imin(x.t0 + s.kvt_per_split, (x.len + s.bn - 1) / s.bn);
+  if (x.qt * s.unit_rows >= x.len) x.t1 = x.t0;  // no query row of this sequence
   return x;
 }
 
@@ -117,19 +129,25 @@ struct UnitIter {
   }
   __host__ __device__ __forceinline__ bool next(const FwdSchedule& s, Unit& x) {
     if (s.n_iter == 0 && s.causal) {
-      // a unit past the end in one wave means none in later waves either
-      const int u = i * s.grid + ((i & 1) ? s.grid - 1 - blk : blk);
-      if (u >= end) return false;
-      x = decode_unit(u, s);
-      ++i;
-      return true;
+      // a unit past the end in one wave means none in later waves either;
+      // units without query rows (varlen) are skipped by every role alike
+      for (;;) {
+        const int u = i * s.grid + ((i & 1) ? s.grid - 1 - blk : blk);
+        if (u >= end) return false;
+        x = decode_unit(u, s);
+        ++i;
+        if (x.t1 > x.t0) return true;
+      }
+    }
+    if (s.n_iter == 0) {
+      for (;;) {
+        if (i >= end) return false;
+        x = decode_unit(i, s);
+        i += s.grid;
+        if (x.t1 > x.t0) return true;
+      }
     }
     if (i >= end) return false;
-    if (s.n_iter == 0) {
-      x = decode_unit(i, s);
-      i += s.grid;
-      return true;
-    }
     const int u = i / s.n_kvt;
     const int ubeg = u * s.n_kvt, uend = ubeg + s.n_kvt;
     x = decode_unit(u, s);  // n_split = 1: the whole K/V range
@@ -304,7 +322,10 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
 template <class T, int D>
 __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, uint32_t taddr,
                                           int q_row, float m, float l, const WaitCtl& w) {
-  const bool live = q_row < p.N;
+  const bool live = q_row < un.len;
+  // the row's token along the memory token axis (p.total tokens a batch entry)
+  const size_t tok = (size_t)un.tb * p.total + un.tok0 + q_row;
+  const size_t lse_at = ((size_t)un.tb * p.H + un.h) * p.total + un.tok0 + q_row;
   const float inv_l = 1.f / l;
   const float lse2 = m + lg2(l);
   if (un.kind == kStorePartial) {
@@ -360,7 +381,7 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
         tot += ex2(__ldcg(p.bal_lse + (size_t)c * p.unit_rows + ur) - mx);
     const float L2 = mx + lg2(tot);
     const float w_own = ex2(lse2 - L2) * inv_l;
-    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
+    T* orow = reinterpret_cast<T*>(p.o) + (tok * p.H + un.h) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -393,11 +414,11 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
         for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
       }
     }
-    if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = L2 * kLn2;
+    if (live) p.lse[lse_at] = L2 * kLn2;
     return true;
   }
   if (p.o_part == nullptr) {
-    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)un.b * p.N + q_row) * p.H + un.h) * D;
+    T* orow = reinterpret_cast<T*>(p.o) + (tok * p.H + un.h) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -416,7 +437,7 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
         for (int j = 0; j < 4; ++j) dst[j] = pkd[j];
       }
     }
-    if (live) p.lse[((size_t)un.b * p.H + un.h) * p.N + q_row] = lse2 * kLn2;
+    if (live) p.lse[lse_at] = lse2 * kLn2;
   } else {
     float* orow = p.o_part + ((((size_t)un.sp * p.B + un.b) * p.N + q_row) * p.H + un.h) * D;
 #pragma unroll
@@ -548,7 +569,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64,
-                        un.h, (2 * un.qt + t) * BM, un.b);
+                        un.h, un.tok0 + (2 * un.qt + t) * BM, un.tb);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t ks = kc % KST;
@@ -559,7 +580,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
-                        c * 64, un.h, t * BN, un.b);
+                        c * 64, un.h, un.tok0 + t * BN, un.tb);
           ++kc;
           const uint32_t vs = vc % VST;
           if (vc >= (uint32_t)VST &&
@@ -569,7 +590,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
-                        c * 64, un.h, t * BN, un.b);
+                        c * 64, un.h, un.tok0 + t * BN, un.tb);
           ++vc;
         }
       }
@@ -750,7 +771,7 @@ __global__ void __launch_bounds__(384, 1)
         // key columns this row sees in K/V tile t: below N, and with the
         // causal mask up to the row's own position
         const int t = un.t0 + j;
-        int valid = p.N - t * BN;
+        int valid = un.len - t * BN;
         if (p.causal) valid = imin(valid, (2 * un.qt + wg) * BM + row - t * BN + 1);
         const float alpha = softmax_step<T, BN, Tr::EMU>(r, valid, c, m, l, pk);
         if constexpr (Tr::SEP_P) {
@@ -893,7 +914,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int c = 0; c < Tr::KCH; ++c)
           tma_load_4d(leader, sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64, un.h,
-                      un.qt * Tr::BM, un.b);
+                      un.tok0 + un.qt * Tr::BM, un.tb);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t ks = kc % KST;
@@ -904,7 +925,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
-                        c * 64, un.h, t * BN, un.b);
+                        c * 64, un.h, un.tok0 + t * BN, un.tb);
           ++kc;
         }
       }
@@ -931,7 +952,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
-                        c * 64, un.h, t * BN, un.b);
+                        c * 64, un.h, un.tok0 + t * BN, un.tb);
           ++vc;
         }
       }
@@ -1024,7 +1045,7 @@ __global__ void __launch_bounds__(224, 1)
         for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
         uint32_t pk[BN / 2];
         const int t = un.t0 + i;
-        int valid = p.N - t * BN;
+        int valid = un.len - t * BN;
         if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
         const float alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
 #pragma unroll
@@ -1132,6 +1153,9 @@ int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedu
   x.N = N;
   x.d = d;
   x.causal = (flags & 1u) ? 1 : 0;
+  x.cu = nullptr;
+  x.total = N;
+  const bool varlen = (flags & kPlanVarlen) != 0;
   // Two Q tiles per unit once a head has more than one tile's worth of rows;
   // a single tile per unit for short sequences and for d = 256 (whose O
   // accumulator leaves tensor memory room for only one Q tile).
@@ -1144,12 +1168,13 @@ int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedu
   if (base_units >= (1ll << 31)) return FA_ERR_SHAPE;
   // causal units differ in length: they are neither split nor cut, and run
   // longest first (decode_unit)
-  int n_split = x.causal ? 1 : choose_splits(base_units, x.n_kvt, sm_count);
+  int n_split = (x.causal || varlen) ? 1 : choose_splits(base_units, x.n_kvt, sm_count);
   x.kvt_per_split = (x.n_kvt + n_split - 1) / n_split;
   x.n_split = (x.n_kvt + x.kvt_per_split - 1) / x.kvt_per_split;  // no empty split
   x.n_units = (int)(base_units * x.n_split);
   const bool balanced =
-      !x.causal && x.pair && x.n_split == 1 && use_balanced(base_units, x.n_kvt, sm_count);
+      !x.causal && !varlen && x.pair && x.n_split == 1 &&
+      use_balanced(base_units, x.n_kvt, sm_count);
   x.grid = balanced ? sm_count : (x.n_units < sm_count ? x.n_units : sm_count);
   if (balanced) {
     x.n_iter = (int)(base_units * x.n_kvt);
@@ -1194,9 +1219,11 @@ static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const vo
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv;
   int rc;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, s.B, s.N, s.H, D, 128, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, s.B, s.N, s.H, D, BN, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, s.B, s.N, s.H, D, BN, tok_in)) != FA_OK) return rc;
+  // memory view: B batch entries of N tokens, or one entry of all tokens (varlen)
+  const int mB = s.cu ? 1 : s.B, mN = s.total;
+  if ((rc = make_tmap_bnhd(&tmq, q, bf16, mB, mN, s.H, D, 128, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, bf16, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, bf16, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
 
   FwdParams p{};
   static_cast<FwdSchedule&>(p) = s;
@@ -1284,12 +1311,18 @@ static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void
 
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream) {
+               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream,
+               const int* cu, int total) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
   FwdSchedule s;
-  if ((rc = plan_fwd(B, H, N, d, flags, dev.sm_count, &s)) != FA_OK) return rc;
+  if ((rc = plan_fwd(B, H, N, d, flags | (cu ? kPlanVarlen : 0u), dev.sm_count, &s)) != FA_OK)
+    return rc;
+  if (cu != nullptr) {
+    s.cu = cu;
+    s.total = total;
+  }
   switch (d) {
     case 64:
       return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, tok_in, stream)
@@ -1307,8 +1340,10 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
 }
 
 template int fwd_launch<__nv_bfloat16>(const void*, const void*, const void*, void*, float*, int,
-                                       int, int, int, float, unsigned, long long, cudaStream_t);
+                                       int, int, int, float, unsigned, long long, cudaStream_t,
+                                       const int*, int);
 template int fwd_launch<__half>(const void*, const void*, const void*, void*, float*, int, int,
-                                int, int, float, unsigned, long long, cudaStream_t);
+                                int, int, float, unsigned, long long, cudaStream_t, const int*,
+                                int);
 
 }  // namespace fa

@@ -67,14 +67,19 @@ int check_bwd_args(const void* q, const void* k, const void* v, const void* o, c
 
 // Flags of the *_ex entry points that the library knows (FA_FLAG_* bits).
 constexpr unsigned kKnownFlags = 1u;  // FA_FLAG_CAUSAL
+// Internal plan_fwd flag (never accepted from callers): a varlen batch, whose
+// units are neither split nor cut.
+constexpr unsigned kPlanVarlen = 0x100u;
 
 // Work decomposition of one forward call (fa_fwd.cu).  A unit is unit_rows
 // query rows of one (batch, head), possibly limited to one share of the K/V
 // tiles (split mode); blocks walk units round-robin, or in the balanced
 // schedule each block takes a contiguous range of (unit, K/V tile) steps.
 struct FwdSchedule {
-  int B, H, N, d;
+  int B, H, N, d;     // varlen: B sequences of at most N (max_seqlen) tokens
   int causal;         // 1: row i sees keys j <= i (units ordered longest first)
+  const int* cu;      // varlen: device [B+1] sequence starts in the packed token axis; else null
+  int total;          // tokens a batch entry holds in memory: N, or all B sequences' (varlen)
   int pair;           // 1: fa_fwd_pp_kernel (two 128-row Q tiles a unit), 0: fa_fwd_kernel
   int unit_rows;      // 256 (pair) or 128
   int bn;             // K/V tile rows
@@ -105,13 +110,15 @@ int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 // Launchers (argument validation is done by the callers in fa_api.cu).
 // tok_in: token stride of q, k, v (elements); tok_g: of dq, dk, dv.  o, lse,
 // dout are always contiguous [B,N,H,d] / [B,H,N].
+// cu (varlen): device [B+1] sequence starts, N = max_seqlen, total tokens; else null.
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream);
+               int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream,
+               const int* cu = nullptr, int total = 0);
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                float scale, unsigned flags, long long tok_in, long long tok_g,
-               cudaStream_t stream);
+               cudaStream_t stream, const int* cu = nullptr, int total = 0);
 
 }  // namespace fa

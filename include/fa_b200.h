@@ -148,6 +148,39 @@ int fa_bwd_qkvpacked(const void *qkv, const void *o, const void *dout, const flo
                      unsigned flags, cudaStream_t stream);
 
 /*
+ * Variable-length batches (the YOLOv12 image page's
+ * flash_attn_varlen_qkvpacked_func form, unpacked): B sequences of different
+ * lengths packed along one token axis of `total` tokens.  q, k, v, o, dout,
+ * dq, dk, dv are contiguous [total, H, d] device arrays; lse is [H, total]
+ * fp32.  cu_seqlens is a device array of B + 1 int32 with cu_seqlens[0] = 0,
+ * non-decreasing, cu_seqlens[B] = total: sequence b is tokens
+ * [cu_seqlens[b], cu_seqlens[b+1]), and attention (with FA_FLAG_CAUSAL, the
+ * causal mask by position within the sequence) stays inside each sequence.
+ * max_seqlen must be at least the longest sequence.  The library does not
+ * read cu_seqlens on the host: the kernels clamp each sequence into
+ * [0, total) and to max_seqlen tokens, so malformed contents cannot cause an
+ * out-of-bounds access (the results are then meaningless).  Rows of tokens
+ * that no sequence covers are not written.  Errors as fa_fwd_ex /
+ * fa_bwd_ex; FA_ERR_ALIGN if cu_seqlens is not 4-byte aligned.
+ */
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int B, int total, int max_seqlen, int H, int d,
+                  float scale, int dtype, unsigned flags, cudaStream_t stream);
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                  const int *cu_seqlens, int B, int total, int max_seqlen, int H, int d,
+                  float scale, int dtype, unsigned flags, cudaStream_t stream);
+
+/*
+ * Host copy of the rule the varlen kernels apply to sequence b: its first
+ * token and length after clamping cu_seqlens[b], cu_seqlens[b+1] into
+ * [0, total] and to at most max_seqlen tokens.  cu_seqlens_host is host
+ * memory here.  Returns FA_OK, FA_ERR_NULL or FA_ERR_SHAPE.
+ */
+int fa_varlen_bounds(const int *cu_seqlens_host, int b, int max_seqlen, int total, int *tok0,
+                     int *len);
+
+/*
  * Backward pass, bf16, for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it exists for hosts
  * such as plugin runtimes with their own static memory plan, code that runs

@@ -137,3 +137,19 @@ def test_ex_entry_points_reject_bad_flags_and_types():
     assert lib.fa_bwd_ex(*bargs, 0, 0x80, None) == fa.FA_ERR_FLAGS
     assert lib.fa_bwd_ex(*bargs, -1, 1, None) == fa.FA_ERR_DTYPE
     assert fa.fa_status_string(fa.FA_ERR_FLAGS) == "unknown flag bits"
+
+
+def test_varlen_bounds_clamp_every_input_into_range():
+    # the rule the varlen kernels apply to cu_seqlens: whatever the contents,
+    # each sequence lies inside [0, total) and holds at most max_seqlen tokens
+    import exact_attention_144_b200 as fa
+    total, ms = 1000, 300
+    assert fa.fa_varlen_bounds([0, 100, 400, 1000], 0, ms, total) == (0, 100)
+    assert fa.fa_varlen_bounds([0, 100, 400, 1000], 1, ms, total) == (100, 300)
+    assert fa.fa_varlen_bounds([0, 100, 400, 1000], 2, ms, total) == (400, 300)  # 600 clamped to 300
+    rng = __import__("numpy").random.default_rng(3)
+    for _ in range(2000):
+        cu = [int(x) for x in rng.integers(-2000, 3000, size=5)]
+        for b in range(4):
+            t0, n = fa.fa_varlen_bounds(cu, b, ms, total)
+            assert 0 <= t0 <= total and 0 <= n <= ms and t0 + n <= total
