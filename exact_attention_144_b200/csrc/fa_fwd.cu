@@ -63,12 +63,15 @@ __host__ __device__ __forceinline__ int range_begin(const FwdSchedule& s, int c)
   return c * s.iter_per + imin(c, s.iter_rem);
 }
 
+// VARLEN = false compiles the fixed-length location (s.cu is then unused).
+template <bool VARLEN>
 __host__ __device__ __forceinline__ void locate_seq(const FwdSchedule& s, int b, int& tb,
                                                    int& tok0, int& len) {
-  seq_bounds(s.cu, b, s.N, s.total, tb, tok0, len);
+  seq_bounds(VARLEN ? s.cu : nullptr, b, s.N, s.total, tb, tok0, len);
 }
 
 // Unit u; t1 <= t0 when the unit holds no query row of its sequence (varlen).
+template <bool VARLEN>
 __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s) {
   Unit x;
   x.u = u;
@@ -82,7 +85,7 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
     x.sp = 0;
     x.h = bh % s.H;
     x.b = bh / s.H;
-    locate_seq(s, x.b, x.tb, x.tok0, x.len);
+    locate_seq<VARLEN>(s, x.b, x.tb, x.tok0, x.len);
     x.t0 = 0;
     const int rows_end = imin(x.len, (x.qt + 1) * s.unit_rows);
     x.t1 = x.qt * s.unit_rows < x.len ? (rows_end + s.bn - 1) / s.bn : 0;
@@ -94,7 +97,7 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
   r /= s.n_split;
   x.h = r % s.H;
   x.b = r / s.H;
-  locate_seq(s, x.b, x.tb, x.tok0, x.len);
+  locate_seq<VARLEN>(s, x.b, x.tb, x.tok0, x.len);
   x.t0 = x.sp * s.kvt_per_split;
   x.t1 = imin(x.t0 + s.kvt_per_split, (x.len + s.bn - 1) / s.bn);
   if (x.qt * s.unit_rows >= x.len) x.t1 = x.t0;  // no query row of this sequence
@@ -113,6 +116,7 @@ __host__ __device__ __forceinline__ Unit decode_unit(int u, const FwdSchedule& s
 //             (kStorePartial); the piece holding K/V tile 0 of a unit cut in
 //             pieces is its block's last piece and merges the others
 //             (kStoreMerge), whose blocks all come after it.
+template <bool VARLEN>
 struct UnitIter {
   int i, end, blk;
   __host__ __device__ __forceinline__ UnitIter(const FwdSchedule& s, int blk_) : blk(blk_) {
@@ -134,7 +138,7 @@ struct UnitIter {
       for (;;) {
         const int u = i * s.grid + ((i & 1) ? s.grid - 1 - blk : blk);
         if (u >= end) return false;
-        x = decode_unit(u, s);
+        x = decode_unit<VARLEN>(u, s);
         ++i;
         if (x.t1 > x.t0) return true;
       }
@@ -142,7 +146,7 @@ struct UnitIter {
     if (s.n_iter == 0) {
       for (;;) {
         if (i >= end) return false;
-        x = decode_unit(i, s);
+        x = decode_unit<VARLEN>(i, s);
         i += s.grid;
         if (x.t1 > x.t0) return true;
       }
@@ -150,7 +154,7 @@ struct UnitIter {
     if (i >= end) return false;
     const int u = i / s.n_kvt;
     const int ubeg = u * s.n_kvt, uend = ubeg + s.n_kvt;
-    x = decode_unit(u, s);  // n_split = 1: the whole K/V range
+    x = decode_unit<VARLEN>(u, s);  // n_split = 1: the whole K/V range
     x.t0 = i - ubeg;
     x.t1 = imin(end, uend) - ubeg;
     if (x.t0 > 0) {
@@ -500,7 +504,7 @@ struct FwdPPTraits {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <class T, class Tr>
+template <class T, class Tr, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk,
@@ -560,7 +564,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, vc = 0, qc = 0;
       bool ok = true;
-      UnitIter it(p, blockIdx.x);
+      UnitIter<VARLEN> it(p, blockIdx.x);
       for (Unit un; ok && it.next(p, un);) {
         if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
         mbar_expect_tx(leader, bar(Tr::B_Q_FULL), 2 * Tr::QT_BYTES);
@@ -633,7 +637,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
                   desc_advance(vd, kk * 16 * 128), kIdescPV, (!first || kk > 0) ? 1u : 0u);
       };
-      UnitIter it(p, blockIdx.x);
+      UnitIter<VARLEN> it(p, blockIdx.x);
       if constexpr (Tr::SEP_P) {
         // S_0, S_1 of the next K/V tile are issued as soon as both softmax
         // warpgroups have read the current ones (S_FREE), ahead of P.V; the
@@ -748,7 +752,7 @@ __global__ void __launch_bounds__(384, 1)
     const float c = p.sl2;
     uint32_t g = 0;
     bool ok = true;
-    UnitIter it(p, blockIdx.x);
+    UnitIter<VARLEN> it(p, blockIdx.x);
     for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
@@ -850,7 +854,7 @@ struct FwdTraits {
   static_assert(D % 64 == 0 && BN % 32 == 0, "tile shape");
 };
 
-template <class T, class Tr>
+template <class T, class Tr, bool VARLEN>
 __global__ void __launch_bounds__(224, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -907,7 +911,7 @@ __global__ void __launch_bounds__(224, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t kc = 0, qc = 0;
       bool ok = true;
-      UnitIter it(p, blockIdx.x);
+      UnitIter<VARLEN> it(p, blockIdx.x);
       for (Unit un; ok && it.next(p, un);) {
         if (qc > 0 && !(ok = mbar_wait_warp(bar(Tr::B_Q_EMPTY), (qc - 1) & 1u, w, kSiteQEmpty))) break;
         mbar_expect_tx(leader, bar(Tr::B_Q_FULL), Tr::Q_BYTES);
@@ -941,7 +945,7 @@ __global__ void __launch_bounds__(224, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       uint32_t vc = 0;
       bool ok = true;
-      UnitIter it(p, blockIdx.x);
+      UnitIter<VARLEN> it(p, blockIdx.x);
       for (Unit un; ok && it.next(p, un);) {
         for (int t = un.t0; t < un.t1; ++t) {
           const uint32_t vs = vc % VST;
@@ -987,7 +991,7 @@ __global__ void __launch_bounds__(224, 1)
         ++vc;
         return true;
       };
-      UnitIter it(p, blockIdx.x);
+      UnitIter<VARLEN> it(p, blockIdx.x);
       for (Unit un; ok && it.next(p, un);) {
         if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
         tc_fence_after();
@@ -1027,7 +1031,7 @@ __global__ void __launch_bounds__(224, 1)
     const float c = p.sl2;
     uint32_t g = 0;
     bool ok = true;
-    UnitIter it(p, blockIdx.x);
+    UnitIter<VARLEN> it(p, blockIdx.x);
     for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
@@ -1196,7 +1200,7 @@ size_t fwd_scratch_bytes(const FwdSchedule& s) {
 }
 
 int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces) {
-  UnitIter it(s, blk);
+  UnitIter<false> it(s, blk);
   int n = 0;
   for (Unit x; it.next(s, x); ++n) {
     if (n < max_pieces) {
@@ -1297,7 +1301,8 @@ template <class T, class Tr>
 static int run_single(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
                       float* lse, float scale, long long tok_in, cudaStream_t stream) {
   static_assert(Tr::BM == 128, "unit rows");
-  return launch_fwd<T, Tr::D, Tr::BN, 224, Tr::SMEM_BYTES, false>(fa_fwd_kernel<T, Tr>, s, q, k,
+  return launch_fwd<T, Tr::D, Tr::BN, 224, Tr::SMEM_BYTES, false>(
+      s.cu ? fa_fwd_kernel<T, Tr, true> : fa_fwd_kernel<T, Tr, false>, s, q, k,
                                                                    v, o, lse, scale, tok_in, stream);
 }
 
@@ -1305,7 +1310,8 @@ template <class T, class Tr>
 static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
                   float* lse, float scale, long long tok_in, cudaStream_t stream) {
   static_assert(2 * Tr::BM == 256, "unit rows");
-  return launch_fwd<T, Tr::D, Tr::BN, 384, Tr::SMEM_BYTES, true>(fa_fwd_pp_kernel<T, Tr>, s, q, k,
+  return launch_fwd<T, Tr::D, Tr::BN, 384, Tr::SMEM_BYTES, true>(
+      s.cu ? fa_fwd_pp_kernel<T, Tr, true> : fa_fwd_pp_kernel<T, Tr, false>, s, q, k,
                                                                  v, o, lse, scale, tok_in, stream);
 }
 
