@@ -44,14 +44,14 @@ L2_FLUSH_BYTES = 512 << 20
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the kernel sources hash to the recorded value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.911040e6 + 24.141312e6,
-                                                    "src": "dc416eca56698d71"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.546176e6 + 1.655040e6,
-                                                       "src": "dc416eca56698d71"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.842112e6 + 4.565504e6,
-                                                    "src": "dc416eca56698d71"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.319936e6 + 21.545472e6,
-                                                     "src": "dc416eca56698d71"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.761280e6 + 23.508992e6,
+                                                    "src": "bd813f6e40aaedbe"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.487040e6 + 1.794560e6,
+                                                       "src": "bd813f6e40aaedbe"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.907904e6 + 4.252672e6,
+                                                    "src": "bd813f6e40aaedbe"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.240832e6 + 19.283712e6,
+                                                     "src": "bd813f6e40aaedbe"},
 }
 
 
