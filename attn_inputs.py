@@ -8,7 +8,8 @@ The oracle is then fed exactly those rounded values widened to fp64.
 
 Workloads follow the shapes the pages measure: detector feature maps flattened
 into sequences (20x20 -> N=400, 80x80 -> N=6400), and the long-sequence case
-(N=8192, d=128) from the LLM explainer page.  The pages measure on trained
+(N=8192, d=128) from the LLM explainer page, and the 160x160 first stage of
+the YOLOv12 image page (N=25600, d=96).  The pages measure on trained
 detectors and image datasets; the seeded N(0,1) draws stand in for those
 feature maps at the same shapes.
 """
@@ -70,6 +71,11 @@ for _n in (1024, 2048, 4096, 8192):
 # backward, to measure and test the d = 128 backward at full size.
 WORKLOADS["c4train"] = Workload("c4_train_n8192_h8_d128", 1, 8192, 8, 128, "bf16", 1006,
                                 backward=True, note="long-sequence shape, forward + backward")
+# The first stage of the YOLOv12 image page's network: a 160x160 feature map
+# (N = 25600 tokens) with 96 channels, attended as one head of d = 96, fp16,
+# Q, K, V packed per token.
+WORKLOADS["y12s1"] = Workload("yolov12_stage1_n25600_h1_d96", 1, 25600, 1, 96, "fp16", 1007,
+                              backward=True, note="160x160 map, 96 channels as one head")
 
 
 def draw(B: int, N: int, H: int, d: int, dtype: str, seed: int, count: int = 3,

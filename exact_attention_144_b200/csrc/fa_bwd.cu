@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ===========================================================================
-// fa_bwd_tq_kernel: d = 128.  At 128 queries per inner tile the five
+// fa_bwd_tq_kernel: d = 96 and 128.  At 128 queries per inner tile the five
 // accumulators (S^T, dP^T, dQ, dV, dK: 5 x 128 columns) exceed tensor memory,
 // so the inner tile holds 64 queries and dQ is produced transposed,
 //   dQ_i^T = K^T dS_i^T   (M = d = 128 lanes, N = 64 queries, K = 128 keys),
@@ -515,6 +515,11 @@ __global__ void __launch_bounds__(384, 1)
 // rewrite it for tile i only after dP^T_i has completed, and dP^T_i is
 // committed after the dQ MMA of tile i - 1 (its last reader) by the same
 // thread, so that commit also covers the read.
+// At d = 96 the tiles keep the d = 128 layout: the second 64-column chunk of
+// every shared-memory row is half zero fill from the tensor map; S^T and dP^T
+// contract the 96 real columns, dV and dK are 96 columns wide (dK at
+// [352,448)), and dQ^T is still a 128-lane tile whose lanes 96-127 (K^T rows
+// of zeros) are never drained.
 // ===========================================================================
 template <int D_, int QST_>
 struct BwdTqTraits {
@@ -522,9 +527,11 @@ struct BwdTqTraits {
   static constexpr int BN = 128;  // keys per block
   static constexpr int BM = 64;   // queries per inner tile
   static constexpr int QST = QST_;
-  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int QT_BYTES = BM * D * 2;
+  // 128-byte chunks along d; at d = 96 the last 32 columns of the second
+  // chunk are the tensor map's zero fill
+  static constexpr int KCH = (D + 63) / 64;
+  static constexpr int KV_BYTES = BN * KCH * 128;
+  static constexpr int QT_BYTES = BM * KCH * 128;
   static constexpr int DS_BYTES = BN * BM * 2;       // dS^T tile: keys x 64 queries, 16-bit
   static constexpr int BOX_BYTES = 32 * 32 * 4;      // a warp's dQ staging box
   static constexpr int OFF_K = 0;
@@ -546,7 +553,8 @@ struct BwdTqTraits {
   static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries
-  static_assert(D == 128, "the transposed-dQ layout is laid out for d = 128");
+  // dQ^T has d rows: one 128-lane MMA tile (rows past d are zero and never drained)
+  static_assert(D == 96 || D == 128, "the transposed-dQ layout holds d <= 128 rows");
   static_assert(TM_DK + D <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0 && OFF_DS % 1024 == 0 &&
@@ -555,6 +563,7 @@ struct BwdTqTraits {
 };
 
 using BwdTq128 = BwdTqTraits<128, 3>;
+using BwdTq96 = BwdTqTraits<96, 3>;
 
 template <class T, class Tr, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
@@ -785,7 +794,7 @@ __global__ void __launch_bounds__(384, 1)
                                   (lane & 3) * 4) = __uint_as_float(v[j]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && *abort_flag == 0) {
+      if (lane == 0 && *abort_flag == 0 && quad * 32 < D) {  // d rows past D are padding
         const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)(i0 + i) * BM + hf * 32);
         tma_reduce_add_2d(&tmacc, box, quad * 32, row);
         bulk_commit();
@@ -873,15 +882,16 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (ok && n_qt > 0) ok = drain_dq(n_qt - 1);
     if (lane == 0) bulk_wait_all();
-    // ---- epilogue: dV and scale * dK, key row r, d columns [64 hf, 64 hf + 64)
+    // ---- epilogue: dV and scale * dK, key row r, the 32-column d chunks
+    // hf, hf + 2, ... (d = 96: chunks 0 and 2 for hf = 0, chunk 1 for hf = 1)
     if (ok) ok = mbar_wait(bar(Tr::B_KV_DONE), 0, w, kBSiteKvDone);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
       const size_t off = ((size_t)tb * p.total + tok0 + key) * p.tok_g + (size_t)h * D;
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int col = hf * (D / 2) + cc * 32;
+      for (int cc = hf; cc < D / 32; cc += 2) {
+        const int col = cc * 32;
         uint32_t a[32], k2[32];
         tmem_ld32(tl + Tr::TM_DV + col, a);
         tmem_ld32(tl + Tr::TM_DK + col, k2);
@@ -918,10 +928,14 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
+// Lanes of fa_bwd_pre_kernel per row: d / 8 rounded up to a power of two.
+constexpr int bwd_pre_lanes(int d) { return d <= 64 ? 8 : 16; }
+
 // D_i = sum_x dO_ix O_ix; minus the base-2 LSE; zero the dQ accumulator.
 // Accumulator rows are (b, h, i) with i < Npad for every sequence b; rows past
-// the sequence's length get D = 0 and -LSE = -inf (so P = 0 there).  D / 8
-// lanes take one row, 16 bytes of O and of dO each.
+// the sequence's length get D = 0 and -LSE = -inf (so P = 0 there).  A row
+// takes bwd_pre_lanes(D) lanes, each with 16 bytes of O and of dO (the last
+// four lanes of a d = 96 row have none).
 template <class T, int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o,
                                                          const T* __restrict__ dout,
@@ -931,11 +945,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
                                                          float* __restrict__ dq_acc, int B, int H,
                                                          int N, int Npad, const int* cu,
                                                          int total) {
-  constexpr int LPR = D / 8;     // lanes per row
-  constexpr int RPW = 32 / LPR;  // rows per warp
+  constexpr int LPR = bwd_pre_lanes(D);  // lanes per row (a power of two)
+  constexpr int RPW = 32 / LPR;          // rows per warp
   const int lane = threadIdx.x & 31, sub = lane % LPR;
   const long long row = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
   const bool in = row < (long long)B * H * Npad;
+  const bool part = sub * 8 < D;  // d = 96: 12 of a row's 16 lanes hold data
   int i = 0, h = 0, tb = 0, tok0 = 0, len = 0;
   float acc = 0.f;
   if (in) {
@@ -943,7 +958,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
     h = (int)((row / Npad) % H);
     const int b = (int)(row / ((long long)Npad * H));
     seq_bounds(cu, b, N, total, tb, tok0, len);
-    if (i < len) {
+    if (i < len && part) {
       const size_t at = (((size_t)tb * total + tok0 + i) * H + h) * D + sub * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(o + at);
       const uint4 c = *reinterpret_cast<const uint4*>(dout + at);
@@ -958,9 +973,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const T* __restrict__ o
 #pragma unroll
   for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (in) {
-    float4* arow = reinterpret_cast<float4*>(dq_acc + (size_t)row * D + sub * 8);
-    arow[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    arow[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (part) {
+      float4* arow = reinterpret_cast<float4*>(dq_acc + (size_t)row * D + sub * 8);
+      arow[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      arow[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (sub == 0) {
       dvec[row] = acc;
       lse2[row] = (i < len) ? -(lse[((size_t)tb * H + h) * total + tok0 + i] * kLog2e) : -INFINITY;
@@ -1049,7 +1066,7 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
 
   // The pre-pass rewrites every scratch word the pass reads (it zeroes the
   // accumulator), so earlier contents of the scratch never leak in.
-  constexpr int kPreRowsPerBlock = 8 * (32 / (D / 8));
+  constexpr int kPreRowsPerBlock = 8 * (32 / bwd_pre_lanes(D));
   fa_bwd_pre_kernel<T, D>
       <<<(unsigned)((rows + kPreRowsPerBlock - 1) / kPreRowsPerBlock), 256, 0, stream>>>(
           static_cast<const T*>(o), static_cast<const T*>(dout), lse, lse2, dvec, p.dq_acc, B, H,
@@ -1110,6 +1127,14 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
                                      : fa_bwd_kernel<T, BwdTraits64, false, false>);
       return run_bwd<T, BwdTraits64>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale,
                                      tok_in, tok_g, stream, cu, total);
+    }
+    case 96: {
+      auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq96, true, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq96, true, false>)
+                               : (cu ? fa_bwd_tq_kernel<T, BwdTq96, false, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq96, false, false>);
+      return run_bwd<T, BwdTq96>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
+                                 tok_g, stream, cu, total);
     }
     case 128: {
       auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq128, true, true>

@@ -9,7 +9,7 @@
 //
 // Two persistent kernels, both one block per SM looping over work units:
 //
-// fa_fwd_pp_kernel (d = 64, 128; 384 threads) -- two 128-row Q tiles per unit
+// fa_fwd_pp_kernel (d = 64, 96, 128; 384 threads) -- two 128-row Q tiles per unit
 //   warps 0-3  softmax + epilogue of Q tile 0 (thread t owns row t, TMEM lane t)
 //   warps 4-7  softmax + epilogue of Q tile 1
 //   warp  8    TMA producer: the Q pair once per unit, then K_j, V_j in turn
@@ -25,6 +25,12 @@
 //   one 128-row Q tile per unit, S double buffered in TMEM
 //   warps 0-3 softmax + epilogue, warp 4 Q/K producer, warp 5 V producer,
 //   warp 6 TMEM allocator + MMA issuer.
+//
+// Shared-memory tiles are rows of 64-element (128-byte, swizzled) chunks.  A
+// d = 96 head uses two chunks a row: the second TMA box reaches past the
+// head's last element and the tensor map fills those 32 columns with zeros
+// (no memory is read for them); Q K^T contracts only the 96 real columns (six
+// k-steps of 16) and P.V and the O accumulator are 96 columns wide.
 //
 // In both, P (16-bit) is written back over the first BN/2 columns of its S
 // buffer and consumed from there by the P.V MMA (A operand in TMEM).  O is
@@ -475,9 +481,11 @@ struct FwdPPTraits {
   static constexpr int BN = 128;
   static constexpr int KST = KST_;
   static constexpr int VST = VST_;
-  static constexpr int KCH = D / 64;
-  static constexpr int QT_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
+  // 128-byte chunks along d; at d = 96 the second chunk's last 32 columns
+  // are the tensor map's zero fill and only the first 96 are contracted
+  static constexpr int KCH = (D + 63) / 64;
+  static constexpr int QT_BYTES = BM * KCH * 128;
+  static constexpr int KV_BYTES = BN * KCH * 128;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
@@ -834,9 +842,9 @@ struct FwdTraits {
   static constexpr int BN = BN_;
   static constexpr int KST = KST_;
   static constexpr int VST = VST_;
-  static constexpr int KCH = D / 64;                 // 128-byte chunks along d
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int KCH = (D + 63) / 64;          // 128-byte chunks along d (zero-filled tail)
+  static constexpr int Q_BYTES = BM * KCH * 128;
+  static constexpr int KV_BYTES = BN * KCH * 128;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
@@ -851,7 +859,7 @@ struct FwdTraits {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(2 * BN + D <= 512, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(D % 64 == 0 && BN % 32 == 0, "tile shape");
+  static_assert(D % 32 == 0 && BN % 32 == 0, "tile shape");
 };
 
 template <class T, class Tr, bool VARLEN>
@@ -1101,21 +1109,30 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float* __restrict
   float tot = 0.f;
   for (int s = 0; s < S; ++s) tot += ex2(lse_part[(((size_t)s * B + b) * H + h) * N + n] - mx);
   const float L2 = mx + lg2(tot);
-  constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
-  float acc[PER];
+  // lane x owns the column pairs 2 (x + 32 j), j < NP (d = 96 leaves lanes
+  // 16-31 idle in the second pair)
+  constexpr int NP = (D / 2 + 31) / 32;
+  float2 acc[NP];
 #pragma unroll
-  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  for (int j = 0; j < NP; ++j) acc[j] = make_float2(0.f, 0.f);
   for (int s = 0; s < S; ++s) {
     const float wgt = ex2(lse_part[(((size_t)s * B + b) * H + h) * N + n] - L2);
-    const float* src = o_part + ((((size_t)s * B + b) * N + n) * H + h) * D + lane * PER;
+    const float* src = o_part + ((((size_t)s * B + b) * N + n) * H + h) * D;
 #pragma unroll
-    for (int j = 0; j < PER; ++j) acc[j] += wgt * src[j];
+    for (int j = 0; j < NP; ++j) {
+      const int col = 2 * (lane + 32 * j);
+      if (col < D) {
+        const float2 x = *reinterpret_cast<const float2*>(src + col);
+        acc[j].x = fmaf(wgt, x.x, acc[j].x);
+        acc[j].y = fmaf(wgt, x.y, acc[j].y);
+      }
+    }
   }
-  T* dst = o + (((size_t)b * N + n) * H + h) * D + lane * PER;
+  T* dst = o + (((size_t)b * N + n) * H + h) * D;
 #pragma unroll
-  for (int j = 0; j < PER; j += 2) {
-    uint32_t v = Elem<T>::pack(acc[j], acc[j + 1]);
-    *reinterpret_cast<uint32_t*>(dst + j) = v;
+  for (int j = 0; j < NP; ++j) {
+    const int col = 2 * (lane + 32 * j);
+    if (col < D) *reinterpret_cast<uint32_t*>(dst + col) = Elem<T>::pack(acc[j].x, acc[j].y);
   }
   if (lane == 0) lse[((size_t)b * H + h) * N + n] = L2 * kLn2;
 }
@@ -1138,19 +1155,20 @@ static int choose_splits(long long base_units, int n_kvt, int sm_count) {
 // give every SM the same number of (unit, K/V tile) steps instead.  Units are
 // then cut into pieces across neighbouring blocks and merged in the kernel,
 // so it is kept for units long enough (>= 16 K/V tiles) that the extra
-// Q loads and merges stay small, and for more than one wave of units (with
-// fewer units than SMs nearly every unit would be cut, and measured on B200
-// the merges then cost more than the idle SMs: 128 units of 32 tiles ran
-// 79 us balanced against 74 us round-robin).
+// Q loads and merges stay small.  With fewer units than SMs nearly every unit
+// is cut, which pays only for long units (measured on B200: 128 units of 32
+// tiles ran 79 us balanced against 74 us round-robin, while 100 units of 200
+// tiles -- one d = 96 head of 25600 rows -- ran 300 us against 397 us).
 static bool use_balanced(long long units, int n_kvt, int sm_count) {
-  if (n_kvt < 16 || units <= sm_count || units * n_kvt >= (1ll << 31)) return false;
+  if (n_kvt < 16 || units * n_kvt >= (1ll << 31)) return false;
+  if (units <= sm_count && n_kvt < 64) return false;
   const long long waves = (units + sm_count - 1) / sm_count;
   return (double)units / (double)(waves * sm_count) < 0.95;
 }
 
 int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedule* s) {
   if (B < 1 || H < 1 || N < 1 || sm_count < 1) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
+  if (d != 64 && d != 96 && d != 128 && d != 256) return FA_ERR_HEADDIM;
   FwdSchedule x{};
   x.B = B;
   x.H = H;
@@ -1333,6 +1351,10 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
     case 64:
       return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, tok_in, stream)
                     : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale, tok_in,
+                                                               stream);
+    case 96:
+      return s.pair ? run_pp<T, FwdPPTraits<96, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream)
+                    : run_single<T, FwdTraits<96, 128, 3, 2>>(s, q, k, v, o, lse, scale, tok_in,
                                                                stream);
     case 128:
       return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream)

@@ -20,7 +20,7 @@
  *   16-bit floats (bf16 for the unsuffixed entry points, fp16 for *_f16);
  *   token stride H*d elements, head stride d.  lse: contiguous [B, H, N]
  *   fp32 device array (natural log).  Every pointer must be 16-byte aligned.
- *   d is 64, 128 or 256 (fa_bwd: 64 or 128); B, H, N >= 1; each tensor
+ *   d is 64, 96, 128 or 256 (fa_bwd: 64, 96 or 128); B, H, N >= 1; each tensor
  *   holds fewer than 2^31 elements.  scale is any finite float (normally
  *   1/sqrt(d)).  Arithmetic: 16-bit inputs, fp32 accumulation and softmax,
  *   outputs rounded to nearest even.
@@ -107,10 +107,10 @@ int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
 /*
  * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
  * Inputs q, k, v, o (the forward output), dout (upstream gradient of o) and
- * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64 or 128
- * (d = 64: 128-query inner tiles; d = 128: 64-query inner tiles with dQ
- * produced transposed, since five 128-column accumulators exceed tensor
- * memory); other d return FA_ERR_HEADDIM.
+ * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64, 96 or
+ * 128 (d = 64: 128-query inner tiles; d = 96 and 128: 64-query inner tiles
+ * with dQ produced transposed, since five 128-column accumulators exceed
+ * tensor memory); other d return FA_ERR_HEADDIM.
  */
 int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            const void *dout, const float *lse, void *dq, void *dk, void *dv,

@@ -76,11 +76,11 @@ def test_forward_validation(fa):
     assert _fwd(fa, ok, H=0) == fa.FA_ERR_SHAPE
     assert _fwd(fa, ok, N=0) == fa.FA_ERR_SHAPE
     assert _fwd(fa, ok, B=1 << 10, N=1 << 16, H=1, d=64) == fa.FA_ERR_SHAPE  # 2^32 elements
-    for d in (0, 32, 96, 100, 512):
+    for d in (0, 32, 80, 100, 160, 512):
         assert _fwd(fa, ok, d=d) == fa.FA_ERR_HEADDIM
     assert _fwd(fa, ok, scale=math.nan) == fa.FA_ERR_SCALE
     assert _fwd(fa, ok, scale=math.inf) == fa.FA_ERR_SCALE
-    assert fa.lib().fa_fwd_f16(*ok, 1, 1, 8, 96, ctypes.c_float(1.0), None) == fa.FA_ERR_HEADDIM
+    assert fa.lib().fa_fwd_f16(*ok, 1, 1, 8, 80, ctypes.c_float(1.0), None) == fa.FA_ERR_HEADDIM
 
 
 def test_backward_validation(fa):
@@ -92,7 +92,7 @@ def test_backward_validation(fa):
         p[i] = MIS
         assert _bwd(fa, p) == fa.FA_ERR_ALIGN
     assert _bwd(fa, ok, N=-3) == fa.FA_ERR_SHAPE
-    for d in (32, 96, 256):
+    for d in (32, 80, 160, 256):
         assert _bwd(fa, ok, d=d) == fa.FA_ERR_HEADDIM
     assert _bwd(fa, ok, scale=-math.inf) == fa.FA_ERR_SCALE
 

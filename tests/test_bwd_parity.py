@@ -75,6 +75,18 @@ def test_head_dim_128_fp16(fa, N):
     check_grads(fa, 1, N, 3, 128, "fp16", 900 + N)
 
 
+@pytest.mark.parametrize("N", [1, 17, 64, 65, 127, 128, 129, 300, 640])
+def test_head_dim_96_bf16(fa, N):
+    # d = 96 runs the transposed-dQ kernel on the d = 128 tile layout with
+    # the last 32 columns of every row zero filled
+    check_grads(fa, 2, N, 2, 96, "bf16", 1100 + N)
+
+
+@pytest.mark.parametrize("B,N,H", [(1, 100, 3), (1, 257, 3), (1, 2048, 2)])
+def test_head_dim_96_fp16(fa, B, N, H):
+    check_grads(fa, B, N, H, 96, "fp16", 1150 + N)
+
+
 def test_head_dim_128_many_tiles(fa):
     # 16 key tiles per head, 32 query tiles each: both dQ^T buffers and every
     # Q/dO stage are reused many times over
@@ -115,7 +127,7 @@ def test_training_workload_sampled_heads(fa):
         assert torch.isfinite(t.float()).all()
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 def test_deterministic_dk_dv(fa, d):
     # dK and dV are owned by one block each (no atomics): bitwise repeatable.
     q, k, v, dout = attn_inputs.draw(1, 700, 2, d, "bf16", 702, 4, device="cuda")

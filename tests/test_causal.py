@@ -58,7 +58,7 @@ def test_causal_forward_ragged_d64(fa, N):
     check_fwd(fa, 2, N, 2, 64, "bf16", 1100 + N)
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("N", [100, 300])
 def test_causal_forward_head_sizes_and_types(fa, d, dtype, N):
@@ -112,7 +112,7 @@ def check_bwd(fa, B, N, H, d, dtype, seed):
         assert s["max"] <= GRAD_MAX, (name, s)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("N", [1, 17, 64, 127, 128, 129, 300, 640])
 def test_causal_backward_ragged(fa, d, N):
     check_bwd(fa, 2, N, 2, d, "bf16", 1400 + N + d)

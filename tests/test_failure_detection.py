@@ -49,7 +49,7 @@ def test_errors_leave_outputs_untouched(fa):
     lib = fa.lib()
     import ctypes
     rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                    1, 1, 64, 96, ctypes.c_float(0.1), None)
+                    1, 1, 64, 80, ctypes.c_float(0.1), None)
     assert rc == fa.FA_ERR_HEADDIM
     rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr() + 2, lse.data_ptr(),
                     1, 1, 64, 64, ctypes.c_float(0.1), None)

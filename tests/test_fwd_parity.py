@@ -57,7 +57,7 @@ def test_ragged_lengths_d64_bf16(fa, N):
     check_full(fa, 2, N, 3, 64, "bf16", 100 + N)
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("N", [1, 65, 129, 300])
 def test_head_sizes_and_types(fa, d, dtype, N):
@@ -70,10 +70,11 @@ def test_split_kv_path(fa):
     check_full(fa, 1, 3000, 1, 64, "bf16", 301)
     check_full(fa, 1, 2500, 1, 128, "fp16", 302)
     check_full(fa, 1, 1900, 1, 256, "bf16", 303)
+    check_full(fa, 1, 3000, 1, 96, "fp16", 304)
 
 
 @pytest.mark.parametrize("B,N,H,d,dtype", [(1, 2000, 20, 64, "bf16"), (1, 2000, 20, 128, "fp16"),
-                                             (1, 4096, 10, 64, "bf16")])
+                                             (1, 4096, 10, 64, "bf16"), (1, 2000, 20, 96, "bf16")])
 def test_balanced_schedule(fa, B, N, H, d, dtype):
     # 160 units of 256 query rows on 148 SMs: every block takes an equal range
     # of (unit, K/V tile) steps, so units are cut in pieces on neighbouring

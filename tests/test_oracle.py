@@ -280,6 +280,9 @@ def test_page_printed_shapes():
     assert e["map"][0] * e["map"][1] == e["N"] == w3.N and w3.H * w3.d == e["C"]
     f = items["yolov12_stage1_map160"]
     assert f["map"][0] * f["map"][1] == f["N"]
+    assert f["qkv_width"] == 3 * f["C"]
+    w6 = WORKLOADS["y12s1"]
+    assert (w6.N, w6.H * w6.d) == (f["N"], f["C"])
 
 
 # ------------------------------------------------- tests on the real oracle

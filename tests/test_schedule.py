@@ -20,6 +20,7 @@ SHAPES = [
     (1, 8, 1024, 64), (1, 8, 2048, 64), (1, 8, 4096, 64), (1, 8, 8192, 64), (4, 8, 4096, 64),
     (1, 10, 2000, 64), (1, 20, 2000, 64), (1, 10, 4096, 64), (1, 3, 8192, 64), (2, 3, 5000, 128), (1, 1, 1, 64), (3, 1, 129, 128),
     (1, 7, 4097, 64), (2, 16, 4096, 128), (1, 1, 100000, 64), (8, 16, 2048, 64),
+    (1, 1, 400, 96), (2, 4, 1600, 96), (1, 8, 8192, 96),  # d = 96: the d = 128 tile shapes
 ]
 SMS = [148, 132, 7, 1]
 
@@ -107,6 +108,13 @@ def test_workload_plans():
     # the detector deep stage: short units (4 K/V tiles) stay round-robin
     plan = fa.fa_fwd_plan(32, 4, 400, 64, 148)
     assert (plan["kernel"], plan["n_units"], plan["balanced"], plan["n_split"]) == (1, 256, 0, 1)
+    # one long head (the YOLOv12 stage-1 map, d = 96): 100 units of 200 K/V
+    # tiles leave 48 SMs idle round-robin, and long units are worth cutting
+    plan = fa.fa_fwd_plan(1, 1, 25600, 96, 148)
+    assert (plan["kernel"], plan["n_units"], plan["balanced"], plan["grid"]) == (1, 100, 1, 148)
+    # fewer units than SMs but short ones (32 K/V tiles) stay whole
+    plan = fa.fa_fwd_plan(1, 8, 4096, 64, 148)
+    assert (plan["n_units"], plan["balanced"], plan["grid"]) == (128, 0, 128)
     # a single short head: one 128-row tile kernel unit per tile
     plan = fa.fa_fwd_plan(1, 2, 128, 64, 148)
     assert (plan["kernel"], plan["unit_rows"], plan["n_units"]) == (0, 128, 2)
@@ -118,7 +126,7 @@ def test_plan_rejects_bad_arguments():
             fa.fa_fwd_plan(*args)
         assert e.value.status == fa.FA_ERR_SHAPE
     with pytest.raises(fa.FAError) as e:
-        fa.fa_fwd_plan(1, 1, 64, 96, 148)
+        fa.fa_fwd_plan(1, 1, 64, 80, 148)
     assert e.value.status == fa.FA_ERR_HEADDIM
     with pytest.raises(fa.FAError):
         fa.fa_fwd_plan_pieces(1, 1, 64, 64, 148, 5)  # block past the grid

@@ -36,7 +36,7 @@ def packed(lengths, H, d, dtype, seed):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (128, "fp16"), (256, "bf16")])
+@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (96, "fp16"), (128, "fp16"), (256, "bf16")])
 def test_varlen_forward_per_sequence(fa, d, dtype, causal):
     H = 2
     (q, k, v, _), cu, total = packed(LENGTHS, H, d, dtype, 1900 + d)
@@ -58,7 +58,7 @@ def test_varlen_forward_per_sequence(fa, d, dtype, causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 def test_varlen_backward_per_sequence(fa, d, causal):
     H = 2
     (q, k, v, do), cu, total = packed(LENGTHS, H, d, "bf16", 2000 + d)
