@@ -3,7 +3,7 @@
 This module is shared by the tests, the bench and the oracle checks.  It holds
 no attention arithmetic: it only draws i.i.d. normal numbers from a seeded
 numpy PCG64 stream, scales them by a power of two, and rounds them to the
-16-bit type the GPU receives (round-to-nearest-even, done by torch's CPU cast).
+16-bit or 8-bit (E4M3) type the GPU receives (round-to-nearest-even, done by torch's CPU cast).
 The oracle is then fed exactly those rounded values widened to fp64.
 
 Workloads follow the shapes the pages measure: detector feature maps flattened
@@ -21,7 +21,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp8": torch.float8_e4m3fn}
 
 
 @dataclass(frozen=True)
@@ -31,7 +31,7 @@ class Workload:
     N: int
     H: int
     d: int
-    dtype: str           # element type handed to the GPU ("bf16" or "fp16")
+    dtype: str           # element type handed to the GPU ("bf16", "fp16" or "fp8": E4M3)
     seed: int
     std: float = 1.0     # the draws are N(0,1) * std (std is a power of two)
     backward: bool = False
@@ -74,6 +74,9 @@ WORKLOADS["c4train"] = Workload("c4_train_n8192_h8_d128", 1, 8192, 8, 128, "bf16
 # The first stage of the YOLOv12 image page's network: a 160x160 feature map
 # (N = 25600 tokens) with 96 channels, attended as one head of d = 96, fp16,
 # Q, K, V packed per token.
+# The long-sequence shape on 8-bit (E4M3) inputs, forward only.
+WORKLOADS["c4fp8"] = Workload("c4_long_fp8_n8192_h8_d128", 1, 8192, 8, 128, "fp8", 1008,
+                              note="long-sequence shape, E4M3 Q, K, V, descale factors 1")
 WORKLOADS["y12s1"] = Workload("yolov12_stage1_n25600_h1_d96", 1, 25600, 1, 96, "fp16", 1007,
                               backward=True, note="160x160 map, 96 channels as one head")
 

@@ -139,18 +139,39 @@ def job_tflops(flop_per_step: float, ms_per_step: float, world: int) -> float:
     return world * flop_per_step / (ms_per_step * 1e-3) / 1e12
 
 
+def entry_points(fa, w: attn_inputs.Workload):
+    """(forward, backward, output dtype) of the library for the workload's
+    element type; the 8-bit workloads are forward only, with bf16 O."""
+    if w.dtype == "fp8":
+        def fwd(q, k, v, o=None, lse=None, scale=None, stream=None):
+            return fa.fa_fwd_fp8(q, k, v, o=o, lse=lse, scale=scale, stream=stream)
+        return fwd, None, torch.bfloat16
+    if w.dtype == "bf16":
+        return fa.fa_fwd, fa.fa_bwd, torch.bfloat16
+    return fa.fa_fwd_f16, fa.fa_bwd_f16, torch.float16
+
+
+def tensor_peak(pk: dict, w: attn_inputs.Workload) -> tuple:
+    """Dense tensor-core peak for the workload's operand type: the measured
+    bf16 figure, doubled for 8-bit operands (the nominal fp8:bf16 ratio,
+    4.5 : 2.25 PFLOP/s dense)."""
+    if w.dtype == "fp8":
+        return 2.0 * pk["bf16_tflops"], 2.0 * pk["bf16_tflops_sustained"], "2 x bf16_tflops"
+    return pk["bf16_tflops"], pk["bf16_tflops_sustained"], "bf16_tflops"
+
+
 def e2e_pipelined(fa, w, args, dev, q, k, v, do, train, mk):
     """Per-step time (ms) of steps that each upload their inputs from pinned
     host memory, compute, and download their results, overlapped across
     steps on three streams with two device buffer sets.  Returns (ms per step,
     bytes uploaded per step, bytes downloaded per step)."""
-    fwd = fa.fa_fwd if w.dtype == "bf16" else fa.fa_fwd_f16
-    bwd = fa.fa_bwd if w.dtype == "bf16" else fa.fa_bwd_f16
+    fwd, bwd, out_dtype = entry_points(fa, w)
     host_in = [t.cpu().pin_memory() for t in ((q, k, v, do) if train else (q, k, v))]
     sets = []
     for _ in range(2):
         ins = [torch.empty_like(t, device=dev) for t in host_in]
-        outs = [torch.empty_like(q), torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)]
+        outs = [torch.empty(q.shape, dtype=out_dtype, device=dev),
+                torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)]
         if train:
             outs += [torch.empty_like(q) for _ in range(3)]
         hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
@@ -296,12 +317,12 @@ def main():
     # Each rank owns one replica of the workload (its own seeded batch).
     q, k, v, do = attn_inputs.draw(w.B, w.N, w.H, w.d, w.dtype, replica_seed(w, rank), 4,
                                    std=w.std, device=dev)
-    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    fwd, bwd, out_dtype = entry_points(fa, w)
+    o = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    fwd = fa.fa_fwd if w.dtype == "bf16" else fa.fa_fwd_f16
-    bwd = fa.fa_bwd if w.dtype == "bf16" else fa.fa_bwd_f16
-    train = w.backward
+    train = w.backward and bwd is not None
 
     def step():
         fwd(q, k, v, o=o, lse=lse, scale=w.scale)
@@ -357,17 +378,18 @@ def main():
     achieved = dom_flop / (dom_ms * 1e-3) / 1e12
     tr = TRAFFIC.get((dom, w.name))
     traffic = tr["bytes"] if tr and tr["src"] == kernel_source_hash() else None
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+    peak, peak_sus, peak_name = tensor_peak(pk, w)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                 "kernel": dom, "kernel_ms": dom_ms,
-                "peak_source": f"bf16_tflops (burst) of {pk_src} MEASURED_PEAKS.json",
-                "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
+                "peak_source": f"{peak_name} (burst) of {pk_src} MEASURED_PEAKS.json",
+                "frac_of_sustained": achieved / peak_sus}
     kernels = {fwd_name: {"ms": statistics.mean(fwd_ms),
                           "tflops": w.fwd_flop / (statistics.mean(fwd_ms) * 1e-3) / 1e12}}
     if train:
         kernels[bwd_name] = {"ms": statistics.mean(bwd_ms), "tflops": achieved}
     for kv in kernels.values():
-        kv["frac"] = kv["tflops"] / pk["bf16_tflops"]
+        kv["frac"] = kv["tflops"] / peak
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -388,13 +410,16 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": {"bf16": "bf16", "fp16": "fp16", "fp8": "fp8e4m3"}[w.dtype],
             "data": "synthetic",
             "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
                        "heads": w.H, "head_dim": w.d, "causal": False,
                        "parallelism": f"replicas x{world} (batch per rank, no collective)",
                        "l2": "512 MiB written between timed steps",
-                       "inputs": "seeded N(0,1) draws rounded to the 16-bit type"},
+                       "inputs": "seeded N(0,1) draws rounded to the "
+                                 + ("E4M3 type (descale factors 1), bf16 O" if w.dtype == "fp8"
+                                    else "16-bit type")},
             "e2e": {"value": job_tflops(flop_step, e2e_ms, world), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "how": "pinned host -> device inputs, step, device -> pinned host results "
@@ -406,6 +431,7 @@ def main():
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
             "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
+            "pct_of_dtype_peak": 100.0 * value / world / peak,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

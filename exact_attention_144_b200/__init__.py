@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
     lib.fa_bwd_f16.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes
     lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, f, f, f, ctypes.c_uint, vp]
     lib.fa_bwd_ex.argtypes = [vp] * 9 + [i, i, i, i, f, i, ctypes.c_uint, vp]
     lib.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, f, i, ctypes.c_uint, vp]
     lib.fa_bwd_qkvpacked.argtypes = [vp] * 5 + [i, i, i, i, f, i, ctypes.c_uint, vp]
@@ -63,7 +64,7 @@ def _load() -> ctypes.CDLL:
     lib.fa_varlen_bounds.argtypes = [ctypes.POINTER(ctypes.c_int), i, i, i,
                                      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.fa_varlen_bounds.restype = i
-    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc", "fa_fwd_ex",
+    for n in ("fa_fwd", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_noalloc", "fa_fwd_ex", "fa_fwd_fp8",
               "fa_bwd_ex", "fa_fwd_qkvpacked", "fa_bwd_qkvpacked", "fa_fwd_varlen",
               "fa_bwd_varlen"):
         getattr(lib, n).restype = i
@@ -247,6 +248,31 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale=None, stream=None):
 
 _FWD = {torch.bfloat16: fa_fwd, torch.float16: fa_fwd_f16}
 _BWD = {torch.bfloat16: fa_bwd, torch.float16: fa_bwd_f16}
+
+
+def fa_fwd_fp8(q, k, v, descale_q=1.0, descale_k=1.0, descale_v=1.0, o=None, lse=None,
+               scale=None, flags=0, stream=None):
+    """Forward on E4M3 inputs (torch.float8_e4m3fn [B, N, H, 128]) with
+    per-tensor descale factors: attention of (descale_q q, descale_k k,
+    descale_v v).  Returns (o [B, N, H, d] bf16, lse [B, H, N] fp32)."""
+    _check_bnhd("q", q, torch.float8_e4m3fn)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, N, H, d]")
+    B, N, H, d = q.shape
+    for name, t in (("k", k), ("v", v)):
+        _check_bnhd(name, t, torch.float8_e4m3fn, q.shape)
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q.device) if o is None else o
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_bnhd("o", o, torch.bfloat16, (B, N, H, d))
+    _check_bnhd("lse", lse, torch.float32, (B, H, N))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = _load().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                            float(scale), float(descale_q), float(descale_k), float(descale_v),
+                            int(flags), _stream(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_fp8", rc)
+    return o, lse
 
 
 def fa_fwd_ex(q, k, v, o=None, lse=None, scale=None, flags=0, stream=None):

@@ -169,18 +169,21 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d,
+int make_tmap_bnhd(CUtensorMap* map, const void* base, int fmt, int B, int N, int H, int d,
                    int box_rows, long long tok_stride) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return FA_ERR_LAUNCH;
+  const cuuint64_t eb = fmt == 2 ? 1 : 2;  // bytes an element
   // dims innermost first: element within head, head, token, batch
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)tok_stride * 2,
-                                 (cuuint64_t)N * tok_stride * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * eb, (cuuint64_t)tok_stride * eb,
+                                 (cuuint64_t)N * tok_stride * eb};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                  4, const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = fmt == 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : fmt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
@@ -273,6 +276,25 @@ static int bwd_packed_entry(const void* qkv, const void* o, const void* dout, co
   const long long hd = (long long)H * d;
   return bwd_launch<T>(base, base + hd, base + 2 * hd, o, dout, lse, g, g + hd, g + 2 * hd, B, H,
                        N, d, scale, flags, 3 * hd, 3 * hd, stream);
+}
+
+// E4M3 Q, K, V with per-tensor descale factors: the problem is attention on
+// (descale_q Q, descale_k K, descale_v V); O is bf16.
+static int fwd_fp8_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, float scale, float descale_q, float descale_k,
+                         float descale_v, unsigned flags, cudaStream_t stream) {
+  int rc = check_ptrs({q, k, v, o, lse});
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK && d != 128) rc = FA_ERR_HEADDIM;
+  const float s_eff = scale * descale_q * descale_k;
+  if (rc == FA_OK && !(isfinite(descale_q) && isfinite(descale_k) && isfinite(descale_v) &&
+                       isfinite(s_eff)))
+    rc = FA_ERR_SCALE;
+  if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
+  if (rc == FA_OK)
+    rc = fwd_launch<__nv_fp8_e4m3>(q, k, v, o, lse, B, H, N, d, s_eff, flags, (long long)H * d,
+                                   stream, nullptr, 0, descale_v);
+  return rc;
 }
 
 // Variable-length batch: B sequences packed along one token axis of `total`
@@ -377,6 +399,13 @@ FA_EXPORT int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
   if (dtype == FA_FP16)
     return fa::fwd_entry<__half>(q, k, v, o, lse, B, H, N, d, scale, flags, stream);
   return FA_ERR_DTYPE;
+}
+
+FA_EXPORT int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, float scale, float descale_q, float descale_k,
+                         float descale_v, unsigned flags, cudaStream_t stream) {
+  return fa::fwd_fp8_entry(q, k, v, o, lse, B, H, N, d, scale, descale_q, descale_k, descale_v,
+                           flags, stream);
 }
 
 FA_EXPORT int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, int N, int d,

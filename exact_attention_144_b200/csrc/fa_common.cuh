@@ -13,6 +13,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -174,6 +175,28 @@ __device__ __forceinline__ void umma_ts(bool issue, uint32_t d_tmem, uint32_t a_
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"((uint32_t)issue)
       : "memory");
 }
+// The same two products for 8-bit operands (kind::f8f6f4; K = 32 elements
+// per instruction, the same 32 bytes of each operand row as kind::f16).
+__device__ __forceinline__ void umma_ss_f8(bool issue, uint32_t d_tmem, uint64_t adesc,
+                                           uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"((uint32_t)issue)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_f8(bool issue, uint32_t d_tmem, uint32_t a_tmem,
+                                           uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"((uint32_t)issue)
+      : "memory");
+}
 // Arrive (once) on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(bool issue, uint32_t bar) {
   asm volatile(
@@ -257,6 +280,8 @@ __device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) 
 
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 // fmt: 0 = fp16, 1 = bf16 (same for A and B).  b_mn: B operand is MN-major.
+// kind::f8f6f4 reads the same fields; there format 0 is E4M3 (the MN-major
+// B operand is allowed for E4M3).
 __host__ __device__ constexpr uint32_t f16_idesc(uint32_t fmt, int M, int N, bool b_mn) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -265,9 +290,17 @@ __host__ __device__ constexpr uint32_t f16_idesc(uint32_t fmt, int M, int N, boo
 // ------------------------------------------------------------ element types
 template <class T>
 struct Elem;
+// kFmt: instruction-descriptor format; kBytes: bytes an element; kF8: 8-bit
+// operands (kind::f8f6f4); Out: the type O is stored in; kMapFmt: tensor-map
+// element type (0 fp16, 1 bf16, 2 one byte).  pack(lo, hi) rounds two values
+// to the element type, lo in the low bits (16-bit types: one 32-bit word;
+// E4M3: the low 16 bits).
 template <>
 struct Elem<__nv_bfloat16> {
   static constexpr uint32_t kFmt = 1;
+  static constexpr int kBytes = 2, kMapFmt = 1;
+  static constexpr bool kF8 = false;
+  using Out = __nv_bfloat16;
   __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -280,6 +313,9 @@ struct Elem<__nv_bfloat16> {
 template <>
 struct Elem<__half> {
   static constexpr uint32_t kFmt = 0;
+  static constexpr int kBytes = 2, kMapFmt = 0;
+  static constexpr bool kF8 = false;
+  using Out = __half;
   __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -289,6 +325,36 @@ struct Elem<__half> {
     return __half22float2(v);
   }
 };
+
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr uint32_t kFmt = 0;  // E4M3 in kind::f8f6f4
+  static constexpr int kBytes = 1, kMapFmt = 2;
+  static constexpr bool kF8 = true;
+  using Out = __nv_bfloat16;
+  // round to nearest even, saturating at +-448 (no value here reaches it)
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+  }
+};
+
+// D (+)= A B for the element type T (kind::f16 or kind::f8f6f4).
+template <class T>
+__device__ __forceinline__ void mma_ss(bool issue, uint32_t d_tmem, uint64_t adesc,
+                                       uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  if constexpr (Elem<T>::kF8)
+    umma_ss_f8(issue, d_tmem, adesc, bdesc, idesc, accumulate);
+  else
+    umma_ss(issue, d_tmem, adesc, bdesc, idesc, accumulate);
+}
+template <class T>
+__device__ __forceinline__ void mma_ts(bool issue, uint32_t d_tmem, uint32_t a_tmem,
+                                       uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  if constexpr (Elem<T>::kF8)
+    umma_ts_f8(issue, d_tmem, a_tmem, bdesc, idesc, accumulate);
+  else
+    umma_ts(issue, d_tmem, a_tmem, bdesc, idesc, accumulate);
+}
 
 // ------------------------------------------------------ register rebalance
 // Per-warpgroup register limits for the 384-thread kernels: launched with 168

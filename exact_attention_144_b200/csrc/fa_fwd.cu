@@ -186,6 +186,7 @@ struct FwdParams : FwdSchedule {
   float* bal_lse;   // balanced: [grid, unit_rows] base-2 LSE of those rows
   unsigned* bal_flag;  // balanced: [grid] warps that have stored their partial rows; zeroed
   float sl2;        // scale * log2(e)
+  float o_scale;    // factor applied to O when it is stored (the V descale; 1 for 16-bit)
   unsigned long long limit_ns;
   unsigned long long* status;
 };
@@ -306,6 +307,27 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
   return alpha;
 }
 
+// Writes this thread's packed P row (pk from softmax_step) into tensor memory
+// at taddr, where the P.V product reads it as its A operand: 16-bit P two
+// keys a column (BN/2 columns); 8-bit P four keys a column (BN/4 columns),
+// key 4i in the low byte of column i.
+template <class T, int BN>
+__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t (&pk)[BN / 2]) {
+  if constexpr (Elem<T>::kBytes == 2) {
+#pragma unroll
+    for (int q = 0; q < BN / 32; ++q) tmem_st16(taddr + q * 16, &pk[q * 16]);
+  } else {
+    static_assert(BN % 128 == 0, "8-bit P is written 32 columns at a time");
+#pragma unroll
+    for (int q = 0; q < BN / 128; ++q) {
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = pk[q * 64 + 2 * i] | (pk[q * 64 + 2 * i + 1] << 16);
+      tmem_st32(taddr + q * 32, w);
+    }
+  }
+}
+
 // Multiplies this thread's O row (D fp32 columns at taddr) by alpha.
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
@@ -336,7 +358,7 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
   // the row's token along the memory token axis (p.total tokens a batch entry)
   const size_t tok = (size_t)un.tb * p.total + un.tok0 + q_row;
   const size_t lse_at = ((size_t)un.tb * p.H + un.h) * p.total + un.tok0 + q_row;
-  const float inv_l = 1.f / l;
+  const float inv_l = p.o_scale / l;
   const float lse2 = m + lg2(l);
   if (un.kind == kStorePartial) {
     const int ur = q_row - un.qt * p.unit_rows;
@@ -474,18 +496,21 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
 // ===========================================================================
 // fa_fwd_pp_kernel: two Q tiles per unit
 // ===========================================================================
-template <int D_, int KST_, int VST_>
+template <int D_, int KST_, int VST_, int EB_ = 2>
 struct FwdPPTraits {
   static constexpr int D = D_;
+  static constexpr int EB = EB_;          // bytes an element of Q, K, V
+  static constexpr int CH_ELEMS = 128 / EB;  // elements in a 128-byte chunk
   static constexpr int BM = 128;  // rows per Q tile; a unit holds two
   static constexpr int BN = 128;
   static constexpr int KST = KST_;
   static constexpr int VST = VST_;
   // 128-byte chunks along d; at d = 96 the second chunk's last 32 columns
   // are the tensor map's zero fill and only the first 96 are contracted
-  static constexpr int KCH = (D + 63) / 64;
+  static constexpr int KCH = (D * EB + 127) / 128;
   static constexpr int QT_BYTES = BM * KCH * 128;
   static constexpr int KV_BYTES = BN * KCH * 128;
+  static constexpr int P_COLS = BN * EB / 4;  // TMEM columns of one packed P tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
@@ -501,7 +526,7 @@ struct FwdPPTraits {
   // 2 x 64, O 2 x 64 = 512): Q K^T of the next K/V tile may then overwrite S
   // as soon as the softmax warps have read it, before P.V has consumed P.
   // Otherwise (d = 128) P is written over the first BN/2 columns of its S.
-  static constexpr bool SEP_P = 2 * BN + 2 * (BN / 2) + 2 * D <= 512;
+  static constexpr bool SEP_P = 2 * BN + 2 * P_COLS + 2 * D <= 512;
   // exponentials on the FMA pipe per 8 column pairs (see softmax_step): the
   // d = 128 warpgroups take turns, the d = 64 ones run together
   static constexpr int EMU = SEP_P ? 0 : 2;
@@ -580,7 +605,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
-            tma_load_4d(leader, sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64,
+            tma_load_4d(leader, sQ + t * Tr::QT_BYTES + c * (BM * 128), &tmq, bar(Tr::B_Q_FULL),
+                        c * Tr::CH_ELEMS,
                         un.h, un.tok0 + (2 * un.qt + t) * BM, un.tb);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
@@ -592,7 +618,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
-                        c * 64, un.h, un.tok0 + t * BN, un.tb);
+                        c * Tr::CH_ELEMS, un.h, un.tok0 + t * BN, un.tb);
           ++kc;
           const uint32_t vs = vc % VST;
           if (vc >= (uint32_t)VST &&
@@ -602,7 +628,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
-                        c * 64, un.h, un.tok0 + t * BN, un.tb);
+                        c * Tr::CH_ELEMS, un.h, un.tok0 + t * BN, un.tb);
           ++vc;
         }
       }
@@ -630,20 +656,21 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t kd = desc_advance(k_desc0, (kc % KST) * Tr::KV_BYTES);
         const uint64_t qd = desc_advance(q_desc0, t * Tr::QT_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D * Tr::EB / 32; ++kk) {  // 32 bytes of each row a step
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-          umma_ss(leader, tmem + t * BN, desc_advance(qd, ch * (BM * 128) + in),
+          mma_ss<T>(leader, tmem + t * BN, desc_advance(qd, ch * (BM * 128) + in),
                   desc_advance(kd, ch * (BN * 128) + in), kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V for the V stage of counter vc
       auto issue_pv = [&](int t, bool first) {
         const uint64_t vd = desc_advance(v_desc0, (vc % VST) * Tr::KV_BYTES);
-        const uint32_t pa = Tr::SEP_P ? Tr::TM_P + t * (BN / 2) : t * BN;
+        const uint32_t pa = Tr::SEP_P ? Tr::TM_P + t * Tr::P_COLS : t * BN;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
-                  desc_advance(vd, kk * 16 * 128), kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN * Tr::EB / 32; ++kk)  // 32 keys x 16 bits, or 32 x 8 bits
+          mma_ts<T>(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
+                    desc_advance(vd, kk * (32 / Tr::EB) * 128), kIdescPV,
+                    (!first || kk > 0) ? 1u : 0u);
       };
       UnitIter<VARLEN> it(p, blockIdx.x);
       if constexpr (Tr::SEP_P) {
@@ -755,7 +782,7 @@ __global__ void __launch_bounds__(384, 1)
     const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = tl + wg * BN;
-    const uint32_t p_col = tl + Tr::TM_P + wg * (BN / 2);  // used when SEP_P
+    const uint32_t p_col = tl + Tr::TM_P + wg * Tr::P_COLS;  // used when SEP_P
     const uint32_t o_col = tl + Tr::TM_O + wg * D;
     const float c = p.sl2;
     uint32_t g = 0;
@@ -797,12 +824,12 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
           }
 #pragma unroll
-          for (int q = 0; q < BN / 32; ++q) tmem_st16(p_col + q * 16, &pk[q * 16]);
+          store_p<T, BN>(p_col, pk);
           tmem_wait_st();
           if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
         } else {
 #pragma unroll
-          for (int q = 0; q < BN / 32; ++q) tmem_st16(s_col + q * 16, &pk[q * 16]);
+          store_p<T, BN>(s_col, pk);
           tmem_wait_st();
           if (j > 0) {
             // the previous P.V into this O must have landed before O is touched
@@ -820,7 +847,7 @@ __global__ void __launch_bounds__(384, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      ok = store_row<T, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l, w);
+      ok = store_row<typename Elem<T>::Out, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l, w);
     }
   }
 
@@ -835,14 +862,16 @@ __global__ void __launch_bounds__(384, 1)
 // ===========================================================================
 // fa_fwd_kernel: one Q tile per unit, S double buffered
 // ===========================================================================
-template <int D_, int BN_, int KST_, int VST_>
+template <int D_, int BN_, int KST_, int VST_, int EB_ = 2>
 struct FwdTraits {
   static constexpr int D = D_;
+  static constexpr int EB = EB_;             // bytes an element of Q, K, V
+  static constexpr int CH_ELEMS = 128 / EB;  // elements in a 128-byte chunk
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
   static constexpr int KST = KST_;
   static constexpr int VST = VST_;
-  static constexpr int KCH = (D + 63) / 64;          // 128-byte chunks along d (zero-filled tail)
+  static constexpr int KCH = (D * EB + 127) / 128;   // 128-byte chunks along d (zero-filled tail)
   static constexpr int Q_BYTES = BM * KCH * 128;
   static constexpr int KV_BYTES = BN * KCH * 128;
   static constexpr int OFF_Q = 0;
@@ -925,7 +954,7 @@ __global__ void __launch_bounds__(224, 1)
         mbar_expect_tx(leader, bar(Tr::B_Q_FULL), Tr::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < Tr::KCH; ++c)
-          tma_load_4d(leader, sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * 64, un.h,
+          tma_load_4d(leader, sQ + c * (Tr::BM * 128), &tmq, bar(Tr::B_Q_FULL), c * Tr::CH_ELEMS, un.h,
                       un.tok0 + un.qt * Tr::BM, un.tb);
         ++qc;
         for (int t = un.t0; t < un.t1; ++t) {
@@ -937,7 +966,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sK + ks * Tr::KV_BYTES + c * (BN * 128), &tmk, bar(Tr::B_K_FULL + ks),
-                        c * 64, un.h, un.tok0 + t * BN, un.tb);
+                        c * Tr::CH_ELEMS, un.h, un.tok0 + t * BN, un.tb);
           ++kc;
         }
       }
@@ -964,7 +993,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int c = 0; c < Tr::KCH; ++c)
             tma_load_4d(leader, sV + vs * Tr::KV_BYTES + c * (BN * 128), &tmv, bar(Tr::B_V_FULL + vs),
-                        c * 64, un.h, un.tok0 + t * BN, un.tb);
+                        c * Tr::CH_ELEMS, un.h, un.tok0 + t * BN, un.tb);
           ++vc;
         }
       }
@@ -991,8 +1020,9 @@ __global__ void __launch_bounds__(224, 1)
         tc_fence_after();
         const uint64_t vd = desc_advance(v_desc0, vs * Tr::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8, desc_advance(vd, kk * 16 * 128),
+        for (int kk = 0; kk < BN * Tr::EB / 32; ++kk)
+          mma_ts<T>(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
+                  desc_advance(vd, kk * (32 / Tr::EB) * 128),
                   kIdescPV, (!first || kk > 0) ? 1u : 0u);
         umma_commit(leader, bar(Tr::B_V_EMPTY + vs));
         umma_commit(leader, bar(Tr::B_O_DONE));
@@ -1011,9 +1041,9 @@ __global__ void __launch_bounds__(224, 1)
           const uint32_t sb = g & 1u;
           const uint64_t kd = desc_advance(k_desc0, ks * Tr::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D * Tr::EB / 32; ++kk) {
             const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
-            umma_ss(leader, tmem + sb * BN, desc_advance(q_desc0, ch * (Tr::BM * 128) + in),
+            mma_ss<T>(leader, tmem + sb * BN, desc_advance(q_desc0, ch * (Tr::BM * 128) + in),
                     desc_advance(kd, ch * (BN * 128) + in), kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(leader, bar(Tr::B_K_EMPTY + ks));
@@ -1061,7 +1091,7 @@ __global__ void __launch_bounds__(224, 1)
         if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
         const float alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q) tmem_st16(scol + q * 16, &pk[q * 16]);
+        store_p<T, BN>(scol, pk);
         tmem_wait_st();
         if (i > 0) {
           // O holds P_{<j} V_{<j}: once the previous P.V has landed, rescale it
@@ -1078,7 +1108,8 @@ __global__ void __launch_bounds__(224, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      ok = store_row<T, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l, w);
+      ok = store_row<typename Elem<T>::Out, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l,
+                                               w);
     }
   }
 
@@ -1236,22 +1267,23 @@ int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces) {
 
 template <class T, int D, int BN, int THREADS, int SMEM, bool SPLIT_REGS, class Kernel>
 static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const void* k,
-                      const void* v, void* o, float* lse, float scale, long long tok_in,
-                      cudaStream_t stream) {
-  const bool bf16 = Elem<T>::kFmt == 1;
+                      const void* v, void* o, float* lse, float scale, float o_scale,
+                      long long tok_in, cudaStream_t stream) {
+  const int fmt = Elem<T>::kMapFmt;
   CUtensorMap tmq, tmk, tmv;
   int rc;
   // memory view: B batch entries of N tokens, or one entry of all tokens (varlen)
   const int mB = s.cu ? 1 : s.B, mN = s.total;
-  if ((rc = make_tmap_bnhd(&tmq, q, bf16, mB, mN, s.H, D, 128, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmk, k, bf16, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
-  if ((rc = make_tmap_bnhd(&tmv, v, bf16, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmq, q, fmt, mB, mN, s.H, D, 128, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmk, k, fmt, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
+  if ((rc = make_tmap_bnhd(&tmv, v, fmt, mB, mN, s.H, D, BN, tok_in)) != FA_OK) return rc;
 
   FwdParams p{};
   static_cast<FwdSchedule&>(p) = s;
   p.o = o;
   p.lse = lse;
   p.sl2 = scale * kLog2e;
+  p.o_scale = o_scale;
   p.limit_ns = 4000000000ull;
   p.status = device_status_ptr();
 
@@ -1306,8 +1338,9 @@ static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const vo
   note_launches(1);
   if (rc == FA_OK && s.n_split > 1) {
     const long long rows = (long long)s.B * s.N * s.H;
-    fa_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-        p.o_part, p.lse_part, static_cast<T*>(o), lse, s.B, s.H, s.N, s.n_split);
+    fa_combine_kernel<typename Elem<T>::Out, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        p.o_part, p.lse_part, static_cast<typename Elem<T>::Out*>(o), lse, s.B, s.H, s.N,
+        s.n_split);
     rc = launch_status(cudaGetLastError());
     note_launches(1);
   }
@@ -1317,26 +1350,27 @@ static int launch_fwd(Kernel kern, const FwdSchedule& s, const void* q, const vo
 
 template <class T, class Tr>
 static int run_single(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
-                      float* lse, float scale, long long tok_in, cudaStream_t stream) {
-  static_assert(Tr::BM == 128, "unit rows");
+                      float* lse, float scale, float o_scale, long long tok_in,
+                      cudaStream_t stream) {
+  static_assert(Tr::BM == 128 && Tr::EB == Elem<T>::kBytes, "unit rows, element size");
   return launch_fwd<T, Tr::D, Tr::BN, 224, Tr::SMEM_BYTES, false>(
-      s.cu ? fa_fwd_kernel<T, Tr, true> : fa_fwd_kernel<T, Tr, false>, s, q, k,
-                                                                   v, o, lse, scale, tok_in, stream);
+      s.cu ? fa_fwd_kernel<T, Tr, true> : fa_fwd_kernel<T, Tr, false>, s, q, k, v, o, lse, scale,
+      o_scale, tok_in, stream);
 }
 
 template <class T, class Tr>
 static int run_pp(const FwdSchedule& s, const void* q, const void* k, const void* v, void* o,
-                  float* lse, float scale, long long tok_in, cudaStream_t stream) {
-  static_assert(2 * Tr::BM == 256, "unit rows");
+                  float* lse, float scale, float o_scale, long long tok_in, cudaStream_t stream) {
+  static_assert(2 * Tr::BM == 256 && Tr::EB == Elem<T>::kBytes, "unit rows, element size");
   return launch_fwd<T, Tr::D, Tr::BN, 384, Tr::SMEM_BYTES, true>(
-      s.cu ? fa_fwd_pp_kernel<T, Tr, true> : fa_fwd_pp_kernel<T, Tr, false>, s, q, k,
-                                                                 v, o, lse, scale, tok_in, stream);
+      s.cu ? fa_fwd_pp_kernel<T, Tr, true> : fa_fwd_pp_kernel<T, Tr, false>, s, q, k, v, o, lse,
+      scale, o_scale, tok_in, stream);
 }
 
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream,
-               const int* cu, int total) {
+               const int* cu, int total, float o_scale) {
   DeviceInfo dev;
   int rc = current_device(&dev);
   if (rc != FA_OK) return rc;
@@ -1347,31 +1381,48 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
     s.cu = cu;
     s.total = total;
   }
-  switch (d) {
-    case 64:
-      return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, tok_in, stream)
-                    : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale, tok_in,
-                                                               stream);
-    case 96:
-      return s.pair ? run_pp<T, FwdPPTraits<96, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream)
-                    : run_single<T, FwdTraits<96, 128, 3, 2>>(s, q, k, v, o, lse, scale, tok_in,
-                                                               stream);
-    case 128:
-      return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream)
-                    : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale, tok_in,
-                                                                stream);
-    case 256:
-      return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, tok_in, stream);
-    default:
-      return FA_ERR_HEADDIM;
+  if constexpr (Elem<T>::kF8) {
+    // 8-bit Q, K, V: d = 128 (one 128-byte chunk a row); the stages are half
+    // the bytes of the 16-bit ones, so the pair kernel keeps four of each
+    if (d != 128) return FA_ERR_HEADDIM;
+    return s.pair ? run_pp<T, FwdPPTraits<128, 4, 4, 1>>(s, q, k, v, o, lse, scale, o_scale,
+                                                         tok_in, stream)
+                  : run_single<T, FwdTraits<128, 128, 3, 2, 1>>(s, q, k, v, o, lse, scale,
+                                                                o_scale, tok_in, stream);
+  } else {
+    switch (d) {
+      case 64:
+        return s.pair ? run_pp<T, FwdPPTraits<64, 4, 4>>(s, q, k, v, o, lse, scale, o_scale,
+                                                         tok_in, stream)
+                      : run_single<T, FwdTraits<64, 128, 4, 4>>(s, q, k, v, o, lse, scale,
+                                                                 o_scale, tok_in, stream);
+      case 96:
+        return s.pair ? run_pp<T, FwdPPTraits<96, 2, 2>>(s, q, k, v, o, lse, scale, o_scale,
+                                                         tok_in, stream)
+                      : run_single<T, FwdTraits<96, 128, 3, 2>>(s, q, k, v, o, lse, scale,
+                                                                 o_scale, tok_in, stream);
+      case 128:
+        return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2>>(s, q, k, v, o, lse, scale, o_scale,
+                                                          tok_in, stream)
+                      : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale,
+                                                                  o_scale, tok_in, stream);
+      case 256:
+        return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, o_scale,
+                                                        tok_in, stream);
+      default:
+        return FA_ERR_HEADDIM;
+    }
   }
 }
 
 template int fwd_launch<__nv_bfloat16>(const void*, const void*, const void*, void*, float*, int,
                                        int, int, int, float, unsigned, long long, cudaStream_t,
-                                       const int*, int);
+                                       const int*, int, float);
 template int fwd_launch<__half>(const void*, const void*, const void*, void*, float*, int, int,
                                 int, int, float, unsigned, long long, cudaStream_t, const int*,
-                                int);
+                                int, float);
+template int fwd_launch<__nv_fp8_e4m3>(const void*, const void*, const void*, void*, float*, int,
+                                       int, int, int, float, unsigned, long long, cudaStream_t,
+                                       const int*, int, float);
 
 }  // namespace fa

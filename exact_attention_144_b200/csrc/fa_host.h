@@ -47,12 +47,13 @@ void scratch_free(void* ptr, cudaStream_t stream);
 // Device address of this library's status word on the current device.
 unsigned long long* device_status_ptr();
 
-// Tensor map over a contiguous [B, N, H, d] 16-bit tensor for TMA tile loads
-// of `box_rows` tokens x 64 elements of one head (128 bytes, 128-byte swizzle).
-// Rows past N are filled with zeros by the hardware.
+// Tensor map over a contiguous [B, N, H, d] tensor for TMA tile loads of
+// `box_rows` tokens x 128 bytes of one head (64 16-bit or 128 8-bit elements,
+// 128-byte swizzle).  fmt: 0 fp16, 1 bf16, 2 one-byte elements (E4M3).
+// Rows past N, and elements past d, are filled with zeros by the hardware.
 // tok_stride: elements from one token to the next (H*d for [B,N,H,d]; 3*H*d
 // for one of Q, K, V inside a packed [B,N,3,H,d] tensor).
-int make_tmap_bnhd(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d,
+int make_tmap_bnhd(CUtensorMap* map, const void* base, int fmt, int B, int N, int H, int d,
                    int box_rows, long long tok_stride);
 
 // Tensor map over a contiguous [rows, cols] fp32 matrix for TMA tiles of
@@ -111,10 +112,12 @@ int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 // tok_in: token stride of q, k, v (elements); tok_g: of dq, dk, dv.  o, lse,
 // dout are always contiguous [B,N,H,d] / [B,H,N].
 // cu (varlen): device [B+1] sequence starts, N = max_seqlen, total tokens; else null.
+// T = __nv_fp8_e4m3: q, k, v are E4M3 (d = 128 only), o is bf16, and o_scale
+// multiplies O as it is stored (the V descale; the Q, K descales are in scale).
 template <class T>
 int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int N, int d, float scale, unsigned flags, long long tok_in, cudaStream_t stream,
-               const int* cu = nullptr, int total = 0);
+               const int* cu = nullptr, int total = 0, float o_scale = 1.f);
 template <class T>
 int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,

@@ -105,6 +105,27 @@ int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
               cudaStream_t stream);
 
 /*
+ * Forward pass on 8-bit inputs.  The pages point this way through the
+ * multiplied gains of reduced-precision inputs with FlashAttention-2 (YOLO11
+ * page, section 5.3) and 8-bit deployment (YOLO integration page, deployment
+ * paragraph).  q, k, v: contiguous [B, N, H, d] device arrays of
+ * OCP FP8 E4M3 bytes (1 sign, 4 exponent, 3 mantissa bits, bias 7, no
+ * infinities; torch.float8_e4m3fn), each with a per-tensor descale factor:
+ * the attention computed is the one of (descale_q q, descale_k k, descale_v v)
+ * with `scale`, i.e. S = scale descale_q descale_k q k^T, O = descale_v
+ * softmax(S) v.  o: [B, N, H, d] bf16; lse: [B, H, N] fp32, natural log of
+ * that S.  d must be 128 (FA_ERR_HEADDIM otherwise); flags as fa_fwd_ex
+ * (FA_FLAG_CAUSAL).  Arithmetic: Q K^T and P V on the 8-bit tensor-core path
+ * with fp32 accumulation; the softmax in fp32; P is rounded to E4M3 (round
+ * to nearest even) before P V, while the row sums use the unrounded values.
+ * A non-finite descale, or scale * descale_q * descale_k not finite, gives
+ * FA_ERR_SCALE.  Pointers 16-byte aligned; ownership and errors as fa_fwd.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+               int B, int H, int N, int d, float scale, float descale_q,
+               float descale_k, float descale_v, unsigned flags, cudaStream_t stream);
+
+/*
  * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
  * Inputs q, k, v, o (the forward output), dout (upstream gradient of o) and
  * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64, 96 or

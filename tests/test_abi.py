@@ -139,6 +139,43 @@ def test_ex_entry_points_reject_bad_flags_and_types():
     assert fa.fa_status_string(fa.FA_ERR_FLAGS) == "unknown flag bits"
 
 
+def test_fp8_entry_validates_before_any_cuda_call():
+    import ctypes
+    import exact_attention_144_b200 as fa
+    lib = fa.lib()
+    buf = (ctypes.c_char * 4096)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    mis = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256 + 8)
+    one = ctypes.c_float(1.0)
+
+    def call(ptrs=None, d=128, scale=0.125, dq=1.0, dk=1.0, dv=1.0, flags=0, B=1):
+        ptrs = ptrs or [p] * 5
+        return lib.fa_fwd_fp8(*ptrs, B, 1, 8, d, ctypes.c_float(scale), ctypes.c_float(dq),
+                              ctypes.c_float(dk), ctypes.c_float(dv), flags, None)
+    for i in range(5):
+        ptrs = [p] * 5
+        ptrs[i] = None
+        assert call(ptrs) == fa.FA_ERR_NULL
+        ptrs[i] = mis
+        assert call(ptrs) == fa.FA_ERR_ALIGN
+    for d in (64, 96, 256):  # the 8-bit path is built for d = 128 only
+        assert call(d=d) == fa.FA_ERR_HEADDIM
+    assert call(B=0) == fa.FA_ERR_SHAPE
+    assert call(dq=math.nan) == fa.FA_ERR_SCALE
+    assert call(dv=math.inf) == fa.FA_ERR_SCALE
+    assert call(scale=1e30, dq=1e30) == fa.FA_ERR_SCALE  # the folded score scale overflows
+    assert call(flags=2) == fa.FA_ERR_FLAGS
+    del one
+
+
+def test_fp8_binding_checks_types():
+    import torch
+    import exact_attention_144_b200 as fa
+    x = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises((TypeError, ValueError)):
+        fa.fa_fwd_fp8(x, x, x)
+
+
 def test_varlen_bounds_clamp_every_input_into_range():
     # the rule the varlen kernels apply to cu_seqlens: whatever the contents,
     # each sequence lies inside [0, total) and holds at most max_seqlen tokens
