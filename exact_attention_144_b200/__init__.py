@@ -90,6 +90,9 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_plan_pieces_ex.argtypes = [i, i, i, i, ctypes.c_uint, i, i,
                                           ctypes.POINTER(ctypes.c_int), i]
     lib.fa_fwd_plan_pieces_ex.restype = i
+    lib.fa_bwd_plan.argtypes = [i, i, i, i, ctypes.c_uint, i, ctypes.POINTER(ctypes.c_int),
+                                ctypes.POINTER(ctypes.c_int)]
+    lib.fa_bwd_plan.restype = i
     _lib = lib
     return lib
 
@@ -273,6 +276,16 @@ def fa_fwd_fp8(q, k, v, descale_q=1.0, descale_k=1.0, descale_v=1.0, o=None, lse
     if rc != FA_OK:
         raise FAError("fa_fwd_fp8", rc)
     return o, lse
+
+
+def fa_bwd_plan(B, H, N, d, sm_count, flags=0):
+    """The backward's decomposition: {"n_split": blocks per key tile,
+    "grid": blocks} (host only; same code as the launch)."""
+    ns, grid = ctypes.c_int(), ctypes.c_int()
+    rc = _load().fa_bwd_plan(B, H, N, d, int(flags), sm_count, ctypes.byref(ns), ctypes.byref(grid))
+    if rc != FA_OK:
+        raise FAError("fa_bwd_plan", rc)
+    return {"n_split": ns.value, "grid": grid.value}
 
 
 def fa_fwd_ex(q, k, v, o=None, lse=None, scale=None, flags=0, stream=None):

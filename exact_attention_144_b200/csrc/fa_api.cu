@@ -511,6 +511,13 @@ FA_EXPORT int fa_fwd_plan(int B, int H, int N, int d, int sm_count, fa_fwd_plan_
   return fa_fwd_plan_ex(B, H, N, d, 0u, sm_count, plan);
 }
 
+FA_EXPORT int fa_bwd_plan(int B, int H, int N, int d, unsigned flags, int sm_count,
+                          int* n_split, int* grid_blocks) {
+  if (n_split == nullptr || grid_blocks == nullptr) return FA_ERR_NULL;
+  if ((flags & ~fa::kKnownFlags) != 0) return FA_ERR_FLAGS;
+  return fa::plan_bwd(B, H, N, d, flags, sm_count, n_split, grid_blocks);
+}
+
 FA_EXPORT int fa_fwd_plan_pieces_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
                                     int block, int* pieces, int max_pieces) {
   if (pieces == nullptr && max_pieces > 0) return FA_ERR_NULL;

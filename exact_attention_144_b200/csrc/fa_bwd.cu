@@ -88,7 +88,56 @@ struct BwdParams {
   float scale;
   unsigned long long limit_ns;
   unsigned long long* status;
+  // split query ranges (kernels instantiated with SPLIT): n_split blocks per
+  // key tile, block x = key tile * n_split + split; each writes its fp32
+  // partial dK (scaled), dV to dk_part / dv_part + split * part_stride, laid
+  // out [B*N tokens, H, D], and fa_bwd_dkv_kernel sums them
+  int n_split;
+  float* dk_part;
+  float* dv_part;
+  long long part_stride;
 };
+
+// Stores 32 d columns (from column col) of key row `key`'s dV and scale*dK
+// (fp32 TMEM words a, k2): rounded to T at dk/dv + off, or, for a split
+// block, as fp32 into its partial slice.
+template <class T, bool SPLIT>
+__device__ __forceinline__ void store_dkv32(const BwdParams& p, size_t tok, int h, int col, int sp,
+                                            const uint32_t (&a)[32], const uint32_t (&k2)[32],
+                                            int D) {
+  if constexpr (SPLIT) {
+    const size_t at = (size_t)sp * p.part_stride + (tok * p.H + h) * D + col;
+    float4* dvp = reinterpret_cast<float4*>(p.dv_part + at);
+    float4* dkp = reinterpret_cast<float4*>(p.dk_part + at);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      dvp[j] = make_float4(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1]),
+                           __uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3]));
+      dkp[j] = make_float4(__uint_as_float(k2[4 * j]) * p.scale,
+                           __uint_as_float(k2[4 * j + 1]) * p.scale,
+                           __uint_as_float(k2[4 * j + 2]) * p.scale,
+                           __uint_as_float(k2[4 * j + 3]) * p.scale);
+    }
+  } else {
+    const size_t off = tok * p.tok_g + (size_t)h * D + col;
+    uint4 va[4], vk[4];
+    uint32_t* pa = reinterpret_cast<uint32_t*>(va);
+    uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
+      pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
+                             __uint_as_float(k2[2 * j + 1]) * p.scale);
+    }
+    uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dv) + off);
+    uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dk) + off);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dvp[j] = va[j];
+      dkp[j] = vk[j];
+    }
+  }
+}
 
 enum { kBSiteQEmpty = 0x21, kBSiteKV, kBSiteQFull, kBSiteDsReady, kBSiteDqFree, kBSiteSFull,
        kBSiteDpFull, kBSiteQFullSm, kBSiteDsBuf, kBSiteDqFull, kBSiteKvDone, kBSitePReady };
@@ -128,7 +177,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <class T, class Tr, bool CAUSAL, bool VARLEN>
+template <class T, class Tr, bool CAUSAL, bool VARLEN, bool SPLIT = false>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -151,15 +200,20 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int sp = SPLIT ? (int)blockIdx.x % p.n_split : 0;  // split of the query range
+  const int kt = SPLIT ? (int)blockIdx.x / p.n_split : (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
   int tb, tok0, len;
   seq_bounds(VARLEN ? p.cu : nullptr, b, p.N, p.total, tb, tok0, len);
   if (kt * BN >= len) return;  // block-uniform, before any barrier or allocation
   // causal: query tiles wholly before this key tile see none of its keys
-  const int i0 = CAUSAL ? (kt * BN) / BM : 0;
-  const int n_qt = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - i0;  // tile i is global i0 + i
+  const int q0 = CAUSAL ? (kt * BN) / BM : 0;
+  const int q_all = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - q0;
+  // tile i is global i0 + i; a split block takes its share of the range
+  const int i0 = SPLIT ? q0 + q_all * sp / p.n_split : q0;
+  const int n_qt = SPLIT ? q_all * (sp + 1) / p.n_split - q_all * sp / p.n_split : q_all;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -463,31 +517,14 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = ((size_t)tb * p.total + tok0 + key) * p.tok_g + (size_t)h * D + hf * 32;
       uint32_t a[32], k2[32];
       tmem_ld32(tl + Tr::TM_DV + hf * 32, a);
       tmem_ld32(tl + Tr::TM_DK + hf * 32, k2);
       tmem_wait_ld();
       reg_fence(a);
       reg_fence(k2);
-      uint4 va[4], vk[4];
-      uint32_t* pa = reinterpret_cast<uint32_t*>(va);
-      uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
-        pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
-                               __uint_as_float(k2[2 * j + 1]) * p.scale);
-      }
-      if (key_valid) {
-        uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dv) + off);
-        uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dk) + off);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          dvp[j] = va[j];
-          dkp[j] = vk[j];
-        }
-      }
+      if (key_valid)
+        store_dkv32<T, SPLIT>(p, (size_t)tb * p.total + tok0 + key, h, hf * 32, sp, a, k2, D);
     }
   }
 
@@ -565,7 +602,7 @@ struct BwdTqTraits {
 using BwdTq128 = BwdTqTraits<128, 3>;
 using BwdTq96 = BwdTqTraits<96, 3>;
 
-template <class T, class Tr, bool CAUSAL, bool VARLEN>
+template <class T, class Tr, bool CAUSAL, bool VARLEN, bool SPLIT = false>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_tq_kernel(const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk,
@@ -589,15 +626,20 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int sp = SPLIT ? (int)blockIdx.x % p.n_split : 0;  // split of the query range
+  const int kt = SPLIT ? (int)blockIdx.x / p.n_split : (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
   int tb, tok0, len;
   seq_bounds(VARLEN ? p.cu : nullptr, b, p.N, p.total, tb, tok0, len);
   if (kt * BN >= len) return;  // block-uniform, before any barrier or allocation
   // causal: query tiles wholly before this key tile see none of its keys
-  const int i0 = CAUSAL ? (kt * BN) / BM : 0;
-  const int n_qt = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - i0;  // tile i is global i0 + i
+  const int q0 = CAUSAL ? (kt * BN) / BM : 0;
+  const int q_all = (VARLEN ? (len + BM - 1) / BM : p.n_qt) - q0;
+  // tile i is global i0 + i; a split block takes its share of the range
+  const int i0 = SPLIT ? q0 + q_all * sp / p.n_split : q0;
+  const int n_qt = SPLIT ? q_all * (sp + 1) / p.n_split - q_all * sp / p.n_split : q_all;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -888,7 +930,6 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int key = kt * BN + r;
-      const size_t off = ((size_t)tb * p.total + tok0 + key) * p.tok_g + (size_t)h * D;
 #pragma unroll
       for (int cc = hf; cc < D / 32; cc += 2) {
         const int col = cc * 32;
@@ -898,24 +939,8 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         reg_fence(a);
         reg_fence(k2);
-        uint4 va[4], vk[4];
-        uint32_t* pa = reinterpret_cast<uint32_t*>(va);
-        uint32_t* pkk = reinterpret_cast<uint32_t*>(vk);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          pa[j] = Elem<T>::pack(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
-          pkk[j] = Elem<T>::pack(__uint_as_float(k2[2 * j]) * p.scale,
-                                 __uint_as_float(k2[2 * j + 1]) * p.scale);
-        }
-        if (key_valid) {
-          uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dv) + off + col);
-          uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dk) + off + col);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            dvp[j] = va[j];
-            dkp[j] = vk[j];
-          }
-        }
+        if (key_valid)
+          store_dkv32<T, SPLIT>(p, (size_t)tb * p.total + tok0 + key, h, col, sp, a, k2, D);
       }
     }
   }
@@ -1013,15 +1038,75 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
   *reinterpret_cast<uint4*>(dq + ((size_t)tb * total + tok0 + i) * tok_g + (size_t)h * D + x) = out;
 }
 
+// dK, dV = sum over the splits of the fp32 partials, rounded; 8 elements per
+// thread over the [B*N tokens, H, D] partial layout.  dk, dv rows are tok_g
+// elements apart.
+template <class T, int D>
+__global__ void __launch_bounds__(256) fa_bwd_dkv_kernel(const float* __restrict__ dk_part,
+                                                         const float* __restrict__ dv_part,
+                                                         int n_split, long long part_stride,
+                                                         T* __restrict__ dk, T* __restrict__ dv,
+                                                         int H, long long tok_g) {
+  const long long e = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
+  if (e >= part_stride) return;
+  const long long tok = e / ((long long)H * D);
+  const int hx = (int)(e % ((long long)H * D));
+  float a[8], c[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = c[j] = 0.f;
+  for (int sp = 0; sp < n_split; ++sp) {
+    const float4* pk = reinterpret_cast<const float4*>(dk_part + sp * part_stride + e);
+    const float4* pv = reinterpret_cast<const float4*>(dv_part + sp * part_stride + e);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float4 x = __ldcs(pk + h2), y = __ldcs(pv + h2);
+      a[4 * h2] += x.x; a[4 * h2 + 1] += x.y; a[4 * h2 + 2] += x.z; a[4 * h2 + 3] += x.w;
+      c[4 * h2] += y.x; c[4 * h2 + 1] += y.y; c[4 * h2 + 2] += y.z; c[4 * h2 + 3] += y.w;
+    }
+  }
+  uint4 ok, ov;
+  ok.x = Elem<T>::pack(a[0], a[1]); ok.y = Elem<T>::pack(a[2], a[3]);
+  ok.z = Elem<T>::pack(a[4], a[5]); ok.w = Elem<T>::pack(a[6], a[7]);
+  ov.x = Elem<T>::pack(c[0], c[1]); ov.y = Elem<T>::pack(c[2], c[3]);
+  ov.z = Elem<T>::pack(c[4], c[5]); ov.w = Elem<T>::pack(c[6], c[7]);
+  *reinterpret_cast<uint4*>(dk + tok * tok_g + hx) = ok;
+  *reinterpret_cast<uint4*>(dv + tok * tok_g + hx) = ov;
+}
+
+// Number of blocks per key tile: one, unless splitting each key tile's query
+// range over s blocks fills the waves of one-block-per-SM launches clearly
+// better (efficiency = blocks / (waves * SMs), less 0.03 per extra split for
+// the partial dK/dV traffic and pipeline refills), keeping >= 8 query tiles
+// a block.
+static int choose_bwd_split(long long blocks, int n_qt, int sm_count) {
+  auto eff = [&](long long b) {
+    const long long waves = (b + sm_count - 1) / sm_count;
+    return (double)b / (double)(waves * sm_count);
+  };
+  int best = 1;
+  double best_e = eff(blocks);
+  for (int sp = 2; sp <= 4 && n_qt / sp >= 8; ++sp) {
+    const double e = eff(blocks * sp) - 0.03 * (sp - 1);
+    if (e > best_e + 0.02) {
+      best = sp;
+      best_e = e;
+    }
+  }
+  return best;
+}
+
 // The three launches of one backward pass with scratch at ws (ws_bytes from
-// bwd_scratch_bytes): pre-pass, main kernel, dQ conversion.
+// bwd_scratch_bytes): pre-pass, main kernel, dQ conversion.  With n_split > 1
+// the main kernel is the SPLIT instantiation and a fourth launch sums its
+// partial dK, dV.
 template <class T, class Tr>
 static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                                    const CUtensorMap, const CUtensorMap, const BwdParams),
                       void* ws, const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                       int H, int N, float scale, long long tok_in, long long tok_g,
-                      cudaStream_t stream, bool timed, const int* cu, int total) {
+                      cudaStream_t stream, bool timed, const int* cu, int total,
+                      int n_split = 1) {
   constexpr int D = Tr::D;
   const bool bf16 = Elem<T>::kFmt == 1;
   CUtensorMap tmq, tmk, tmv, tmdo, tmacc;
@@ -1057,6 +1142,12 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   p.scale = scale;
   p.limit_ns = 4000000000ull;
   p.status = device_status_ptr();
+  p.n_split = n_split;
+  if (n_split > 1) {  // partials after the rows' D: bwd_scratch_bytes counts them
+    p.part_stride = (long long)B * N * H * D;
+    p.dk_part = dvec + rows;
+    p.dv_part = p.dk_part + (size_t)n_split * p.part_stride;
+  }
   if ((rc = make_tmap_f32_rows(&tmacc, p.dq_acc, rows, D, 32, Tr::ACC_BOX_ROWS)) != FA_OK)
     return rc;
   if ((rc = check_launch_regs((const void*)kern)) != FA_OK) return rc;
@@ -1076,12 +1167,19 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (timed) take_kernel_events(true, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  kern<<<dim3((N + Tr::BN - 1) / Tr::BN, H, B), 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo,
-                                                                              tmacc, p);
+  kern<<<dim3((N + Tr::BN - 1) / Tr::BN * n_split, H, B), 384, Tr::SMEM_BYTES, stream>>>(
+      tmq, tmk, tmv, tmdo, tmacc, p);
   rc = launch_status(cudaGetLastError());
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);
   if (rc != FA_OK) return rc;
+  if (n_split > 1) {
+    fa_bwd_dkv_kernel<T, D><<<(unsigned)((p.part_stride / 8 + 255) / 256), 256, 0, stream>>>(
+        p.dk_part, p.dv_part, n_split, p.part_stride, static_cast<T*>(dk), static_cast<T*>(dv), H,
+        tok_g);
+    note_launches(1);
+    if ((rc = launch_status(cudaGetLastError())) != FA_OK) return rc;
+  }
   const long long acc_elems = (long long)rows * D;
   fa_bwd_dq_kernel<T, D><<<(unsigned)((acc_elems / 8 + 255) / 256), 256, 0, stream>>>(
       p.dq_acc, static_cast<T*>(dq), B, H, N, Npad, scale, tok_g, cu, total);
@@ -1090,9 +1188,10 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
 }
 
 template <class Tr>
-static size_t bwd_scratch_bytes(int B, int H, int N) {
+static size_t bwd_scratch_bytes(int B, int H, int N, int n_split = 1) {
   const size_t rows = (size_t)B * H * ((N + Tr::BM - 1) / Tr::BM) * Tr::BM;
-  return rows * Tr::D * sizeof(float) + 2 * rows * sizeof(float);
+  const size_t parts = n_split > 1 ? 2 * (size_t)n_split * B * N * H * Tr::D : 0;
+  return (rows * Tr::D + 2 * rows + parts) * sizeof(float);
 }
 
 template <class T, class Tr>
@@ -1101,14 +1200,49 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
                    const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, float scale,
                    long long tok_in, long long tok_g, cudaStream_t stream, const int* cu,
-                   int total) {
+                   int total, int n_split = 1) {
   void* ws = nullptr;
-  int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N), stream);
+  int rc = scratch_alloc(&ws, bwd_scratch_bytes<Tr>(B, H, N, n_split), stream);
   if (rc != FA_OK) return rc;
   rc = launch_bwd<T, Tr>(kern, ws, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in, tok_g,
-                         stream, true, cu, total);
+                         stream, true, cu, total, n_split);
   scratch_free(ws, stream);
   return rc;
+}
+
+// Split choice for a fixed-length, non-causal batch (causal key tiles see
+// unequal query ranges and varlen sequences unequal lengths: those keep one
+// block per key tile).
+template <class Tr>
+static int bwd_split(int B, int H, int N, unsigned flags, const int* cu, int sm_count) {
+  if ((flags & 1u) || cu != nullptr) return 1;
+  const long long blocks = (long long)((N + Tr::BN - 1) / Tr::BN) * H * B;
+  return choose_bwd_split(blocks, (N + Tr::BM - 1) / Tr::BM, sm_count);
+}
+
+int plan_bwd(int B, int H, int N, int d, unsigned flags, int sm_count, int* n_split,
+             int* grid_blocks) {
+  if (B < 1 || H < 1 || N < 1 || sm_count < 1) return FA_ERR_SHAPE;
+  int ns, bn;
+  switch (d) {
+    case 64:
+      ns = bwd_split<BwdTraits64>(B, H, N, flags, nullptr, sm_count);
+      bn = BwdTraits64::BN;
+      break;
+    case 96:
+      ns = bwd_split<BwdTq96>(B, H, N, flags, nullptr, sm_count);
+      bn = BwdTq96::BN;
+      break;
+    case 128:
+      ns = bwd_split<BwdTq128>(B, H, N, flags, nullptr, sm_count);
+      bn = BwdTq128::BN;
+      break;
+    default:
+      return FA_ERR_HEADDIM;
+  }
+  *n_split = ns;
+  *grid_blocks = (int)((long long)((N + bn - 1) / bn) * ns * H * B);
+  return FA_OK;
 }
 
 template <class T>
@@ -1121,28 +1255,34 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
   if (rc != FA_OK) return rc;
   switch (d) {
     case 64: {
+      const int ns = bwd_split<BwdTraits64>(B, H, N, flags, cu, dev.sm_count);
       auto kern = (flags & 1u) ? (cu ? fa_bwd_kernel<T, BwdTraits64, true, true>
                                      : fa_bwd_kernel<T, BwdTraits64, true, false>)
                                : (cu ? fa_bwd_kernel<T, BwdTraits64, false, true>
-                                     : fa_bwd_kernel<T, BwdTraits64, false, false>);
+                                     : ns > 1 ? fa_bwd_kernel<T, BwdTraits64, false, false, true>
+                                              : fa_bwd_kernel<T, BwdTraits64, false, false>);
       return run_bwd<T, BwdTraits64>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale,
-                                     tok_in, tok_g, stream, cu, total);
+                                     tok_in, tok_g, stream, cu, total, ns);
     }
     case 96: {
+      const int ns = bwd_split<BwdTq96>(B, H, N, flags, cu, dev.sm_count);
       auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq96, true, true>
                                      : fa_bwd_tq_kernel<T, BwdTq96, true, false>)
                                : (cu ? fa_bwd_tq_kernel<T, BwdTq96, false, true>
-                                     : fa_bwd_tq_kernel<T, BwdTq96, false, false>);
+                                     : ns > 1 ? fa_bwd_tq_kernel<T, BwdTq96, false, false, true>
+                                              : fa_bwd_tq_kernel<T, BwdTq96, false, false>);
       return run_bwd<T, BwdTq96>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
-                                 tok_g, stream, cu, total);
+                                 tok_g, stream, cu, total, ns);
     }
     case 128: {
+      const int ns = bwd_split<BwdTq128>(B, H, N, flags, cu, dev.sm_count);
       auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq128, true, true>
                                      : fa_bwd_tq_kernel<T, BwdTq128, true, false>)
                                : (cu ? fa_bwd_tq_kernel<T, BwdTq128, false, true>
-                                     : fa_bwd_tq_kernel<T, BwdTq128, false, false>);
+                                     : ns > 1 ? fa_bwd_tq_kernel<T, BwdTq128, false, false, true>
+                                              : fa_bwd_tq_kernel<T, BwdTq128, false, false>);
       return run_bwd<T, BwdTq128>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
-                                  tok_g, stream, cu, total);
+                                  tok_g, stream, cu, total, ns);
     }
     default:
       return FA_ERR_HEADDIM;

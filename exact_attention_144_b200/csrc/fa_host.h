@@ -108,6 +108,11 @@ size_t fwd_scratch_bytes(const FwdSchedule& s);
 // Returns the number of pieces (writes at most max_pieces).
 int fwd_block_pieces(const FwdSchedule& s, int blk, int* out, int max_pieces);
 
+// Backward decomposition for fixed-length batches: blocks per key tile
+// (n_split; > 1 splits each key tile's query range) and blocks in the grid.
+int plan_bwd(int B, int H, int N, int d, unsigned flags, int sm_count, int* n_split,
+             int* grid_blocks);
+
 // Launchers (argument validation is done by the callers in fa_api.cu).
 // tok_in: token stride of q, k, v (elements); tok_g: of dq, dk, dv.  o, lse,
 // dout are always contiguous [B,N,H,d] / [B,H,N].

@@ -266,6 +266,19 @@ int fa_fwd_plan_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
                    fa_fwd_plan_t *plan);
 
 /*
+ * Host-only description of the backward's decomposition for a fixed-length
+ * batch on a device with sm_count SMs: *n_split blocks per 128-key tile
+ * (each takes an equal share of the tile's query tiles, and an extra kernel
+ * sums their fp32 dK, dV partials) and *grid_blocks blocks in all.  The split
+ * is used only without FA_FLAG_CAUSAL, when it fills the waves of
+ * one-block-per-SM launches clearly better (at least 8 query tiles a block).
+ * Returns FA_OK, FA_ERR_NULL, FA_ERR_FLAGS, FA_ERR_SHAPE or FA_ERR_HEADDIM
+ * (d other than 64, 96, 128).
+ */
+int fa_bwd_plan(int B, int H, int N, int d, unsigned flags, int sm_count, int *n_split,
+                int *grid_blocks);
+
+/*
  * The pieces block `block` (0 <= block < plan.grid) processes, in order,
  * 6 ints each: unit index, first K/V tile, end K/V tile, store kind
  * (0: whole result, 1: partial rows to the block's slot, 2: merge with the

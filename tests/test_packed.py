@@ -25,7 +25,7 @@ def fa():
 @pytest.mark.parametrize("B,N,H,d,dtype,causal", [
     (2, 300, 3, 64, "bf16", False), (1, 1000, 2, 128, "fp16", False), (1, 257, 2, 256, "bf16", False),
     (2, 513, 2, 64, "bf16", True), (1, 400, 4, 128, "bf16", True), (1, 700, 2, 96, "fp16", False),
-    (2, 300, 1, 96, "bf16", True)])
+    (2, 300, 1, 96, "bf16", True), (1, 2048, 2, 64, "bf16", False)])
 def test_packed_equals_unpacked(fa, B, N, H, d, dtype, causal):
     q, k, v, dout = attn_inputs.draw(B, N, H, d, dtype, 1800 + N + d, 4, device="cuda")
     qkv = torch.stack([q, k, v], dim=2).contiguous()  # [B, N, 3, H, d]

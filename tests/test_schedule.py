@@ -173,3 +173,25 @@ def test_unknown_flags_are_rejected():
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd_plan(1, 1, 64, 64, 148, 2)
     assert e.value.status == fa.FA_ERR_FLAGS
+
+
+# ------------------------------------------------------------ backward
+def test_backward_split_plans():
+    # one 384-thread block per SM: the split is taken when it fills the waves
+    # clearly better, never for causal batches, and keeps >= 8 query tiles a block
+    plan = lambda *a, **k: fa.fa_bwd_plan(*a, **k)  # noqa: E731
+    assert plan(4, 8, 4096, 64, 148) == {"n_split": 1, "grid": 1024}    # 99 % of 7 waves
+    assert plan(1, 8, 8192, 128, 148) == {"n_split": 2, "grid": 1024}   # 512 blocks: 86 %
+    assert plan(1, 1, 25600, 96, 148) == {"n_split": 2, "grid": 400}    # 200 blocks: 68 %
+    assert plan(1, 1, 25600, 96, 148, CAUSAL)["n_split"] == 1
+    assert plan(1, 2, 2048, 64, 148)["n_split"] == 2                    # 16 query tiles
+    assert plan(3, 5, 200, 64, 148)["n_split"] == 1                     # 2 query tiles
+    for B, H, N, d in [(1, 1, 1, 64), (2, 3, 5000, 128), (1, 7, 4097, 96), (8, 16, 2048, 64)]:
+        p = plan(B, H, N, d, 148)
+        n_q = -(-N // (128 if d == 64 else 64))
+        assert p["n_split"] == 1 or n_q // p["n_split"] >= 8
+        assert p["grid"] == -(-N // 128) * H * B * p["n_split"]
+    with pytest.raises(fa.FAError):
+        plan(1, 1, 64, 256, 148)
+    with pytest.raises(fa.FAError):
+        plan(1, 1, 64, 64, 148, 2)
