@@ -496,7 +496,7 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
 // ===========================================================================
 // fa_fwd_pp_kernel: two Q tiles per unit
 // ===========================================================================
-template <int D_, int KST_, int VST_, int EB_ = 2>
+template <int D_, int KST_, int VST_, int EB_ = 2, int EMU_ = -1>
 struct FwdPPTraits {
   static constexpr int D = D_;
   static constexpr int EB = EB_;          // bytes an element of Q, K, V
@@ -528,8 +528,10 @@ struct FwdPPTraits {
   // Otherwise (d = 128) P is written over the first BN/2 columns of its S.
   static constexpr bool SEP_P = 2 * BN + 2 * P_COLS + 2 * D <= 512;
   // exponentials on the FMA pipe per 8 column pairs (see softmax_step): the
-  // d = 128 warpgroups take turns, the d = 64 ones run together
-  static constexpr int EMU = SEP_P ? 0 : 2;
+  // d = 128 warpgroups take turns, the d = 64 ones run together.  Measured on
+  // B200 for d = 128 (bf16 / 8-bit, [1,8192,8,128], us): 1: 269.6 / 243.0,
+  // 2: 271.6 / 238.8, 3: 284.0 / 245.1 -- 2 is kept
+  static constexpr int EMU = EMU_ >= 0 ? EMU_ : (SEP_P ? 0 : 2);
   static constexpr uint32_t TM_P = 2 * BN;                      // used when SEP_P
   static constexpr uint32_t TM_O = SEP_P ? 3 * BN : 2 * BN;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -1382,10 +1384,11 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
     s.total = total;
   }
   if constexpr (Elem<T>::kF8) {
-    // 8-bit Q, K, V: d = 128 (one 128-byte chunk a row); the stages are half
-    // the bytes of the 16-bit ones, so the pair kernel keeps four of each
+    // 8-bit Q, K, V: d = 128 (one 128-byte chunk a row).  Two K and two V
+    // stages (measured on B200 at [1,8192,8,128]: 236.8 us, against 238.8 us
+    // with four of each)
     if (d != 128) return FA_ERR_HEADDIM;
-    return s.pair ? run_pp<T, FwdPPTraits<128, 4, 4, 1>>(s, q, k, v, o, lse, scale, o_scale,
+    return s.pair ? run_pp<T, FwdPPTraits<128, 2, 2, 1>>(s, q, k, v, o, lse, scale, o_scale,
                                                          tok_in, stream)
                   : run_single<T, FwdTraits<128, 128, 3, 2, 1>>(s, q, k, v, o, lse, scale,
                                                                 o_scale, tok_in, stream);
