@@ -44,14 +44,16 @@ L2_FLUSH_BYTES = 512 << 20
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the kernel sources hash to the recorded value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.761280e6 + 23.508992e6,
-                                                    "src": "bd813f6e40aaedbe"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.487040e6 + 1.794560e6,
-                                                       "src": "bd813f6e40aaedbe"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.907904e6 + 4.252672e6,
-                                                    "src": "bd813f6e40aaedbe"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.240832e6 + 19.283712e6,
-                                                     "src": "bd813f6e40aaedbe"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.759232e6 + 21.073152e6,
+                                                    "src": "532207f4dfa00c07"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.580736e6 + 2.517248e6,
+                                                       "src": "532207f4dfa00c07"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 51.360256e6 + 5.298176e6,
+                                                    "src": "532207f4dfa00c07"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.644544e6 + 113.935872e6,
+                                                     "src": "532207f4dfa00c07"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.289472e6 + 0.524288e6,
+                                                        "src": "532207f4dfa00c07"},
 }
 
 
