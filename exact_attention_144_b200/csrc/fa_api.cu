@@ -208,7 +208,8 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static int check_common(int B, int H, int N, int d, float scale, bool bwd) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
-  if (!(d == 64 || d == 96 || d == 128 || (!bwd && d == 256))) return FA_ERR_HEADDIM;
+  if (!(d == 64 || d == 96 || d == 128 || d == 256)) return FA_ERR_HEADDIM;
+  (void)bwd;
   if ((long long)B * N * H * d >= (1ll << 31)) return FA_ERR_SHAPE;
   if (!isfinite(scale)) return FA_ERR_SCALE;
   return FA_OK;

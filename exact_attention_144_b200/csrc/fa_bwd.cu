@@ -41,6 +41,7 @@
 namespace fa {
 
 struct BwdTraits64 {
+  static constexpr int NHALF = 1;  // blocks per key tile, one per slice of d
   static constexpr int D = 64;
   static constexpr int BN = 128;  // keys per block
   static constexpr int BM = 128;  // queries per inner tile
@@ -564,6 +565,15 @@ struct BwdTqTraits {
   static constexpr int BN = 128;  // keys per block
   static constexpr int BM = 64;   // queries per inner tile
   static constexpr int QST = QST_;
+  // d columns of dK, dV (and d rows of dQ^T) a block produces: all of them up
+  // to d = 128; at d = 256 two blocks per key tile take one 128-wide half
+  // each (S^T and dP^T still contract all 256)
+  static constexpr int DW = D < 128 ? D : 128;
+  static constexpr int NHALF = D / DW;
+  // dQ staging: one 32 x 32 fp32 box per compute warp, or (d = 256, where the
+  // full K, V tiles leave less room) one per lane quadrant, drained by warps
+  // 0-3 for both query halves
+  static constexpr int NBOX = NHALF > 1 ? 4 : 8;
   // 128-byte chunks along d; at d = 96 the last 32 columns of the second
   // chunk are the tensor map's zero fill
   static constexpr int KCH = (D + 63) / 64;
@@ -577,7 +587,7 @@ struct BwdTqTraits {
   static constexpr int OFF_DO = OFF_Q + QST * QT_BYTES;
   static constexpr int OFF_DS = OFF_DO + QST * QT_BYTES;
   static constexpr int OFF_STG = OFF_DS + DS_BYTES;
-  static constexpr int OFF_L = OFF_STG + 8 * BOX_BYTES;  // minus the base-2 LSE, per stage
+  static constexpr int OFF_L = OFF_STG + NBOX * BOX_BYTES;  // minus the base-2 LSE, per stage
   static constexpr int OFF_DD = OFF_L + QST * BM * 4;    // D per stage
   static constexpr int OFF_BAR = OFF_DD + QST * BM * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = B_Q_FULL + QST,
@@ -587,12 +597,12 @@ struct BwdTqTraits {
                        B_KV_DONE = B_DQ_FREE + 2, B_DRAIN = B_KV_DONE + 1, NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 256 + D;
+  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 256 + DW;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries
-  // dQ^T has d rows: one 128-lane MMA tile (rows past d are zero and never drained)
-  static_assert(D == 96 || D == 128, "the transposed-dQ layout holds d <= 128 rows");
-  static_assert(TM_DK + D <= TMEM_COLS, "tensor memory budget");
+  // dQ^T has DW rows: one 128-lane MMA tile (rows past d are zero and never drained)
+  static_assert(D == 96 || D == 128 || D == 256, "head sizes of the transposed-dQ kernel");
+  static_assert(TM_DK + DW <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0 && OFF_DS % 1024 == 0 &&
                     OFF_STG % 1024 == 0 && QT_BYTES % 1024 == 0,
@@ -601,6 +611,7 @@ struct BwdTqTraits {
 
 using BwdTq128 = BwdTqTraits<128, 3>;
 using BwdTq96 = BwdTqTraits<96, 3>;
+using BwdTq256 = BwdTqTraits<256, 1>;  // resident 64 KB K and V tiles leave one Q/dO stage
 
 template <class T, class Tr, bool CAUSAL, bool VARLEN, bool SPLIT = false>
 __global__ void __launch_bounds__(384, 1)
@@ -626,8 +637,12 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
+  static_assert(!(SPLIT && Tr::NHALF > 1), "query splits and d halves are not combined");
+  constexpr int DW = Tr::DW, NHALF = Tr::NHALF;
   const int sp = SPLIT ? (int)blockIdx.x % p.n_split : 0;  // split of the query range
-  const int kt = SPLIT ? (int)blockIdx.x / p.n_split : (int)blockIdx.x;
+  const int dh = NHALF > 1 ? (int)blockIdx.x % NHALF : 0;  // d half this block produces
+  const int kt = SPLIT ? (int)blockIdx.x / p.n_split
+                       : (NHALF > 1 ? (int)blockIdx.x / NHALF : (int)blockIdx.x);
   const int h = blockIdx.y, b = blockIdx.z;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
@@ -654,7 +669,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(Tr::B_DS_READY), 256);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Tr::B_DQ_FULL + s), 1);
-      mbar_init(bar(Tr::B_DQ_FREE + s), 256);
+      mbar_init(bar(Tr::B_DQ_FREE + s), 32 * Tr::NBOX);  // the draining warps
     }
     mbar_init(bar(Tr::B_KV_DONE), 2);
     mbar_init(bar(Tr::B_DRAIN), 2);
@@ -725,7 +740,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t fmt = Elem<T>::kFmt;
       constexpr uint32_t kIdescSP = f16_idesc(fmt, 128, BM, false);              // K-major x K-major
-      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, D, true);               // TS, B MN-major
+      constexpr uint32_t kIdescAcc = f16_idesc(fmt, 128, DW, true);              // TS, B MN-major
       constexpr uint32_t kIdescDQ = f16_idesc(fmt, 128, BM, true) | (1u << 15);  // A, B MN-major
       // Packed 16-bit P^T / dS^T: query half hf sits in the first 16 columns of
       // its own 32-column half of the S^T / dP^T region.
@@ -734,12 +749,17 @@ __global__ void __launch_bounds__(384, 1)
                      q_kmaj = sw128_desc(sQ, 16, 1024), do_kmaj = sw128_desc(sDO, 16, 1024),
                      q_mn = sw128_desc(sQ, BM * 128, 1024), do_mn = sw128_desc(sDO, BM * 128, 1024),
                      k_mn = sw128_desc(sK, BN * 128, 1024), ds_mn = sw128_desc(sDS, BN * 128, 1024);
+      // the block's d half starts DW/64 chunks into the Q, dO and K tiles
+      const uint32_t d_off_q = (uint32_t)(dh * (DW / 64) * (BM * 128));
+      const uint32_t d_off_k = (uint32_t)(dh * (DW / 64) * (BN * 128));
       // S^T = K Q_i^T into TM_S (stream a); dP^T = V dO_i^T into TM_DP (stream b)
       auto issue_first = [&](int i) {
         const uint64_t a0 = stream_a ? k_kmaj : v_kmaj;
         const uint64_t b0 = desc_advance(stream_a ? q_kmaj : do_kmaj, (i % QST) * Tr::QT_BYTES);
         const uint32_t d_tmem = tmem + (stream_a ? Tr::TM_S : Tr::TM_DP);
-#pragma unroll
+        // (at d = 256 partly unrolled: the issuing warps run on 88 registers)
+        constexpr int kUnroll = D > 128 ? 4 : D / 16;
+#pragma unroll kUnroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ch = kk >> 2, in = (kk & 3) * 32;
           umma_ss(leader, d_tmem, desc_advance(a0, ch * (BN * 128) + in),
@@ -762,7 +782,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             umma_ts(leader, tmem + Tr::TM_DV, tmem + Tr::TM_S + packed_col(kk),
-                    desc_advance(do_mn, qs * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    desc_advance(do_mn, qs * Tr::QT_BYTES + d_off_q + kk * 16 * 128), kIdescAcc,
                     (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_Q_EMPTY + qs));
         } else {
@@ -772,7 +792,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             umma_ts(leader, tmem + Tr::TM_DK, tmem + Tr::TM_DP + packed_col(kk),
-                    desc_advance(q_mn, qs * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
+                    desc_advance(q_mn, qs * Tr::QT_BYTES + d_off_q + kk * 16 * 128), kIdescAcc,
                     (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_Q_EMPTY + qs));
           // dQ_i^T = K^T dS_i^T  (A = K: d contiguous, MN-major; B = dS^T: queries
@@ -784,7 +804,8 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ss(leader, tmem + Tr::TM_DQ + qb * BM, desc_advance(k_mn, kk * 16 * 128),
+            umma_ss(leader, tmem + Tr::TM_DQ + qb * BM,
+                    desc_advance(k_mn, d_off_k + kk * 16 * 128),
                     desc_advance(ds_mn, kk * 16 * 128), kIdescDQ, kk > 0 ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_DQ_FULL + qb));
         }
@@ -810,36 +831,47 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const bool key_valid = kt * BN + r < len;
     const float c = p.sl2;
-    const uint32_t box = sSTG + warp * Tr::BOX_BYTES;
-    uint8_t* gbox = gSTG + warp * Tr::BOX_BYTES;
+    // staging box: one per warp, or (NBOX = 4) one per lane quadrant, whose
+    // warp 0-3 drains both query halves
+    constexpr int NH = 8 / Tr::NBOX;  // query halves a draining warp handles
+    const bool drains = warp < Tr::NBOX;
+    const uint32_t box = sSTG + (Tr::NBOX == 8 ? warp : quad) * Tr::BOX_BYTES;
+    uint8_t* gbox = gSTG + (Tr::NBOX == 8 ? warp : quad) * Tr::BOX_BYTES;
     bool ok = true;
 
-    // dQ^T tile i: TMEM -> this warp's swizzled fp32 staging box (32 queries x
+    // dQ^T tile i: TMEM -> the warp's swizzled fp32 staging box (32 queries x
     // 32 d) -> TMA reduce-add into the accumulator, issued by lane 0.
     auto drain_dq = [&](int i) -> bool {
       const int qb = i & 1;
       bool good = mbar_wait(bar(Tr::B_DQ_FULL + qb), (i >> 1) & 1, w, kBSiteDqFull);
       if (!__all_sync(0xffffffffu, good)) return false;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tl + Tr::TM_DQ + qb * BM + hf * 32, v);
-      tmem_wait_ld();
-      reg_fence(v);
-      tc_fence_before();
-      mbar_arrive(bar(Tr::B_DQ_FREE + qb));
-      if (lane == 0) bulk_wait_read_all();  // the previous reduce has read the box
-      __syncwarp();
-      // v[j] = dQ[query 32 hf + j][d = 32 quad + lane]; box row j holds query j
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        *reinterpret_cast<float*>(gbox + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) +
-                                  (lane & 3) * 4) = __uint_as_float(v[j]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && *abort_flag == 0 && quad * 32 < D) {  // d rows past D are padding
-        const int row = (int)(((size_t)b * p.H + h) * p.Npad + (size_t)(i0 + i) * BM + hf * 32);
-        tma_reduce_add_2d(&tmacc, box, quad * 32, row);
-        bulk_commit();
+      for (int e = 0; e < NH; ++e) {
+        const int half = NH == 1 ? hf : e;
+        uint32_t v[32];
+        tmem_ld32(tl + Tr::TM_DQ + qb * BM + half * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        if (e == NH - 1) {  // every read of this dQ^T buffer is done
+          tc_fence_before();
+          mbar_arrive(bar(Tr::B_DQ_FREE + qb));
+        }
+        if (lane == 0) bulk_wait_read_all();  // the previous reduce has read the box
+        __syncwarp();
+        // v[j] = dQ[query 32 half + j][d = 32 quad + lane]; box row j holds query j
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          *reinterpret_cast<float*>(gbox + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) +
+                                    (lane & 3) * 4) = __uint_as_float(v[j]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && *abort_flag == 0 && quad * 32 < DW) {  // d rows past d are padding
+          const int row =
+              (int)(((size_t)b * p.H + h) * p.Npad + (size_t)(i0 + i) * BM + half * 32);
+          tma_reduce_add_2d(&tmacc, box, dh * DW + quad * 32, row);
+          bulk_commit();
+        }
       }
       return true;
     };
@@ -920,9 +952,9 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(bar(Tr::B_DS_READY));
       // ---- dQ of the previous tile
-      if (i > 0 && !(ok = drain_dq(i - 1))) break;
+      if (drains && i > 0 && !(ok = drain_dq(i - 1))) break;
     }
-    if (ok && n_qt > 0) ok = drain_dq(n_qt - 1);
+    if (drains && ok && n_qt > 0) ok = drain_dq(n_qt - 1);
     if (lane == 0) bulk_wait_all();
     // ---- epilogue: dV and scale * dK, key row r, the 32-column d chunks
     // hf, hf + 2, ... (d = 96: chunks 0 and 2 for hf = 0, chunk 1 for hf = 1)
@@ -931,7 +963,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const int key = kt * BN + r;
 #pragma unroll
-      for (int cc = hf; cc < D / 32; cc += 2) {
+      for (int cc = hf; cc < DW / 32; cc += 2) {  // this block's d slice, from dh * DW
         const int col = cc * 32;
         uint32_t a[32], k2[32];
         tmem_ld32(tl + Tr::TM_DV + col, a);
@@ -940,7 +972,8 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(a);
         reg_fence(k2);
         if (key_valid)
-          store_dkv32<T, SPLIT>(p, (size_t)tb * p.total + tok0 + key, h, col, sp, a, k2, D);
+          store_dkv32<T, SPLIT>(p, (size_t)tb * p.total + tok0 + key, h, dh * DW + col, sp, a, k2,
+                                D);
       }
     }
   }
@@ -954,7 +987,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // Lanes of fa_bwd_pre_kernel per row: d / 8 rounded up to a power of two.
-constexpr int bwd_pre_lanes(int d) { return d <= 64 ? 8 : 16; }
+constexpr int bwd_pre_lanes(int d) { return d <= 64 ? 8 : d <= 128 ? 16 : 32; }
 
 // D_i = sum_x dO_ix O_ix; minus the base-2 LSE; zero the dQ accumulator.
 // Accumulator rows are (b, h, i) with i < Npad for every sequence b; rows past
@@ -1167,7 +1200,8 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (timed) take_kernel_events(true, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  kern<<<dim3((N + Tr::BN - 1) / Tr::BN * n_split, H, B), 384, Tr::SMEM_BYTES, stream>>>(
+  kern<<<dim3((N + Tr::BN - 1) / Tr::BN * n_split * Tr::NHALF, H, B), 384, Tr::SMEM_BYTES,
+         stream>>>(
       tmq, tmk, tmv, tmdo, tmacc, p);
   rc = launch_status(cudaGetLastError());
   if (ev1) cudaEventRecord(ev1, stream);
@@ -1215,7 +1249,7 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
 // block per key tile).
 template <class Tr>
 static int bwd_split(int B, int H, int N, unsigned flags, const int* cu, int sm_count) {
-  if ((flags & 1u) || cu != nullptr) return 1;
+  if ((flags & 1u) || cu != nullptr || Tr::NHALF > 1) return 1;
   const long long blocks = (long long)((N + Tr::BN - 1) / Tr::BN) * H * B;
   return choose_bwd_split(blocks, (N + Tr::BM - 1) / Tr::BM, sm_count);
 }
@@ -1237,11 +1271,15 @@ int plan_bwd(int B, int H, int N, int d, unsigned flags, int sm_count, int* n_sp
       ns = bwd_split<BwdTq128>(B, H, N, flags, nullptr, sm_count);
       bn = BwdTq128::BN;
       break;
+    case 256:  // two blocks per key tile, one per half of d; never split
+      ns = 1;
+      bn = BwdTq256::BN;
+      break;
     default:
       return FA_ERR_HEADDIM;
   }
   *n_split = ns;
-  *grid_blocks = (int)((long long)((N + bn - 1) / bn) * ns * H * B);
+  *grid_blocks = (int)((long long)((N + bn - 1) / bn) * ns * (d == 256 ? 2 : 1) * H * B);
   return FA_OK;
 }
 
@@ -1283,6 +1321,14 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
                                               : fa_bwd_tq_kernel<T, BwdTq128, false, false>);
       return run_bwd<T, BwdTq128>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
                                   tok_g, stream, cu, total, ns);
+    }
+    case 256: {
+      auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq256, true, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq256, true, false>)
+                               : (cu ? fa_bwd_tq_kernel<T, BwdTq256, false, true>
+                                     : fa_bwd_tq_kernel<T, BwdTq256, false, false>);
+      return run_bwd<T, BwdTq256>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
+                                  tok_g, stream, cu, total);
     }
     default:
       return FA_ERR_HEADDIM;

@@ -825,12 +825,10 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = __all_sync(0xffffffffu, ok))) break;
             tc_fence_after();
           }
-#pragma unroll
           store_p<T, BN>(p_col, pk);
           tmem_wait_st();
           if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(o_col, alpha);
         } else {
-#pragma unroll
           store_p<T, BN>(s_col, pk);
           tmem_wait_st();
           if (j > 0) {
@@ -1092,7 +1090,6 @@ __global__ void __launch_bounds__(224, 1)
         int valid = un.len - t * BN;
         if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
         const float alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
-#pragma unroll
         store_p<T, BN>(scol, pk);
         tmem_wait_st();
         if (i > 0) {

@@ -20,7 +20,7 @@
  *   16-bit floats (bf16 for the unsuffixed entry points, fp16 for *_f16);
  *   token stride H*d elements, head stride d.  lse: contiguous [B, H, N]
  *   fp32 device array (natural log).  Every pointer must be 16-byte aligned.
- *   d is 64, 96, 128 or 256 (fa_bwd: 64, 96 or 128); B, H, N >= 1; each tensor
+ *   d is 64, 96, 128 or 256; B, H, N >= 1; each tensor
  *   holds fewer than 2^31 elements.  scale is any finite float (normally
  *   1/sqrt(d)).  Arithmetic: 16-bit inputs, fp32 accumulation and softmax,
  *   outputs rounded to nearest even.
@@ -128,10 +128,11 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
 /*
  * Backward pass, bf16, by recompute (LLM explainer page, section 6.2).
  * Inputs q, k, v, o (the forward output), dout (upstream gradient of o) and
- * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64, 96 or
- * 128 (d = 64: 128-query inner tiles; d = 96 and 128: 64-query inner tiles
- * with dQ produced transposed, since five 128-column accumulators exceed
- * tensor memory); other d return FA_ERR_HEADDIM.
+ * lse (the forward's).  Overwrites dq, dk, dv [B,N,H,d].  d is 64, 96, 128
+ * or 256 (d = 64: 128-query inner tiles; d = 96, 128, 256: 64-query inner
+ * tiles with dQ produced transposed, since five 128-column accumulators
+ * exceed tensor memory; at d = 256 two blocks per key tile each produce one
+ * 128-wide half of dQ, dK, dV); other d return FA_ERR_HEADDIM.
  */
 int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -272,8 +273,9 @@ int fa_fwd_plan_ex(int B, int H, int N, int d, unsigned flags, int sm_count,
  * sums their fp32 dK, dV partials) and *grid_blocks blocks in all.  The split
  * is used only without FA_FLAG_CAUSAL, when it fills the waves of
  * one-block-per-SM launches clearly better (at least 8 query tiles a block).
- * Returns FA_OK, FA_ERR_NULL, FA_ERR_FLAGS, FA_ERR_SHAPE or FA_ERR_HEADDIM
- * (d other than 64, 96, 128).
+ * At d = 256 the grid has two blocks per key tile (one per half of d) and no
+ * split.  Returns FA_OK, FA_ERR_NULL, FA_ERR_FLAGS, FA_ERR_SHAPE or
+ * FA_ERR_HEADDIM (d other than 64, 96, 128, 256).
  */
 int fa_bwd_plan(int B, int H, int N, int d, unsigned flags, int sm_count, int *n_split,
                 int *grid_blocks);

@@ -92,7 +92,7 @@ def test_backward_validation(fa):
         p[i] = MIS
         assert _bwd(fa, p) == fa.FA_ERR_ALIGN
     assert _bwd(fa, ok, N=-3) == fa.FA_ERR_SHAPE
-    for d in (32, 80, 160, 256):
+    for d in (32, 80, 160, 512):
         assert _bwd(fa, ok, d=d) == fa.FA_ERR_HEADDIM
     assert _bwd(fa, ok, scale=-math.inf) == fa.FA_ERR_SCALE
 

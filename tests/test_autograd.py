@@ -22,7 +22,7 @@ def fa():
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 def test_autograd_matches_entry_points_and_oracle(fa, causal, d):
     B, N, H = 2, 300, 2
     q, k, v, dout = attn_inputs.draw(B, N, H, d, "bf16", 1700 + d, 4, device="cuda")

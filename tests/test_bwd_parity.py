@@ -87,6 +87,42 @@ def test_head_dim_96_fp16(fa, B, N, H):
     check_grads(fa, B, N, H, 96, "fp16", 1150 + N)
 
 
+@pytest.mark.parametrize("N", [1, 17, 64, 65, 127, 128, 129, 300, 640])
+def test_head_dim_256_bf16(fa, N):
+    # d = 256: two blocks per key tile, each producing one 128-wide half of
+    # dK, dV and dQ^T while S^T and dP^T contract all 256 columns
+    check_grads(fa, 2, N, 2, 256, "bf16", 1300 + N)
+
+
+@pytest.mark.parametrize("N", [1, 100, 257, 1500])
+def test_head_dim_256_fp16(fa, N):
+    check_grads(fa, 1, N, 2, 256, "fp16", 1350 + N, std=0.5)
+
+
+def test_detector_neck_backward_full_size(fa):
+    # the detector neck workload (one head, d = 256, N = 6400, fp16, x0.5)
+    # at full size: with dO zero outside a set R of query rows, every
+    # gradient is exactly R's contribution (dS vanishes elsewhere), which the
+    # row-restricted oracle returns for all keys
+    w = attn_inputs.WORKLOADS["c3"]
+    q, k, v, dout = attn_inputs.draw_workload(w, count=4, device="cuda")
+    blocks = [(0, 64), (3200, 3264), (w.N - 40, w.N)]
+    keep = torch.zeros(w.N, dtype=torch.bool, device="cuda")
+    for a, b in blocks:
+        keep[a:b] = True
+    dout_r = torch.where(keep.view(1, w.N, 1, 1), dout, torch.zeros_like(dout))
+    dq, dk, dv = run_bwd(fa, q, k, v, dout_r, w.scale)
+    q64, k64, v64, d64 = (to64(t) for t in (q, k, v, dout_r))
+    ref = None
+    for a, b in blocks:
+        part = oracle.attn_bwd_rows(q64, k64, v64, d64, w.scale, a, b)
+        ref = part if ref is None else tuple(x + y for x, y in zip(ref, part))
+    for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        s = err_stats(to64(got), r)
+        assert s["max"] <= GRAD_MAX, (name, s)
+    assert bool((dq[:, ~keep] == 0).all())
+
+
 def test_head_dim_128_many_tiles(fa):
     # 16 key tiles per head, 32 query tiles each: both dQ^T buffers and every
     # Q/dO stage are reused many times over
@@ -142,7 +178,7 @@ def test_split_query_ranges(fa, d, dtype):
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
 
 
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 def test_deterministic_dk_dv(fa, d):
     # dK and dV are owned by one block each (no atomics): bitwise repeatable.
     q, k, v, dout = attn_inputs.draw(1, 700, 2, d, "bf16", 702, 4, device="cuda")

@@ -112,7 +112,7 @@ def check_bwd(fa, B, N, H, d, dtype, seed):
         assert s["max"] <= GRAD_MAX, (name, s)
 
 
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("N", [1, 17, 64, 127, 128, 129, 300, 640])
 def test_causal_backward_ragged(fa, d, N):
     check_bwd(fa, 2, N, 2, d, "bf16", 1400 + N + d)

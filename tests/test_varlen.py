@@ -58,7 +58,7 @@ def test_varlen_forward_per_sequence(fa, d, dtype, causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 def test_varlen_backward_per_sequence(fa, d, causal):
     H = 2
     (q, k, v, do), cu, total = packed(LENGTHS, H, d, "bf16", 2000 + d)
