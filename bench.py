@@ -44,16 +44,16 @@ L2_FLUSH_BYTES = 512 << 20
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the kernel sources hash to the recorded value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.759232e6 + 21.073152e6,
-                                                    "src": "532207f4dfa00c07"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.580736e6 + 2.517248e6,
-                                                       "src": "532207f4dfa00c07"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 51.360256e6 + 5.298176e6,
-                                                    "src": "532207f4dfa00c07"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.644544e6 + 113.935872e6,
-                                                     "src": "532207f4dfa00c07"},
-    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.289472e6 + 0.524288e6,
-                                                        "src": "532207f4dfa00c07"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.869824e6 + 24.427264e6,
+                                                    "src": "5d54eeea6af00ca3"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.543360e6 + 1.550848e6,
+                                                       "src": "5d54eeea6af00ca3"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.879744e6 + 4.389376e6,
+                                                    "src": "5d54eeea6af00ca3"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 103.361280e6 + 115.263744e6,
+                                                     "src": "5d54eeea6af00ca3"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.279488e6 + 0.397568e6,
+                                                        "src": "5d54eeea6af00ca3"},
 }
 
 

@@ -637,12 +637,12 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  static_assert(!(SPLIT && Tr::NHALF > 1), "query splits and d halves are not combined");
+  // block x = (key tile * n_split + split) * NHALF + d half
   constexpr int DW = Tr::DW, NHALF = Tr::NHALF;
-  const int sp = SPLIT ? (int)blockIdx.x % p.n_split : 0;  // split of the query range
   const int dh = NHALF > 1 ? (int)blockIdx.x % NHALF : 0;  // d half this block produces
-  const int kt = SPLIT ? (int)blockIdx.x / p.n_split
-                       : (NHALF > 1 ? (int)blockIdx.x / NHALF : (int)blockIdx.x);
+  const int xs = NHALF > 1 ? (int)blockIdx.x / NHALF : (int)blockIdx.x;
+  const int sp = SPLIT ? xs % p.n_split : 0;  // split of the query range
+  const int kt = SPLIT ? xs / p.n_split : xs;
   const int h = blockIdx.y, b = blockIdx.z;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
@@ -1249,8 +1249,8 @@ static int run_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const CUte
 // block per key tile).
 template <class Tr>
 static int bwd_split(int B, int H, int N, unsigned flags, const int* cu, int sm_count) {
-  if ((flags & 1u) || cu != nullptr || Tr::NHALF > 1) return 1;
-  const long long blocks = (long long)((N + Tr::BN - 1) / Tr::BN) * H * B;
+  if ((flags & 1u) || cu != nullptr) return 1;
+  const long long blocks = (long long)((N + Tr::BN - 1) / Tr::BN) * Tr::NHALF * H * B;
   return choose_bwd_split(blocks, (N + Tr::BM - 1) / Tr::BM, sm_count);
 }
 
@@ -1271,8 +1271,8 @@ int plan_bwd(int B, int H, int N, int d, unsigned flags, int sm_count, int* n_sp
       ns = bwd_split<BwdTq128>(B, H, N, flags, nullptr, sm_count);
       bn = BwdTq128::BN;
       break;
-    case 256:  // two blocks per key tile, one per half of d; never split
-      ns = 1;
+    case 256:  // two blocks per key tile and split, one per half of d
+      ns = bwd_split<BwdTq256>(B, H, N, flags, nullptr, sm_count);
       bn = BwdTq256::BN;
       break;
     default:
@@ -1323,12 +1323,14 @@ int bwd_launch(const void* q, const void* k, const void* v, const void* o, const
                                   tok_g, stream, cu, total, ns);
     }
     case 256: {
+      const int ns = bwd_split<BwdTq256>(B, H, N, flags, cu, dev.sm_count);
       auto kern = (flags & 1u) ? (cu ? fa_bwd_tq_kernel<T, BwdTq256, true, true>
                                      : fa_bwd_tq_kernel<T, BwdTq256, true, false>)
                                : (cu ? fa_bwd_tq_kernel<T, BwdTq256, false, true>
-                                     : fa_bwd_tq_kernel<T, BwdTq256, false, false>);
+                                     : ns > 1 ? fa_bwd_tq_kernel<T, BwdTq256, false, false, true>
+                                              : fa_bwd_tq_kernel<T, BwdTq256, false, false>);
       return run_bwd<T, BwdTq256>(kern, q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, tok_in,
-                                  tok_g, stream, cu, total);
+                                  tok_g, stream, cu, total, ns);
     }
     default:
       return FA_ERR_HEADDIM;

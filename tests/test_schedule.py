@@ -191,8 +191,10 @@ def test_backward_split_plans():
         n_q = -(-N // (128 if d == 64 else 64))
         assert p["n_split"] == 1 or n_q // p["n_split"] >= 8
         assert p["grid"] == -(-N // 128) * H * B * p["n_split"]
-    # d = 256: two blocks per key tile (one per half of d), never split
-    assert plan(1, 1, 6400, 256, 148) == {"n_split": 1, "grid": 100}
+    # d = 256: two blocks per key tile (one per half of d), and the split
+    # on top: 100 blocks -> 4 shares of each key tile's query range
+    assert plan(1, 1, 6400, 256, 148) == {"n_split": 4, "grid": 400}
+    assert plan(1, 1, 6400, 256, 148, CAUSAL) == {"n_split": 1, "grid": 100}
     with pytest.raises(fa.FAError):
         plan(1, 1, 64, 512, 148)
     with pytest.raises(fa.FAError):
