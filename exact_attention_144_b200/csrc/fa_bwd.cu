@@ -94,6 +94,7 @@ struct BwdParams {
   // partial dK (scaled), dV to dk_part / dv_part + split * part_stride, laid
   // out [B*N tokens, H, D], and fa_bwd_dkv_kernel sums them
   int n_split;
+  int n_x;  // blocks per (batch, head); the grid is 1-D: block = (b * H + h) * n_x + x
   float* dk_part;
   float* dv_part;
   long long part_stride;
@@ -201,9 +202,11 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  const int sp = SPLIT ? (int)blockIdx.x % p.n_split : 0;  // split of the query range
-  const int kt = SPLIT ? (int)blockIdx.x / p.n_split : (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // a 1-D grid (B * H may exceed the 65,535 limit of gridDim.y and .z)
+  const int bx = (int)(blockIdx.x % (unsigned)p.n_x), bh = (int)(blockIdx.x / (unsigned)p.n_x);
+  const int sp = SPLIT ? bx % p.n_split : 0;  // split of the query range
+  const int kt = SPLIT ? bx / p.n_split : bx;
+  const int h = bh % p.H, b = bh / p.H;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
   int tb, tok0, len;
@@ -637,13 +640,15 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  // block x = (key tile * n_split + split) * NHALF + d half
+  // a 1-D grid (B * H may exceed the 65,535 limit of gridDim.y and .z); within
+  // a (batch, head): x = (key tile * n_split + split) * NHALF + d half
   constexpr int DW = Tr::DW, NHALF = Tr::NHALF;
-  const int dh = NHALF > 1 ? (int)blockIdx.x % NHALF : 0;  // d half this block produces
-  const int xs = NHALF > 1 ? (int)blockIdx.x / NHALF : (int)blockIdx.x;
+  const int bx = (int)(blockIdx.x % (unsigned)p.n_x), bh = (int)(blockIdx.x / (unsigned)p.n_x);
+  const int dh = NHALF > 1 ? bx % NHALF : 0;  // d half this block produces
+  const int xs = NHALF > 1 ? bx / NHALF : bx;
   const int sp = SPLIT ? xs % p.n_split : 0;  // split of the query range
   const int kt = SPLIT ? xs / p.n_split : xs;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int h = bh % p.H, b = bh / p.H;
   // the block's sequence on the token axis (batch entry tb, tokens tok0 ..
   // tok0 + len); a key tile past a shorter sequence's end has no work
   int tb, tok0, len;
@@ -1200,9 +1205,10 @@ static int launch_bwd(void (*kern)(const CUtensorMap, const CUtensorMap, const C
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (timed) take_kernel_events(true, &ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  kern<<<dim3((N + Tr::BN - 1) / Tr::BN * n_split * Tr::NHALF, H, B), 384, Tr::SMEM_BYTES,
-         stream>>>(
-      tmq, tmk, tmv, tmdo, tmacc, p);
+  p.n_x = (N + Tr::BN - 1) / Tr::BN * n_split * Tr::NHALF;
+  const long long blocks = (long long)p.n_x * H * B;
+  if (blocks >= (1ll << 31)) return FA_ERR_SHAPE;
+  kern<<<(unsigned)blocks, 384, Tr::SMEM_BYTES, stream>>>(tmq, tmk, tmv, tmdo, tmacc, p);
   rc = launch_status(cudaGetLastError());
   if (ev1) cudaEventRecord(ev1, stream);
   note_launches(1);

@@ -123,6 +123,24 @@ def test_detector_neck_backward_full_size(fa):
     assert bool((dq[:, ~keep] == 0).all())
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_batch_beyond_grid_dimension_limit(fa, d):
+    # 66,000 short sequences: more (batch, head) pairs than a grid's y or z
+    # dimension holds (65,535); the backward grid is 1-D, so every pair runs
+    B, N, H = 66000, 20, 1
+    q, k, v, dout = attn_inputs.draw(B, N, H, d, "bf16", 1400 + d, 4, device="cuda")
+    scale = float(np.float32(1.0 / math.sqrt(d)))
+    dq, dk, dv = run_bwd(fa, q, k, v, dout, scale)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+    for b in (0, 1, 65534, 65535, 65536, B - 1):
+        sl = slice(b, b + 1)
+        ref = oracle.attn_bwd(to64(q[sl]), to64(k[sl]), to64(v[sl]), to64(dout[sl]), scale)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            s = err_stats(to64(got[sl]), r)
+            assert s["max"] <= GRAD_MAX, (b, name, s)
+
+
 def test_head_dim_128_many_tiles(fa):
     # 16 key tiles per head, 32 query tiles each: both dQ^T buffers and every
     # Q/dO stage are reused many times over
