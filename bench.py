@@ -44,16 +44,16 @@ L2_FLUSH_BYTES = 512 << 20
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the kernel sources hash to the recorded value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.869824e6 + 24.427264e6,
-                                                    "src": "5d54eeea6af00ca3"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.543360e6 + 1.550848e6,
-                                                       "src": "5d54eeea6af00ca3"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.879744e6 + 4.389376e6,
-                                                    "src": "5d54eeea6af00ca3"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 103.361280e6 + 115.263744e6,
-                                                     "src": "5d54eeea6af00ca3"},
-    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.279488e6 + 0.397568e6,
-                                                        "src": "5d54eeea6af00ca3"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.846016e6 + 23.928064e6,
+                                                    "src": "5457882a8dd61b12"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.527744e6 + 1.632768e6,
+                                                       "src": "5457882a8dd61b12"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.677248e6 + 3.626496e6,
+                                                    "src": "5457882a8dd61b12"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 103.180032e6 + 115.197440e6,
+                                                     "src": "5457882a8dd61b12"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.278208e6 + 0.411392e6,
+                                                        "src": "5457882a8dd61b12"},
 }
 
 
