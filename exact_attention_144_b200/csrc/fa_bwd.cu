@@ -202,8 +202,12 @@ __global__ void __launch_bounds__(384, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
-  // a 1-D grid (B * H may exceed the 65,535 limit of gridDim.y and .z)
-  const int bx = (int)(blockIdx.x % (unsigned)p.n_x), bh = (int)(blockIdx.x / (unsigned)p.n_x);
+  // a 1-D grid (B * H may exceed the 65,535 limit of gridDim.y and .z); causal
+  // key tiles see fewer query tiles the later they are, so there the order is
+  // key-tile major: every head's long key tiles start first
+  const unsigned n_bh = (unsigned)(p.B * p.H);
+  const int bx = CAUSAL ? (int)(blockIdx.x / n_bh) : (int)(blockIdx.x % (unsigned)p.n_x);
+  const int bh = CAUSAL ? (int)(blockIdx.x % n_bh) : (int)(blockIdx.x / (unsigned)p.n_x);
   const int sp = SPLIT ? bx % p.n_split : 0;  // split of the query range
   const int kt = SPLIT ? bx / p.n_split : bx;
   const int h = bh % p.H, b = bh / p.H;
@@ -641,9 +645,13 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl w{abort_flag, p.limit_ns, p.status};
   // a 1-D grid (B * H may exceed the 65,535 limit of gridDim.y and .z); within
-  // a (batch, head): x = (key tile * n_split + split) * NHALF + d half
+  // a (batch, head): x = (key tile * n_split + split) * NHALF + d half.  Causal
+  // key tiles see fewer query tiles the later they are, so there the order is
+  // x-major: every head's long key tiles start first
   constexpr int DW = Tr::DW, NHALF = Tr::NHALF;
-  const int bx = (int)(blockIdx.x % (unsigned)p.n_x), bh = (int)(blockIdx.x / (unsigned)p.n_x);
+  const unsigned n_bh = (unsigned)(p.B * p.H);
+  const int bx = CAUSAL ? (int)(blockIdx.x / n_bh) : (int)(blockIdx.x % (unsigned)p.n_x);
+  const int bh = CAUSAL ? (int)(blockIdx.x % n_bh) : (int)(blockIdx.x / (unsigned)p.n_x);
   const int dh = NHALF > 1 ? bx % NHALF : 0;  // d half this block produces
   const int xs = NHALF > 1 ? bx / NHALF : bx;
   const int sp = SPLIT ? xs % p.n_split : 0;  // split of the query range
