@@ -44,16 +44,16 @@ L2_FLUSH_BYTES = 512 << 20
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the kernel sources hash to the recorded value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.846016e6 + 23.928064e6,
-                                                    "src": "5457882a8dd61b12"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.527744e6 + 1.632768e6,
-                                                       "src": "5457882a8dd61b12"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.677248e6 + 3.626496e6,
-                                                    "src": "5457882a8dd61b12"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 103.180032e6 + 115.197440e6,
-                                                     "src": "5457882a8dd61b12"},
-    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.278208e6 + 0.411392e6,
-                                                        "src": "5457882a8dd61b12"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.760768e6 + 22.263552e6,
+                                                    "src": "69fb3b0fb9fd51ca"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.544896e6 + 2.624768e6,
+                                                       "src": "69fb3b0fb9fd51ca"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.674176e6 + 3.452160e6,
+                                                    "src": "69fb3b0fb9fd51ca"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.681152e6 + 114.389504e6,
+                                                     "src": "69fb3b0fb9fd51ca"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.275904e6 + 0.216832e6,
+                                                        "src": "69fb3b0fb9fd51ca"},
 }
 
 
