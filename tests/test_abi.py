@@ -190,3 +190,30 @@ def test_varlen_bounds_clamp_every_input_into_range():
         for b in range(4):
             t0, n = fa.fa_varlen_bounds(cu, b, ms, total)
             assert 0 <= t0 <= total and 0 <= n <= ms and t0 + n <= total
+
+
+def test_size_limit_is_exact():
+    # every tensor must hold fewer than 2^31 elements: at 2^31 the call is
+    # refused before any CUDA call; one token fewer passes validation (and
+    # then, without a GPU, fails in the CUDA runtime instead)
+    import ctypes
+    import exact_attention_144_b200 as fa
+    lib = fa.lib()
+    buf = (ctypes.c_char * 4096)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    s = ctypes.c_float(0.1)
+    n_max = 1 << 25  # with H = 1, d = 64: 2^31 elements
+    assert lib.fa_fwd(p, p, p, p, p, 1, 1, n_max, 64, s, None) == fa.FA_ERR_SHAPE
+    assert lib.fa_fwd(p, p, p, p, p, 1, 1, n_max - 1, 64, s, None) not in (
+        fa.FA_ERR_SHAPE, fa.FA_OK)
+    assert lib.fa_bwd(*([p] * 9), 1, 1, n_max, 64, s, None) == fa.FA_ERR_SHAPE
+    assert lib.fa_bwd(*([p] * 9), 1, 1, n_max - 1, 64, s, None) not in (fa.FA_ERR_SHAPE, fa.FA_OK)
+    # packed: the [B, N, 3, H, d] tensor counts three times the tokens' elements
+    n3 = (1 << 31) // (3 * 64) + 1
+    assert lib.fa_fwd_qkvpacked(p, p, p, 1, 1, n3, 64, s, 0, 0, None) == fa.FA_ERR_SHAPE
+    assert lib.fa_fwd_qkvpacked(p, p, p, 1, 1, n3 - 1, 64, s, 0, 0, None) not in (
+        fa.FA_ERR_SHAPE, fa.FA_OK)
+    # 8-bit: the same element limit
+    one = ctypes.c_float(1.0)
+    assert lib.fa_fwd_fp8(p, p, p, p, p, 1, 1, 1 << 24, 128, s, one, one, one, 0,
+                          None) == fa.FA_ERR_SHAPE
