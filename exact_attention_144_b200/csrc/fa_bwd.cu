@@ -9,12 +9,18 @@
 //   dK  += scale dS^T Q
 //   dQ  += scale dS K   (fp32, reduced into global memory across K/V tiles)
 //
-// Three kernels:
+// Five kernels:
 //   fa_bwd_pre_kernel   D, minus the base-2 LSE (padded to whole Q tiles) and
 //                       a zeroed fp32 dQ accumulator
-//   fa_bwd_kernel       one block per (K/V tile of 128 keys, head, batch); its
-//                       loop walks the Q tiles of 128 queries
+//   fa_bwd_kernel       d = 64: one block per (K/V tile of 128 keys, head,
+//                       batch); its loop walks the Q tiles of 128 queries
+//   fa_bwd_tq_kernel    d = 96, 128, 256: 64-query inner tiles with dQ produced
+//                       transposed (described where it is defined)
+//   fa_bwd_dkv_kernel   sums the fp32 dK, dV partials of split query ranges
 //   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to 16 bits
+// The main kernels' grids are 1-D (block = (b * H + h) * blocks per head +
+// x, or key-tile major for the causal mask) and may split a key tile's query
+// range over several blocks when few key tiles would leave SMs idle.
 //
 // fa_bwd_kernel layout (384 threads, one block per SM):
 //   warps 0-7  compute: warp w owns TMEM lane quadrant w % 4 and half w / 4 of

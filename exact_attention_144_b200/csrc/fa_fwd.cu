@@ -32,10 +32,12 @@
 // (no memory is read for them); Q K^T contracts only the 96 real columns (six
 // k-steps of 16) and P.V and the O accumulator are 96 columns wide.
 //
-// In both, P (16-bit) is written back over the first BN/2 columns of its S
-// buffer and consumed from there by the P.V MMA (A operand in TMEM).  O is
-// rescaled only when a row's max grows by more than 2^8: until then P and l
-// stay relative to the older max (P <= 2^8), which changes rounding only.
+// In both, P is consumed by the P.V MMA from tensor memory (A operand): written
+// back over the first columns of its S buffer (16-bit P: BN/2 columns; E4M3 P
+// from the 8-bit path: BN/4), or, in the d = 64 pair kernel, into its own
+// columns.  O is rescaled only when a row's max grows by more than 2^8: until
+// then P and l stay relative to the older max (P <= 2^8), which changes
+// rounding only.
 //
 // When the units cannot fill the SMs, the K/V range is split and the partial
 // results (fp32, normalised, base-2 LSE) are merged by fa_combine_kernel:
