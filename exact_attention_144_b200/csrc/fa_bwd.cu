@@ -551,7 +551,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ===========================================================================
-// fa_bwd_tq_kernel: d = 96 and 128.  At 128 queries per inner tile the five
+// fa_bwd_tq_kernel: d = 96, 128 and 256.  At 128 queries per inner tile the five
 // accumulators (S^T, dP^T, dQ, dV, dK: 5 x 128 columns) exceed tensor memory,
 // so the inner tile holds 64 queries and dQ is produced transposed,
 //   dQ_i^T = K^T dS_i^T   (M = d = 128 lanes, N = 64 queries, K = 128 keys),
@@ -571,6 +571,11 @@ __global__ void __launch_bounds__(384, 1)
 // contract the 96 real columns, dV and dK are 96 columns wide (dK at
 // [352,448)), and dQ^T is still a 128-lane tile whose lanes 96-127 (K^T rows
 // of zeros) are never drained.
+// At d = 256 two blocks share each key tile, block half dh producing columns
+// [128 dh, 128 dh + 128) of dK, dV and rows of dQ^T (the same tensor memory
+// layout as d = 128); S^T and dP^T contract all 256 columns in both.  The
+// resident 64 KB K and V tiles leave room for one Q/dO stage and four dQ
+// staging boxes, which warps 0-3 use for both query halves of their quadrant.
 // ===========================================================================
 template <int D_, int QST_>
 struct BwdTqTraits {
