@@ -206,10 +206,11 @@ int make_tmap_f32_rows(CUtensorMap* map, const void* base, size_t rows, int cols
 // ------------------------------------------------------------ validation
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static int check_common(int B, int H, int N, int d, float scale, bool bwd) {
+// Shape, head-size and scale checks shared by every entry point (the 8-bit
+// forward then narrows d to 128).
+static int check_common(int B, int H, int N, int d, float scale) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   if (!(d == 64 || d == 96 || d == 128 || d == 256)) return FA_ERR_HEADDIM;
-  (void)bwd;
   if ((long long)B * N * H * d >= (1ll << 31)) return FA_ERR_SHAPE;
   if (!isfinite(scale)) return FA_ERR_SCALE;
   return FA_OK;
@@ -227,7 +228,7 @@ template <class T>
 static int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int N, int d, float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, lse});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc == FA_OK)
     rc = fwd_launch<T>(q, k, v, o, lse, B, H, N, d, scale, flags, (long long)H * d, stream);
@@ -239,7 +240,7 @@ static int bwd_entry(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                      float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc == FA_OK)
     rc = bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, flags,
@@ -253,7 +254,7 @@ template <class T>
 static int fwd_packed_entry(const void* qkv, void* o, float* lse, int B, int H, int N, int d,
                             float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({qkv, o, lse});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   if (rc == FA_OK && (long long)B * N * 3 * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc != FA_OK) return rc;
@@ -268,7 +269,7 @@ static int bwd_packed_entry(const void* qkv, const void* o, const void* dout, co
                             void* dqkv, int B, int H, int N, int d, float scale, unsigned flags,
                             cudaStream_t stream) {
   int rc = check_ptrs({qkv, o, dout, lse, dqkv});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   if (rc == FA_OK && (long long)B * N * 3 * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc != FA_OK) return rc;
@@ -285,7 +286,7 @@ static int fwd_fp8_entry(const void* q, const void* k, const void* v, void* o, f
                          int H, int N, int d, float scale, float descale_q, float descale_k,
                          float descale_v, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, lse});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, false);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   if (rc == FA_OK && d != 128) rc = FA_ERR_HEADDIM;
   const float s_eff = scale * descale_q * descale_k;
   if (rc == FA_OK && !(isfinite(descale_q) && isfinite(descale_k) && isfinite(descale_v) &&
@@ -302,11 +303,11 @@ static int fwd_fp8_entry(const void* q, const void* k, const void* v, void* o, f
 // tokens ([total, H, d] tensors, lse [H, total]); cu_seqlens (device, B + 1
 // entries) holds each sequence's first token, max_seqlen bounds their lengths.
 static int check_varlen(const int* cu, int B, int total, int max_seqlen, int H, int d,
-                        float scale, bool bwd) {
+                        float scale) {
   if (cu == nullptr) return FA_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return FA_ERR_ALIGN;
   if (total < 1 || max_seqlen < 1) return FA_ERR_SHAPE;
-  int rc = check_common(B, H, max_seqlen, d, scale, bwd);
+  int rc = check_common(B, H, max_seqlen, d, scale);
   if (rc == FA_OK && (long long)total * H * d >= (1ll << 31)) rc = FA_ERR_SHAPE;
   return rc;
 }
@@ -316,7 +317,7 @@ static int fwd_varlen_entry(const void* q, const void* k, const void* v, void* o
                             const int* cu, int B, int total, int max_seqlen, int H, int d,
                             float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, lse});
-  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale, false);
+  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc != FA_OK) return rc;
   return fwd_launch<T>(q, k, v, o, lse, B, H, max_seqlen, d, scale, flags, (long long)H * d,
@@ -329,7 +330,7 @@ static int bwd_varlen_entry(const void* q, const void* k, const void* v, const v
                             const int* cu, int B, int total, int max_seqlen, int H, int d,
                             float scale, unsigned flags, cudaStream_t stream) {
   int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
-  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale, true);
+  if (rc == FA_OK) rc = check_varlen(cu, B, total, max_seqlen, H, d, scale);
   if (rc == FA_OK && (flags & ~kKnownFlags) != 0) rc = FA_ERR_FLAGS;
   if (rc != FA_OK) return rc;
   return bwd_launch<T>(q, k, v, o, dout, lse, dq, dk, dv, B, H, max_seqlen, d, scale, flags,
@@ -340,7 +341,7 @@ int check_bwd_args(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale) {
   int rc = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
-  if (rc == FA_OK) rc = check_common(B, H, N, d, scale, true);
+  if (rc == FA_OK) rc = check_common(B, H, N, d, scale);
   return rc;
 }
 
