@@ -39,6 +39,14 @@ METRIC = "fused attention fwd/bwd TFLOP/s on 1 B200 and % of bf16 tensor-core pe
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
+L2_NOTE = "512 MiB written between timed GPU steps"
+# The pages' five configurations and the N sweep, each timed on its own in the
+# same run (forward; forward + backward for the training workload).
+PER_CONFIG = ("c1", "c2", "c3", "c4", "sweep1024", "sweep2048", "sweep4096", "sweep8192", "c5")
+PER_CONFIG_RUNS = 20
+# The oracle runs a whole configuration when it costs at most this much work,
+# otherwise the first rows of every head, sized to about this much.
+ORACLE_BUDGET_GFLOP = 40.0
 
 # DRAM traffic of the dominant kernel per launch, from an ncu capture of the
 # same workload (dram__bytes_read.sum + dram__bytes_write.sum), valid only
@@ -56,6 +64,47 @@ TRAFFIC = {
     ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.275904e6 + 0.216832e6,
                                                         "src": "212dbf11be8bd47c"},
 }
+
+
+def workload_config(w: attn_inputs.Workload, world: int = 1) -> dict:
+    """The `config` object of the JSON line: the workload, identical for both arms."""
+    return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N, "heads": w.H,
+            "head_dim": w.d, "causal": False,
+            "parallelism": f"replicas x{world} (batch per rank, no collective)",
+            "l2": L2_NOTE,
+            "inputs": "seeded N(0,1) draws rounded to the "
+                      + ("E4M3 type (descale factors 1), bf16 O" if w.dtype == "fp8"
+                         else "16-bit type")}
+
+
+def io_bytes(w: attn_inputs.Workload, backward: bool) -> float:
+    """Algorithmic HBM bytes of one call: forward reads Q, K, V and writes O
+    and the LSE; backward reads Q, K, V, O, dO and the LSE and writes dQ, dK,
+    dV."""
+    eb = 1 if w.dtype == "fp8" else 2
+    elems = float(w.B) * w.N * w.H * w.d
+    lse = 4.0 * w.B * w.H * w.N
+    if backward:
+        return 8 * elems * eb + lse
+    return 3 * elems * eb + elems * (2 if w.dtype == "fp8" else eb) + lse
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def peaks():
@@ -240,7 +289,36 @@ def e2e_pipelined(fa, w, args, dev, q, k, v, do, train, mk):
             ev_out[i].record(s_out)
     t1.record(s_out)
     torch.cuda.synchronize()
-    return t0.elapsed_time(t1) / args.steps, h2d, d2h
+    ms = t0.elapsed_time(t1) / args.steps
+
+    # The same copies without kernels: uploads alone, downloads alone, and
+    # both at once on two streams (the PCIe floor of the pipelined steps).
+    ins, outs, hout = sets[0]
+
+    def timed(up: bool, down: bool) -> float:
+        a, b = mk(), mk()
+        torch.cuda.synchronize()
+        a.record(s_in)
+        s_out.wait_stream(s_in)
+        for _ in range(args.steps):
+            if up:
+                with torch.cuda.stream(s_in):
+                    for hsrc, dst in zip(host_in, ins):
+                        dst.copy_(hsrc, non_blocking=True)
+            if down:
+                with torch.cuda.stream(s_out):
+                    for dsrc, hdst in zip(outs, hout):
+                        hdst.copy_(dsrc, non_blocking=True)
+        s_in.wait_stream(s_out)
+        b.record(s_in)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    copies = {"h2d_ms": timed(True, False), "d2h_ms": timed(False, True),
+              "both_ms": timed(True, True)}
+    copies["h2d_gbs"] = h2d / (copies["h2d_ms"] * 1e-3) / 1e9
+    copies["d2h_gbs"] = d2h / (copies["d2h_ms"] * 1e-3) / 1e9
+    return ms, h2d, d2h, copies
 
 
 def main_kernel_names(fa, w: attn_inputs.Workload, props) -> tuple:
@@ -250,6 +328,152 @@ def main_kernel_names(fa, w: attn_inputs.Workload, props) -> tuple:
     fwd = "fa_fwd_pp_kernel" if plan["kernel"] == 1 else "fa_fwd_kernel"
     bwd = "fa_bwd_kernel" if w.d == 64 else "fa_bwd_tq_kernel"
     return fwd, bwd
+
+
+def _stats(xs):
+    return statistics.mean(xs), statistics.median(xs)
+
+
+def time_config(fa, w: attn_inputs.Workload, dev, flush, runs: int, local: int, pk: dict):
+    """Times one configuration on its own: `runs` forward calls (and backward
+    calls for the training workload), each after a 512 MiB write that evicts
+    L2.  CUDA events bracket the whole call and, through
+    fa_set_kernel_events, the main kernel alone.  Returns the configuration's
+    entry of the JSON line's per_config object (plus the forward output and
+    LSE, for the C1 report on the unrounded draws)."""
+    q, k, v, do = attn_inputs.draw(w.B, w.N, w.H, w.d, w.dtype, w.seed, 4, std=w.std,
+                                   device=dev)
+    fwd, bwd, out_dtype = entry_points(fa, w)
+    train = w.backward and bwd is not None
+    o = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+
+    def call_fwd():
+        fwd(q, k, v, o=o, lse=lse, scale=w.scale)
+
+    def call_bwd():
+        bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, scale=w.scale)
+
+    for _ in range(3):
+        call_fwd()
+        if train:
+            call_bwd()
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [[mk() for _ in range(8)] for _ in range(runs)]
+    with ClockSampler(local) as clk:
+        for e in ev:
+            flush.zero_()
+            fa.fa_set_kernel_events(e[2], e[3], e[6] if train else None, e[7] if train else None)
+            e[0].record()
+            call_fwd()
+            e[1].record()
+            if train:
+                e[4].record()
+                call_bwd()
+                e[5].record()
+        torch.cuda.synchronize()
+    clocks = clk.summary()
+    mhz = clocks["sm_mhz"]
+    props = torch.cuda.get_device_properties(dev)
+    plan = fa.fa_fwd_plan(w.B, w.H, w.N, w.d, props.multi_processor_count)
+    fwd_name, bwd_name = main_kernel_names(fa, w, props)
+    peak, peak_sus, _ = tensor_peak(pk, w)
+
+    def part(kern_ms, call_ms, flop, nbytes, name):
+        k_mean, k_med = _stats(kern_ms)
+        c_mean, c_med = _stats(call_ms)
+        tf = flop / (k_mean * 1e-3) / 1e12
+        gbs = nbytes / (k_mean * 1e-3) / 1e9
+        return {"kernel": name, "kernel_us": 1e3 * k_mean, "kernel_us_median": 1e3 * k_med,
+                "call_us": 1e3 * c_mean, "call_us_median": 1e3 * c_med,
+                "kernel_cycles": (1e3 * k_mean * mhz) if mhz else None,
+                "tflops": tf, "pct_peak": 100.0 * tf / peak,
+                "pct_peak_sustained": 100.0 * tf / peak_sus,
+                "call_tflops": flop / (c_mean * 1e-3) / 1e12,
+                "gbs": gbs, "pct_hbm": 100.0 * gbs / pk["hbm_gbs"],
+                "algorithmic_bytes": nbytes}
+
+    extra = " + fa_combine_kernel" if plan["n_split"] > 1 else ""
+    entry = {"workload": w.name, "shape_bnhd": [w.B, w.N, w.H, w.d], "dtype": w.dtype,
+             "seed": w.seed, "runs": runs, "plan": plan,
+             "fwd": part([e[2].elapsed_time(e[3]) for e in ev],
+                         [e[0].elapsed_time(e[1]) for e in ev], w.fwd_flop, io_bytes(w, False),
+                         fwd_name + extra),
+             "clocks": clocks}
+    if train:
+        entry["bwd"] = part([e[6].elapsed_time(e[7]) for e in ev],
+                            [e[4].elapsed_time(e[5]) for e in ev], w.bwd_flop, io_bytes(w, True),
+                            bwd_name)
+    return entry, o, lse
+
+
+def oracle_time_config(w: attn_inputs.Workload, budget_gflop: float, single_core: bool) -> dict:
+    """Times the fp64 oracle, as it stands, on one configuration's inputs on
+    the host cores: the whole configuration when its work is within
+    budget_gflop, else the first rows of every head sized to about that much
+    (the FLOP rate is then that of the sample).  With single_core, also on
+    one thread."""
+    import oracle  # the CPU-baseline leg is one of the oracle's permitted users
+    q, k, v, do = attn_inputs.draw_workload(w, count=4)
+    f64 = attn_inputs.to_f64
+    Q, K, V, DO = f64(q), f64(k), f64(v), f64(do)
+    flop = w.fwd_flop + (w.bwd_flop if w.backward else 0.0)
+    whole = flop <= budget_gflop * 1e9
+
+    def run():
+        t0 = time.perf_counter()
+        if whole:
+            oracle.attn_fwd(Q, K, V, w.scale)
+            if w.backward:
+                oracle.attn_bwd(Q, K, V, DO, w.scale)
+            done = flop
+        else:
+            rows = max(1, min(w.N, int(w.N * budget_gflop * 1e9 / flop)))
+            sel = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(rows)]
+            oracle.attn_fwd_rows(Q, K, V, w.scale, sel)
+            if w.backward:
+                oracle.attn_bwd_rows(Q, K, V, DO, w.scale, 0, rows)
+            done = (14.0 if w.backward else 4.0) * rows * w.N * w.d * w.B * w.H
+        return time.perf_counter() - t0, done
+
+    threads = oracle.num_threads()
+    dt, done = run()
+    rows = w.N if whole else max(1, min(w.N, int(w.N * budget_gflop * 1e9 / flop)))
+    out = {"tflops": done / dt / 1e12, "seconds": dt, "gflop": done / 1e9, "threads": threads,
+           "sample": ("whole configuration" if whole else
+                      f"query rows [0,{rows}) of all {w.B * w.H} heads"
+                      + (" (forward rows and their backward)" if w.backward else "")),
+           "extrapolated_seconds": dt * flop / done}
+    if single_core:
+        oracle.set_num_threads(1)
+        try:
+            dt1, done1 = run()
+        finally:
+            oracle.set_num_threads(threads)
+        out["single_core"] = {"tflops": done1 / dt1 / 1e12, "seconds": dt1}
+    return out
+
+
+def c1_fp32_report(w: attn_inputs.Workload, o_gpu, lse_gpu) -> dict:
+    """C1 draws fp32 inputs, which the GPU receives rounded to bf16.  Reports
+    the oracle on the unrounded fp32 draws beside the oracle on the rounded
+    inputs (the parity reference) and the GPU result: informational, not a
+    gate."""
+    import oracle
+    raw = attn_inputs.draw_fp32(w.B, w.N, w.H, w.d, w.seed, count=3, std=w.std)
+    q, k, v = attn_inputs.draw_workload(w, count=3)
+    f64 = attn_inputs.to_f64
+    o_raw, lse_raw = oracle.attn_fwd(*(x.astype(np.float64) for x in raw), w.scale)
+    o_rnd, lse_rnd = oracle.attn_fwd(f64(q), f64(k), f64(v), w.scale)
+    o_g = f64(o_gpu)
+    l_g = lse_gpu.detach().cpu().double().numpy()
+    return {"o_max_abs_rounded_vs_fp32_oracle": float(np.abs(o_rnd - o_raw).max()),
+            "lse_max_abs_rounded_vs_fp32_oracle": float(np.abs(lse_rnd - lse_raw).max()),
+            "o_max_abs_gpu_vs_rounded_oracle": float(np.abs(o_g - o_rnd).max()),
+            "o_max_abs_gpu_vs_fp32_oracle": float(np.abs(o_g - o_raw).max()),
+            "lse_max_abs_gpu_vs_fp32_oracle": float(np.abs(l_g - lse_raw).max())}
 
 
 def cpu_oracle_sample(w: attn_inputs.Workload, rows: int, heads: int):
@@ -303,10 +527,9 @@ def run_reference(args, w, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N, "heads": w.H,
-                   "head_dim": w.d, "parallelism": "none (host cores)"},
+        "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu_model": cpu_model(), "host_cores": host_cores()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -321,6 +544,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c5", choices=sorted(attn_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing each configuration on its own")
+    ap.add_argument("--oracle-budget-gflop", type=float, default=ORACLE_BUDGET_GFLOP,
+                    help="per-configuration oracle work above which a row sample is timed")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -394,11 +621,24 @@ def main():
     # Three streams and two device buffer sets let step i+1's upload and step
     # i-1's download run while step i computes; events order each buffer's
     # reuse.  The timed region spans the first upload to the last download.
-    e2e_ms, h2d, d2h = e2e_pipelined(fa, w, args, dev, q, k, v, do, train, mk)
+    e2e_ms, h2d, d2h, copies = e2e_pipelined(fa, w, args, dev, q, k, v, do, train, mk)
     e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    pk, pk_src = peaks()
+
+    # ------------------------------ every configuration on its own (one GPU)
+    per_config = {}
+    c1_out = None
+    if world == 1 and not args.no_per_config:
+        for name in PER_CONFIG:
+            entry, o_c, lse_c = time_config(fa, attn_inputs.WORKLOADS[name], dev, flush,
+                                            PER_CONFIG_RUNS, local, pk)
+            per_config[name] = entry
+            if name == "c1":
+                c1_out = (o_c.cpu(), lse_c.cpu())
+        if fa.fa_get_device_status() != 0:
+            raise RuntimeError("a kernel gave up a bounded wait during the per-config timing")
 
     # ----------------------------------------- roofline of the dominant kernel
-    pk, pk_src = peaks()
     fwd_name, bwd_name = main_kernel_names(fa, w, torch.cuda.get_device_properties(dev))
     if train:
         dom, dom_ms, dom_flop = bwd_name, statistics.mean(bwd_ms), w.bwd_flop
@@ -433,7 +673,15 @@ def main():
             val, dt, threads, desc = cpu_oracle_sample(w, 1024 if train else 256,
                                                        max(1, min(threads, w.B * w.H)))
             cpu = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
-                   "sample": desc, "seconds": dt}
+                   "sample": desc, "seconds": dt, "cpu_model": cpu_model(),
+                   "host_cores": host_cores()}
+            # the oracle on each configuration (after all GPU work)
+            for name, entry in per_config.items():
+                cw = attn_inputs.WORKLOADS[name]
+                entry["oracle"] = oracle_time_config(cw, args.oracle_budget_gflop,
+                                                     single_core=name in ("c1", "c2"))
+                if name == "c1" and c1_out is not None:
+                    entry["c1_fp32_draws"] = c1_fp32_report(cw, *c1_out)
 
     if rank == 0:
         line = {
@@ -442,18 +690,13 @@ def main():
             "scaling": "weak", "vs_baseline": None,
             "dtype": {"bf16": "bf16", "fp16": "fp16", "fp8": "fp8e4m3"}[w.dtype],
             "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N,
-                       "heads": w.H, "head_dim": w.d, "causal": False,
-                       "parallelism": f"replicas x{world} (batch per rank, no collective)",
-                       "l2": "512 MiB written between timed steps",
-                       "inputs": "seeded N(0,1) draws rounded to the "
-                                 + ("E4M3 type (descale factors 1), bf16 O" if w.dtype == "fp8"
-                                    else "16-bit type")},
+            "config": workload_config(w, world),
             "e2e": {"value": job_tflops(flop_step, e2e_ms, world), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "how": "pinned host -> device inputs, step, device -> pinned host results "
                            "every step; uploads, kernels and downloads of neighbouring steps "
-                           "overlap on three streams (two device buffer sets)"},
+                           "overlap on three streams (two device buffer sets)",
+                    "copies_alone": copies},
             "gpu_launches": launches,
             "roofline": roofline,
             "kernels": kernels,
@@ -462,6 +705,8 @@ def main():
             "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
             "pct_of_dtype_peak": 100.0 * value / world / peak,
         }
+        if per_config:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

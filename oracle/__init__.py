@@ -88,11 +88,16 @@ class Oracle:
         lib.oracle_attn_bwd_rows.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, f, i, i, i]
         lib.oracle_attn_dscores.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, f, i]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [i]
         self.lib = lib
 
     def num_threads(self) -> int:
         """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all host cores)."""
         return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        """Use n OpenMP threads in later calls (timing only; no arithmetic changes)."""
+        self.lib.oracle_set_num_threads(int(n))
 
     def attn_fwd(self, q, k, v, scale, causal=False):
         """O = softmax(scale Q K^T) V and LSE (natural log) by the definition;
@@ -193,6 +198,10 @@ def default() -> Oracle:
 
 def num_threads():
     return default().num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    default().set_num_threads(n)
 
 
 def attn_fwd(q, k, v, scale, causal=False):

@@ -45,6 +45,18 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Threads for later calls (n >= 1); used to time the oracle on one core.
+ * Changes no arithmetic: every row is computed by one thread either way. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /*
  * Row i of the probability matrix, by the definition (YOLO11 page, 1.2):
  *   S_ij = scale * sum_x q_ix k_jx,  m_i = max_j S_ij,
