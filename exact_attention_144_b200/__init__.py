@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
     lib.fa_set_kernel_events.argtypes = [vp, vp, vp, vp]
     lib.fa_set_kernel_events.restype = i
     lib.fa_kernel_launches.restype = ctypes.c_ulonglong
+    lib.fa_scratch_allocs.restype = ctypes.c_ulonglong
     lib.fa_last_cuda_error.restype = i
     lib.fa_selftest_exp2.argtypes = [vp, vp, i, vp]
     lib.fa_selftest_exp2.restype = i
@@ -512,6 +513,11 @@ def fa_set_kernel_events(fwd_start=None, fwd_stop=None, bwd_start=None, bwd_stop
 def fa_kernel_launches() -> int:
     """Kernel launches this library has issued since it was loaded."""
     return int(_load().fa_kernel_launches())
+
+
+def fa_scratch_allocs() -> int:
+    """Scratch allocations this library has requested since it was loaded."""
+    return int(_load().fa_scratch_allocs())
 
 
 class _Attention(torch.autograd.Function):

@@ -50,56 +50,132 @@ static void arm_kernel_events(cudaEvent_t fs, cudaEvent_t fe, cudaEvent_t bs, cu
   g_events[3] = be;
 }
 
-unsigned long long* device_status_ptr() {
-  static std::mutex mu;
-  static unsigned long long* cached[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+// ------------------------------------------------------- context identity
+// Device addresses of __device__ variables and memory pools belong to a CUDA
+// context, not to a device number: after cudaDeviceReset, or with another
+// context current, the old values are stale.  Cached values are therefore
+// keyed by the unique ID of the context current on the calling thread
+// (cuCtxGetId, reached through the runtime's driver entry points).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static void* driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPointByVersion(name, &ptr, 12000, cudaEnableDefault, &qres) !=
+          cudaSuccess ||
+      qres != cudaDriverEntryPointSuccess) {
     cudaGetLastError();
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_status) == cudaSuccess)
-      cached[dev] = static_cast<unsigned long long*>(ptr);
-    else
-      cudaGetLastError();
+  return ptr;
+}
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_current = reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+    get_id = reinterpret_cast<CtxGetIdFn>(driver_fn("cuCtxGetId"));
+  });
+  CUcontext ctx = nullptr;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr)
+    return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Small table of (context ID, key) -> value, replaced round-robin when full.
+struct ContextCache {
+  struct Entry {
+    unsigned long long ctx;
+    const void* key;
+    void* value;
+  };
+  std::mutex mu;
+  Entry e[64] = {};
+  int n = 0, next = 0;
+  bool find(unsigned long long ctx, const void* key, void** value) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+      if (e[i].ctx == ctx && e[i].key == key) {
+        *value = e[i].value;
+        return true;
+      }
+    return false;
   }
-  return cached[dev];
+  void insert(unsigned long long ctx, const void* key, void* value) {
+    std::lock_guard<std::mutex> lock(mu);
+    const int i = n < 64 ? n++ : (next++ % 64);
+    e[i] = {ctx, key, value};
+  }
+};
+
+int symbol_address(const void* symbol, void** out) {
+  static ContextCache cache;
+  unsigned long long ctx = 0;
+  bool have = current_context_id(&ctx);
+  if (have && cache.find(ctx, symbol, out)) return FA_OK;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, symbol) != cudaSuccess || ptr == nullptr) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  if (!have) have = current_context_id(&ctx);  // the lookup made a context current
+  if (have) cache.insert(ctx, symbol, ptr);
+  *out = ptr;
+  return FA_OK;
+}
+
+unsigned long long* device_status_ptr() {
+  void* ptr = nullptr;
+  return symbol_address(&g_status, &ptr) == FA_OK ? static_cast<unsigned long long*>(ptr)
+                                                  : nullptr;
 }
 
 // ------------------------------------------------------------ scratch pool
+static std::atomic<unsigned long long> g_scratch_allocs{0};
+
+// The library's memory pool for device dev in the current context.
 static cudaMemPool_t scratch_pool(int dev) {
-  static std::mutex mu;
-  static cudaMemPool_t pools[64] = {nullptr};
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (pools[dev] == nullptr) {
-    cudaMemPoolProps props{};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.handleTypes = cudaMemHandleTypeNone;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t pool = nullptr;
-    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    unsigned long long keep = kScratchRetainBytes;
-    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
-      cudaGetLastError();  // still usable, only without retention
-    pools[dev] = pool;
+  static ContextCache cache;
+  static std::mutex create_mu;
+  const void* key = reinterpret_cast<const void*>((uintptr_t)dev + 1);
+  unsigned long long ctx = 0;
+  bool have = current_context_id(&ctx);
+  void* found = nullptr;
+  if (have && cache.find(ctx, key, &found)) return static_cast<cudaMemPool_t>(found);
+  std::lock_guard<std::mutex> lock(create_mu);
+  if (have && cache.find(ctx, key, &found)) return static_cast<cudaMemPool_t>(found);
+  cudaMemPoolProps props{};
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool = nullptr;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return pools[dev];
+  unsigned long long keep = kScratchRetainBytes;
+  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+    cudaGetLastError();  // still usable, only without retention
+  if (!have) have = current_context_id(&ctx);
+  if (have) cache.insert(ctx, key, pool);
+  return pool;
 }
 
+unsigned long long scratch_allocs() { return g_scratch_allocs.load(); }
+
 int scratch_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+  g_scratch_allocs.fetch_add(1);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_NOMEM;
   }
+  if (dev < 0) return FA_ERR_NOMEM;
   cudaMemPool_t pool = scratch_pool(dev);
   if (pool == nullptr || cudaMallocFromPoolAsync(ptr, bytes, pool, stream) != cudaSuccess) {
     cudaGetLastError();
@@ -609,6 +685,8 @@ FA_EXPORT int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
 }
 
 FA_EXPORT unsigned long long fa_kernel_launches(void) { return fa::g_launches.load(); }
+
+FA_EXPORT unsigned long long fa_scratch_allocs(void) { return fa::scratch_allocs(); }
 
 FA_EXPORT int fa_last_cuda_error(void) { return fa::g_last_cuda_error.load(); }
 

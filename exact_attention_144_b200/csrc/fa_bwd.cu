@@ -39,8 +39,6 @@
 // Tensor memory (d = 64): S^T [0,128), dP^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448).  Packed 16-bit P^T and dS^T overwrite the first
 // 32 columns of each 64-column query half of S^T and dP^T.
-#include <mutex>
-
 #include "fa_common.cuh"
 #include "fa_host.h"
 
@@ -1375,32 +1373,14 @@ template int bwd_launch<__half>(const void*, const void*, const void*, const voi
 // scratch (dQ accumulator, minus the base-2 LSE, D) lives in a file-scope device array
 // instead of a stream-ordered allocation, for callers that cannot allocate.
 // Host code cannot pass g_fixed_scratch itself to a kernel (in host code the
-// name denotes a host-side stand-in); its device address is looked up once
-// per device with cudaGetSymbolAddress and cached.
+// name denotes a host-side stand-in); its device address is looked up with
+// cudaGetSymbolAddress, with the device current, once per CUDA context (the
+// address belongs to the context: a reset device or another context gets its
+// own lookup).
 static constexpr size_t kFixedScratchBytes = (size_t)64 << 20;
 static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
 
-static int fixed_scratch_address(void** out) {
-  static std::mutex mu;
-  static void* cached[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_LAUNCH;
-  }
-  if (dev < 0 || dev >= 64) return FA_ERR_DEVICE;
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_fixed_scratch) != cudaSuccess || ptr == nullptr) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
-    cached[dev] = ptr;
-  }
-  *out = cached[dev];
-  return FA_OK;
-}
+static int fixed_scratch_address(void** out) { return symbol_address(&g_fixed_scratch, out); }
 
 template <class T, class Tr>
 static int run_bwd_fixed_scratch(const void* q, const void* k, const void* v, const void* o,

@@ -44,8 +44,21 @@ constexpr unsigned long long kScratchRetainBytes = 1ull << 30;
 int scratch_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 void scratch_free(void* ptr, cudaStream_t stream);
 
-// Device address of this library's status word on the current device.
+// Device address of this library's status word in the current context.
 unsigned long long* device_status_ptr();
+
+// Unique ID of the CUDA context current on the calling thread (cuCtxGetId);
+// false when none is current or the driver cannot report it.
+bool current_context_id(unsigned long long* id);
+
+// Device address of a __device__ variable of this library in the current
+// context: looked up with cudaGetSymbolAddress once per context (keyed by the
+// context's unique ID, so a reset device or another context never gets a
+// stale address).  FA_OK or FA_ERR_LAUNCH.
+int symbol_address(const void* symbol, void** out);
+
+// Number of scratch_alloc calls since the library was loaded.
+unsigned long long scratch_allocs();
 
 // Tensor map over a contiguous [B, N, H, d] tensor for TMA tile loads of
 // `box_rows` tokens x 128 bytes of one head (64 16-bit or 128 8-bit elements,

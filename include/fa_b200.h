@@ -220,9 +220,12 @@ int fa_varlen_bounds(const int *cu_seqlens_host, int b, int max_seqlen, int tota
  * rejected with FA_ERR_SCRATCH before any launch.  Every GPU that loads the
  * library holds the 64 MiB buffer until the process exits.
  *
- * The first call on a device looks up the buffer's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one buffer and it keeps the previous call's
+ * The first call in a CUDA context looks up the buffer's device address
+ * (cudaGetSymbolAddress, with the device current) and keeps it for that
+ * context only: the cache is keyed by the context's unique ID (cuCtxGetId),
+ * so after cudaDeviceReset, or with another context current, the next call
+ * looks the address up again.  Make the first call in a context before any
+ * stream capture.  All calls share the one buffer and it keeps the previous call's
  * contents (the part that must start at zero is cleared by every call):
  * calls whose work overlaps on the GPU -- on different streams, or from
  * different host threads without ordering -- race on it and give wrong
@@ -339,6 +342,14 @@ int fa_set_kernel_events(cudaEvent_t fwd_start, cudaEvent_t fwd_stop,
 
 /* Number of kernel launches this library has issued since it was loaded. */
 unsigned long long fa_kernel_launches(void);
+
+/*
+ * Number of scratch allocations this library has requested from its memory
+ * pool since it was loaded (one per forward call that needs split-K/V or
+ * balanced-schedule partials, one per backward call; fa_bwd_noalloc makes
+ * none).  Diagnostic only.
+ */
+unsigned long long fa_scratch_allocs(void);
 
 /*
  * The cudaError_t value behind the most recent FA_ERR_LAUNCH returned by any

@@ -14,6 +14,14 @@ import attn_inputs
 
 O_MAX, O_MEAN, LSE_MAX, GRAD_MAX = 2e-2, 2e-3, 1e-3, 5e-2
 
+# Secondary gates beside those bars: the RMS of the error relative to the RMS
+# of the fp64 result.  The max-abs bars are loose where the values are small
+# (the training workload's gradients are about 1e-2 in size), so a regression
+# could hide under them; 16-bit rounding of the outputs alone gives an RMS
+# relative error near 2^-9 / sqrt(3) = 1.1e-3, and the 16-bit P and dS add
+# errors of the same order.
+O_RMS_REL, GRAD_RMS_REL = 1e-2, 1e-2
+
 GUARD = 4096  # elements of sentinel after every output buffer
 
 
@@ -56,3 +64,33 @@ def sample_rows(B, H, N, count, seed=7):
     while len(rows) < count + 3 * B * H:
         rows.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))))
     return sorted(rows)
+
+
+def record(name: str, stats: dict) -> None:
+    """Appends one measured error record (JSON line) to the file named by
+    FA_TEST_RECORD, when that variable is set; the tests' gates do not
+    depend on it."""
+    import json
+    import os
+    path = os.environ.get("FA_TEST_RECORD")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **stats}) + "\n")
+
+
+def _case(name: str) -> str:
+    import os
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    return f"{test} {name}".strip()
+
+
+def o_ok(s: dict, name: str = "") -> bool:
+    """O within the max-abs and mean-abs bars and the RMS-relative gate."""
+    record(_case(name) + " O", s)
+    return s["max"] <= O_MAX and s["mean"] <= O_MEAN and s["rms_rel"] <= O_RMS_REL
+
+
+def grad_ok(s: dict, name: str = "") -> bool:
+    """A gradient within the max-abs bar and the RMS-relative gate."""
+    record(_case(name) + " grad", s)
+    return s["max"] <= GRAD_MAX and s["rms_rel"] <= GRAD_RMS_REL

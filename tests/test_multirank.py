@@ -51,7 +51,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_replicas_and_max_timing():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork after the oracle started threads
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     for r in range(world):

@@ -18,7 +18,8 @@ import torch
 
 import attn_inputs
 import oracle
-from tests.gpu_helpers import GRAD_MAX, LSE_MAX, O_MAX, O_MEAN, err_stats, sample_rows, to64
+from tests.gpu_helpers import (err_stats, grad_ok, o_ok, sample_rows, to64, GRAD_MAX, LSE_MAX,
+                               O_MAX, O_MEAN)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,7 +66,7 @@ def test_stage1_forward_sampled_rows(fa, inputs):
     idx = np.array(rows)
     eo = err_stats(to64(o)[idx[:, 0], idx[:, 2], idx[:, 1]], o_ref)
     el = err_stats(lse.cpu().double().numpy()[idx[:, 0], idx[:, 1], idx[:, 2]], lse_ref)
-    assert eo["max"] <= O_MAX and eo["mean"] <= O_MEAN, eo
+    assert o_ok(eo), eo
     assert el["max"] <= LSE_MAX, el
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
 
@@ -79,7 +80,7 @@ def test_stage1_backward_dq_rows(fa, inputs):
     dq = to64(dqkv[:, :, 0])
     for a, b in ROW_BLOCKS:
         s = err_stats(dq[:, a:b], dq_ref[:, a:b])
-        assert s["max"] <= GRAD_MAX, (a, b, s)
+        assert grad_ok(s, f"dq rows {a}:{b}"), (a, b, s)
 
 
 def test_stage1_backward_every_key_by_linearity(fa, inputs):
@@ -93,6 +94,6 @@ def test_stage1_backward_every_key_by_linearity(fa, inputs):
     ref = rows_oracle(host, to64(dout_r))
     for i, name in enumerate(("dq", "dk", "dv")):
         s = err_stats(to64(dqkv[:, :, i]), ref[i])
-        assert s["max"] <= GRAD_MAX, (name, s)
+        assert grad_ok(s, name), (name, s)
     # rows outside the kept set have dS = 0 exactly, so their dQ is zero
     assert bool((dqkv[:, ~keep, 0] == 0).all())
