@@ -71,6 +71,10 @@ for _n in (1024, 2048, 4096, 8192):
 # backward, to measure and test the d = 128 backward at full size.
 WORKLOADS["c4train"] = Workload("c4_train_n8192_h8_d128", 1, 8192, 8, 128, "bf16", 1006,
                                 backward=True, note="long-sequence shape, forward + backward")
+# The detector neck shape with a backward (not one of the pages'
+# configurations): measures and tests the d = 256 backward.
+WORKLOADS["c3train"] = Workload("c3_train_n6400_h1_d256", 1, 6400, 1, 256, "fp16", 1009, std=0.5,
+                                backward=True, note="detector neck shape, forward + backward")
 # The first stage of the YOLOv12 image page's network: a 160x160 feature map
 # (N = 25600 tokens) with 96 channels, attended as one head of d = 96, fp16,
 # Q, K, V packed per token.

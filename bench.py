@@ -41,8 +41,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 512 << 20
 L2_NOTE = "512 MiB written between timed GPU steps"
 # The pages' five configurations and the N sweep, each timed on its own in the
-# same run (forward; forward + backward for the training workload).
-PER_CONFIG = ("c1", "c2", "c3", "c4", "sweep1024", "sweep2048", "sweep4096", "sweep8192", "c5")
+# same run (forward; forward + backward for the training workload), and the
+# backward at the detector-neck (d = 256) and long-sequence (d = 128) shapes.
+PER_CONFIG = ("c1", "c2", "c3", "c4", "sweep1024", "sweep2048", "sweep4096", "sweep8192", "c5",
+              "c3train", "c4train")
 PER_CONFIG_RUNS = 20
 # The oracle runs a whole configuration when it costs at most this much work,
 # otherwise the first rows of every head, sized to about this much.
