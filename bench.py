@@ -159,7 +159,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.01):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self.period, self.stop_ev, self.thread = period_s, threading.Event(), None
         try:

@@ -34,8 +34,8 @@
 //   warp 11    idle (three whole warpgroups, so registers can move from the
 //              producer/MMA warpgroup to the compute ones)
 // Per Q tile i: dV += P^T dO_i as soon as P^T is written, then S^T for tile
-// i+1 (so the next P^T can start while dS^T is computed); dK += dS^T Q_i and
-// dQ_i = dS K as soon as dS^T is written, then dP^T for tile i+1.
+// i+1 (so the next P^T can start while dS^T is computed); dK += dS^T Q_i as
+// soon as dS^T is written, then dP^T for tile i+1, then dQ_i = dS K.
 // Tensor memory (d = 64): S^T [0,128), dP^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448).  Packed 16-bit P^T and dS^T overwrite the first
 // 32 columns of each 64-column query half of S^T and dP^T.
@@ -351,6 +351,20 @@ __global__ void __launch_bounds__(384, 1)
                     desc_advance(q_mn, (i % QST) * Tr::QT_BYTES + kk * 16 * 128), kIdescAcc,
                     (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_Q_EMPTY + i % QST));
+        }
+        // the next S^T (dP^T) overwrites TM_S (TM_DP) after dV (dK) has read
+        // P^T (dS^T): same issuing thread, so the tensor pipe keeps the order.
+        // Stream b issues it ahead of dQ_i, which reads dS from its own
+        // shared-memory buffer: the compute warps' next dS^T then waits only
+        // for dK, not for dQ and the dQ drain
+        if (more) {
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                                    kBSiteQFull)))
+            break;
+          tc_fence_after();
+          issue_first(i + 1);
+        }
+        if (!stream_a) {
           // dQ_i = dS K  (A = dS from shared memory, queries contiguous; B = K, d contiguous)
           if (i > 0 && !(ok = mbar_wait_warp(bar(Tr::B_DQ_FREE), (i - 1) & 1, w, kBSiteDqFree)))
             break;
@@ -362,15 +376,6 @@ __global__ void __launch_bounds__(384, 1)
                     desc_advance(k_mn, kk * 16 * 128), kIdescDQ, kk > 0 ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_DQ_FULL));
           umma_commit(leader, bar(Tr::B_DSBUF_FREE + (i & 1)));
-        }
-        // the next S^T (dP^T) overwrites TM_S (TM_DP) after dV (dK) has read
-        // P^T (dS^T): same issuing thread, so the tensor pipe keeps the order
-        if (more) {
-          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
-                                    kBSiteQFull)))
-            break;
-          tc_fence_after();
-          issue_first(i + 1);
         }
       }
       umma_commit(leader, bar(Tr::B_KV_DONE));
@@ -560,10 +565,10 @@ __global__ void __launch_bounds__(384, 1)
 // dV [256,384), dK [384,512).  Warps as in fa_bwd_kernel; compute warp w owns
 // lane quadrant w % 4 and query half w / 4 (32 columns) of S^T and dP^T, and
 // d quadrant w % 4, query half w / 4 of dQ^T.
-// The single dS^T staging tile needs no release barrier: the compute warps
-// rewrite it for tile i only after dP^T_i has completed, and dP^T_i is
-// committed after the dQ MMA of tile i - 1 (its last reader) by the same
-// thread, so that commit also covers the read.
+// The single dS^T staging tile is released by a barrier committed after the
+// dQ^T MMA of its tile: dP^T of tile i + 1 is issued right after dK of tile i,
+// ahead of dQ_i^T, so the compute warps may already build dS^T of tile i + 1
+// in registers and tensor memory while dQ_i^T still reads the tile.
 // At d = 96 the tiles keep the d = 128 layout: the second 64-column chunk of
 // every shared-memory row is half zero fill from the tensor map; S^T and dP^T
 // contract the 96 real columns, dV and dK are 96 columns wide (dK at
@@ -610,12 +615,17 @@ struct BwdTqTraits {
                        B_S_FULL = B_Q_EMPTY + QST, B_DP_FULL = B_S_FULL + 1,
                        B_P_READY = B_DP_FULL + 1, B_DS_READY = B_P_READY + 1,
                        B_DQ_FULL = B_DS_READY + 1, B_DQ_FREE = B_DQ_FULL + 2,
-                       B_KV_DONE = B_DQ_FREE + 2, B_DRAIN = B_KV_DONE + 1, NUM_BARS = B_DRAIN + 1;
+                       B_DSBUF_FREE = B_DQ_FREE + 2, B_KV_DONE = B_DSBUF_FREE + 1,
+                       B_DRAIN = B_KV_DONE + 1, NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 256 + DW;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries
+  // dP^T of the next tile ahead of dQ^T (below).  At d = 256 the single Q/dO
+  // stage already serialises the tiles, and the early order measured slower
+  // (B200, [1,6400,1,256] backward: 279.8 against 274.0 us)
+  static constexpr bool EARLY_DP = NHALF == 1;
   // dQ^T has DW rows: one 128-lane MMA tile (rows past d are zero and never drained)
   static_assert(D == 96 || D == 128 || D == 256, "head sizes of the transposed-dQ kernel");
   static_assert(TM_DK + DW <= TMEM_COLS, "tensor memory budget");
@@ -693,6 +703,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(Tr::B_DQ_FULL + s), 1);
       mbar_init(bar(Tr::B_DQ_FREE + s), 32 * Tr::NBOX);  // the draining warps
     }
+    mbar_init(bar(Tr::B_DSBUF_FREE), 1);
     mbar_init(bar(Tr::B_KV_DONE), 2);
     mbar_init(bar(Tr::B_DRAIN), 2);
     fence_mbar_init();
@@ -817,6 +828,19 @@ __global__ void __launch_bounds__(384, 1)
                     desc_advance(q_mn, qs * Tr::QT_BYTES + d_off_q + kk * 16 * 128), kIdescAcc,
                     (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_Q_EMPTY + qs));
+        }
+        // the next S^T (dP^T) after dV (dK) has read P^T (dS^T): same thread,
+        // in order.  With EARLY_DP stream b issues it ahead of dQ_i^T: the
+        // compute warps may then build the next dS^T while dQ_i^T runs, and
+        // wait for DSBUF_FREE before they rewrite the shared dS^T tile it reads
+        if (more && (stream_a || Tr::EARLY_DP)) {
+          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                                    kBSiteQFull)))
+            break;
+          tc_fence_after();
+          issue_first(i + 1);
+        }
+        if (!stream_a) {
           // dQ_i^T = K^T dS_i^T  (A = K: d contiguous, MN-major; B = dS^T: queries
           // contiguous, MN-major) into buffer i & 1, once its previous tile is drained
           const int qb = i & 1;
@@ -830,13 +854,14 @@ __global__ void __launch_bounds__(384, 1)
                     desc_advance(k_mn, d_off_k + kk * 16 * 128),
                     desc_advance(ds_mn, kk * 16 * 128), kIdescDQ, kk > 0 ? 1u : 0u);
           umma_commit(leader, bar(Tr::B_DQ_FULL + qb));
-        }
-        if (more) {
-          if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
-                                    kBSiteQFull)))
-            break;
-          tc_fence_after();
-          issue_first(i + 1);
+          umma_commit(leader, bar(Tr::B_DSBUF_FREE));
+          if (more && !Tr::EARLY_DP) {
+            if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL + (i + 1) % QST), ((i + 1) / QST) & 1, w,
+                                      kBSiteQFull)))
+              break;
+            tc_fence_after();
+            issue_first(i + 1);
+          }
         }
       }
       umma_commit(leader, bar(Tr::B_KV_DONE));
@@ -962,6 +987,12 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       tmem_st16(tl + Tr::TM_DP + hf * 32, ds16);
+      // the shared dS^T tile is rewritten only after dQ^T of the previous tile
+      // has read it (without EARLY_DP, dP^T of this tile already followed it)
+      if (Tr::EARLY_DP && i > 0) {
+        ok = mbar_wait(bar(Tr::B_DSBUF_FREE), (i - 1) & 1, w, kBSiteDsBuf);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      }
       // dS^T row r (key), queries [32 hf, 32 hf + 32): 16-byte chunks 4 hf .. 4 hf + 3
       // of the 128-byte-swizzled row
       uint8_t* ds_row = gDS + r * 128;

@@ -206,6 +206,15 @@ enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteP
 // Growth of the running max (base 2) tolerated before O is rescaled.
 constexpr float kRescaleThreshold = 8.0f;
 
+// k-steps of a P.V product over K/V tile t that hold keys below the
+// sequence's length len (16 keys a step for 16-bit P, 32 for 8-bit P): the
+// ragged last tile needs only those, as P and V are zero past the end.
+template <int BN, int EB>
+__host__ __device__ __forceinline__ int pv_steps(int len, int t) {
+  const int keys = len - t * BN < BN ? len - t * BN : BN;
+  return (keys * EB + 31) / 32;
+}
+
 
 // ---------------------------------------------------------------------------
 // One softmax step for the row a thread owns.  r holds the row's BN raw scores
@@ -219,11 +228,17 @@ constexpr float kRescaleThreshold = 8.0f;
 // on the long-sequence workload); where two warps per SM sub-partition run
 // their softmax together (d = 64) the extra instructions cost more than MUFU
 // time saved (225 -> 241 us), so there it is 0.
-template <class T, int BN, int EMU = 0>
+// SKIP: partial tiles skip the 32-column chunks that hold no valid column of
+// any row of the warp (warp votes; all 32 lanes must call together).
+template <class T, int BN, int EMU = 0, bool SKIP = true>
 __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], int valid, float c,
                                               float& m, float& l, uint32_t (&pk)[BN / 2]) {
   auto S = [&](int j) { return __uint_as_float(r[j / 32][j % 32]); };
-  const bool full = valid >= BN;
+  // full: every column of the row is valid.  With SKIP it is decided for the
+  // whole warp: the partial path then takes warp votes, and a causal
+  // diagonal tile holds full and partial rows in one warp (the partial path
+  // is exact for full rows too).
+  const bool full = SKIP ? __all_sync(0xffffffffu, valid >= BN) : valid >= BN;
   const bool neg = c < 0.f;
   // row max of s*c (the min of s when c < 0): 8 independent chains, two new
   // columns per three-input max
@@ -248,12 +263,20 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
                  fminf(part[6], part[7]));
     }
   } else {
+    // a partial tile (the ragged end of the keys, or the causal diagonal):
+    // 32-column chunks past every valid column of the warp's rows are skipped
     float part[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) part[q] = neg ? INFINITY : -INFINITY;
 #pragma unroll
-    for (int j = 0; j < BN; ++j)
-      if (j < valid) part[j & 7] = neg ? fminf(part[j & 7], S(j)) : fmaxf(part[j & 7], S(j));
+    for (int q = 0; q < BN / 32; ++q)
+      if (!SKIP || __any_sync(0xffffffffu, q * 32 < valid)) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = q * 32 + jj;
+          if (j < valid) part[j & 7] = neg ? fminf(part[j & 7], S(j)) : fmaxf(part[j & 7], S(j));
+        }
+      }
     if (!neg)
       mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
                  fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
@@ -297,11 +320,20 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
 #pragma unroll
     for (int q = 0; q < 8; ++q) sum[q] = 0.f;
 #pragma unroll
-    for (int j = 0; j < BN / 2; ++j) {
-      const float p0 = (2 * j < valid) ? ex2(fmaf(S(2 * j), c, neg_m)) : 0.f;
-      const float p1 = (2 * j + 1 < valid) ? ex2(fmaf(S(2 * j + 1), c, neg_m)) : 0.f;
-      sum[j & 7] += p0 + p1;
-      pk[j] = Elem<T>::pack(p0, p1);
+    for (int q = 0; q < BN / 32; ++q) {
+      if (!SKIP || __any_sync(0xffffffffu, q * 32 < valid)) {
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = q * 16 + jj;
+          const float p0 = (2 * j < valid) ? ex2(fmaf(S(2 * j), c, neg_m)) : 0.f;
+          const float p1 = (2 * j + 1 < valid) ? ex2(fmaf(S(2 * j + 1), c, neg_m)) : 0.f;
+          sum[j & 7] += p0 + p1;
+          pk[j] = Elem<T>::pack(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) pk[q * 16 + jj] = 0u;  // P = 0: finite for P.V
+      }
     }
     rs = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
   }
@@ -498,7 +530,7 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
 // ===========================================================================
 // fa_fwd_pp_kernel: two Q tiles per unit
 // ===========================================================================
-template <int D_, int KST_, int VST_, int EB_ = 2, int EMU_ = -1>
+template <int D_, int KST_, int VST_, int EB_ = 2, int EMU_ = -1, int DUAL_ = -1>
 struct FwdPPTraits {
   static constexpr int D = D_;
   static constexpr int EB = EB_;          // bytes an element of Q, K, V
@@ -529,6 +561,21 @@ struct FwdPPTraits {
   // as soon as the softmax warps have read it, before P.V has consumed P.
   // Otherwise (d = 128) P is written over the first BN/2 columns of its S.
   static constexpr bool SEP_P = 2 * BN + 2 * P_COLS + 2 * D <= 512;
+  // DUAL: each Q tile's products are issued by its own thread (warp 9:
+  // tile 0, warp 10: tile 1); the release barriers of the K and V stages and
+  // of the Q pair then count one commit from each.  Where P has its own
+  // columns (d = 64): measured on B200, [4,4096,8,64] 228.6 -> 213.7 us.
+  // Where P is written over S (d = 96, 128, 8-bit) the products of both
+  // tiles share one issuer: two measured far slower there ([1,8192,8,128]:
+  // 284.6 -> 363.9 us).
+  static constexpr bool DUAL = DUAL_ >= 0 ? DUAL_ != 0 : SEP_P;
+  // Short-sequence measures (warps with no live row skip the softmax, the
+  // ragged last K/V tile skips its empty 32-column chunks and P.V k-steps):
+  // taken where P has its own columns; the d = 96, 128 and 8-bit kernels,
+  // bound by the tensor-core issue rate, keep their plain loops (with the
+  // measures, [1,8192,8,128] took 284.6 us against 272.9 us).
+  static constexpr bool SHORT = SEP_P;
+  static constexpr int NISSUE = DUAL ? 2 : 1;
   // exponentials on the FMA pipe per 8 column pairs (see softmax_step): the
   // d = 128 warpgroups take turns, the d = 64 ones run together.  Measured on
   // B200 for d = 128 (bf16 / 8-bit, [1,8192,8,128], us): 1: 269.6 / 243.0,
@@ -562,14 +609,14 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(Tr::B_Q_FULL), 1);
-    mbar_init(bar(Tr::B_Q_EMPTY), 1);
+    mbar_init(bar(Tr::B_Q_EMPTY), Tr::NISSUE);
     for (int s = 0; s < KST; ++s) {
       mbar_init(bar(Tr::B_K_FULL + s), 1);
-      mbar_init(bar(Tr::B_K_EMPTY + s), 1);
+      mbar_init(bar(Tr::B_K_EMPTY + s), Tr::NISSUE);
     }
     for (int s = 0; s < VST; ++s) {
       mbar_init(bar(Tr::B_V_FULL + s), 1);
-      mbar_init(bar(Tr::B_V_EMPTY + s), 1);
+      mbar_init(bar(Tr::B_V_EMPTY + s), Tr::NISSUE);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Tr::B_S_FULL + s), 1);
@@ -577,7 +624,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(Tr::B_O_DONE + s), 1);
       mbar_init(bar(Tr::B_S_FREE + s), 128);
     }
-    mbar_init(bar(Tr::B_DRAIN), 1);
+    mbar_init(bar(Tr::B_DRAIN), Tr::NISSUE);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -644,8 +691,8 @@ __global__ void __launch_bounds__(384, 1)
         if (vc > s) mbar_drain(bar(Tr::B_V_FULL + s), ((vc - 1 - s) / VST) & 1u, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ----------------------------------------------------- MMA issuer
+  } else if (warp == 9 || (Tr::DUAL && warp == 10)) {
+    // ---------------------------------------------------- MMA issuer(s)
     {
       const bool leader = lane == 0;  // issues; all lanes run the loop
       constexpr uint32_t kIdescQK = f16_idesc(Elem<T>::kFmt, 128, BN, false);
@@ -666,62 +713,76 @@ __global__ void __launch_bounds__(384, 1)
                   desc_advance(kd, ch * (BN * 128) + in), kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t (+)= P_t V for the V stage of counter vc
-      auto issue_pv = [&](int t, bool first) {
+      // O_t (+)= P_t V for the V stage of counter vc; only the k-steps that
+      // hold keys below the sequence's end (P and V are zero past it)
+      auto issue_pv = [&](int t, bool first, int nsteps) {
+        constexpr int kSteps = BN * Tr::EB / 32;  // 32 keys x 16 bits, or 32 x 8 bits
         const uint64_t vd = desc_advance(v_desc0, (vc % VST) * Tr::KV_BYTES);
         const uint32_t pa = Tr::SEP_P ? Tr::TM_P + t * Tr::P_COLS : t * BN;
+        if (nsteps >= kSteps) {
 #pragma unroll
-        for (int kk = 0; kk < BN * Tr::EB / 32; ++kk)  // 32 keys x 16 bits, or 32 x 8 bits
-          mma_ts<T>(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
-                    desc_advance(vd, kk * (32 / Tr::EB) * 128), kIdescPV,
-                    (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kSteps; ++kk)
+            mma_ts<T>(leader, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
+                      desc_advance(vd, kk * (32 / Tr::EB) * 128), kIdescPV,
+                      (!first || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kSteps; ++kk)
+            mma_ts<T>(leader && kk < nsteps, tmem + Tr::TM_O + t * D, tmem + pa + kk * 8,
+                      desc_advance(vd, kk * (32 / Tr::EB) * 128), kIdescPV,
+                      (!first || kk > 0) ? 1u : 0u);
+        }
       };
       UnitIter<VARLEN> it(p, blockIdx.x);
-      if constexpr (Tr::SEP_P) {
-        // S_0, S_1 of the next K/V tile are issued as soon as both softmax
-        // warpgroups have read the current ones (S_FREE), ahead of P.V; the
-        // tensor cores then compute the next scores while the exponentials of
-        // the current tile run, and each warpgroup can go straight on to its
-        // next tile.  Per K/V tile: Q0 K^T, Q1 K^T (next tile), P0 V, P1 V.
-        uint32_t sq = 0;  // S tiles issued per Q tile
-        auto issue_s_pair = [&]() -> bool {
+      if constexpr (Tr::DUAL) {
+        // Issuer t (warp 9 + t) owns Q tile t and walks its chain alone:
+        // S_t(j) = Q_t K_j^T -> softmax of warpgroup t -> O_t += P_t(j) V_j, so
+        // neither tile waits for the other tile's softmax.  With P in its own
+        // columns S_t(j+1) is issued as soon as warpgroup t has read S_t(j)
+        // into registers, ahead of P_t(j) V_j (the tensor cores compute the
+        // next scores while the exponentials run); with P written over S it
+        // follows P_t(j) V_j, which has read P (same thread: in order).
+        const int t = warp - 9;
+        uint32_t gs = 0;  // S tiles this issuer has issued
+        auto issue_s = [&](int j, int n) -> bool {
           if (!mbar_wait_warp(bar(Tr::B_K_FULL + kc % KST), (kc / KST) & 1u, w, kSiteKFull))
             return false;
-#pragma unroll 1
-          for (int t = 0; t < 2; ++t) {
-            if (sq > 0 && !mbar_wait_warp(bar(Tr::B_S_FREE + t), (sq - 1) & 1u, w, kSiteSFree))
-              return false;
-            tc_fence_after();
-            issue_qk(t);
-            umma_commit(leader, bar(Tr::B_S_FULL + t));
-          }
+          if (Tr::SEP_P && gs > 0 &&
+              !mbar_wait_warp(bar(Tr::B_S_FREE + t), (gs - 1) & 1u, w, kSiteSFree))
+            return false;
+          tc_fence_after();
+          issue_qk(t);
+          umma_commit(leader, bar(Tr::B_S_FULL + t));
           umma_commit(leader, bar(Tr::B_K_EMPTY + kc % KST));
+          if (j == n - 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
           ++kc;
-          ++sq;
+          ++gs;
+          return true;
+        };
+        auto issue_o = [&](const Unit& un, int j) -> bool {
+          if (!mbar_wait_warp(bar(Tr::B_P_FULL + t), g & 1u, w, kSitePFull)) return false;
+          if (!mbar_wait_warp(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull))
+            return false;
+          tc_fence_after();
+          issue_pv(t, j == 0, pv_steps<BN, Tr::EB>(un.len, un.t0 + j));
+          umma_commit(leader, bar(Tr::B_O_DONE + t));
+          umma_commit(leader, bar(Tr::B_V_EMPTY + vc % VST));
+          ++vc;
+          ++g;
           return true;
         };
         for (Unit un; ok && it.next(p, un);) {
           const int n = un.t1 - un.t0;
           if (!(ok = mbar_wait_warp(bar(Tr::B_Q_FULL), uc & 1u, w, kSiteQFull))) break;
-          if (!(ok = issue_s_pair())) break;
-          if (n == 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
-          for (int j = 0; j < n; ++j, ++g) {
-            if (j + 1 < n) {
-              if (!(ok = issue_s_pair())) break;
-              if (j + 2 == n) umma_commit(leader, bar(Tr::B_Q_EMPTY));
+          ok = issue_s(0, n);
+          for (int j = 0; j < n && ok; ++j) {
+            if (Tr::SEP_P) {
+              if (j + 1 < n && !(ok = issue_s(j + 1, n))) break;
+              ok = issue_o(un, j);
+            } else {
+              if (!(ok = issue_o(un, j))) break;
+              if (j + 1 < n) ok = issue_s(j + 1, n);
             }
-            if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 0), g & 1u, w, kSitePFull))) break;
-            if (!(ok = mbar_wait_warp(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
-              break;
-            tc_fence_after();
-            issue_pv(0, j == 0);
-            umma_commit(leader, bar(Tr::B_O_DONE + 0));
-            if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
-            tc_fence_after();
-            issue_pv(1, j == 0);
-            umma_commit(leader, bar(Tr::B_O_DONE + 1));
-            umma_commit(leader, bar(Tr::B_V_EMPTY + vc % VST));
-            ++vc;
           }
           if (!ok) break;
           ++uc;
@@ -745,7 +806,8 @@ __global__ void __launch_bounds__(384, 1)
           if (!(ok = mbar_wait_warp(bar(Tr::B_V_FULL + vc % VST), (vc / VST) & 1u, w, kSiteVFull)))
             break;
           tc_fence_after();
-          issue_pv(0, j == 0);
+          const int nsteps = Tr::SHORT ? pv_steps<BN, Tr::EB>(un.len, un.t0 + j) : BN * Tr::EB / 32;
+          issue_pv(0, j == 0, nsteps);
           umma_commit(leader, bar(Tr::B_O_DONE + 0));
           const bool more = j + 1 < n;
           if (more) {
@@ -758,7 +820,7 @@ __global__ void __launch_bounds__(384, 1)
           // tile 1: P1 V_j, then S1 for the next K tile
           if (!(ok = mbar_wait_warp(bar(Tr::B_P_FULL + 1), g & 1u, w, kSitePFull))) break;
           tc_fence_after();
-          issue_pv(1, j == 0);
+          issue_pv(1, j == 0, nsteps);
           umma_commit(leader, bar(Tr::B_O_DONE + 1));
           umma_commit(leader, bar(Tr::B_V_EMPTY + vc % VST));
           ++vc;
@@ -795,6 +857,27 @@ __global__ void __launch_bounds__(384, 1)
     for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
+      // a warp whose 32 rows all lie past the sequence's end (the ragged last
+      // Q tile of short sequences) skips the softmax -- its O rows are never
+      // stored -- but takes every barrier step with the other warps
+      const bool live =
+          !Tr::SHORT || __any_sync(0xffffffffu, (2 * un.qt + wg) * BM + row < un.len);
+      if (!live) {
+        for (int j = 0; j < n; ++j, ++g) {
+          ok = mbar_wait(bar(Tr::B_S_FULL + wg), g & 1u, w, kSiteSFull);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          if constexpr (Tr::SEP_P) {
+            tc_fence_before();
+            mbar_arrive(bar(Tr::B_S_FREE + wg));
+          }
+          if (Tr::SEP_P ? g > 0 : j > 0) {
+            ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteODone);
+            if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          }
+          tc_fence_before();
+          mbar_arrive(bar(Tr::B_P_FULL + wg));
+        }
+      } else
       for (int j = 0; j < n; ++j, ++g) {
         ok = mbar_wait(bar(Tr::B_S_FULL + wg), g & 1u, w, kSiteSFull);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
@@ -816,7 +899,7 @@ __global__ void __launch_bounds__(384, 1)
         const int t = un.t0 + j;
         int valid = un.len - t * BN;
         if (p.causal) valid = imin(valid, (2 * un.qt + wg) * BM + row - t * BN + 1);
-        const float alpha = softmax_step<T, BN, Tr::EMU>(r, valid, c, m, l, pk);
+        const float alpha = softmax_step<T, BN, Tr::EMU, Tr::SHORT>(r, valid, c, m, l, pk);
         if constexpr (Tr::SEP_P) {
           // P has one buffer per Q tile: the previous P.V (the previous tile of
           // this unit, or the last of the previous unit, already waited for by
@@ -1013,19 +1096,29 @@ __global__ void __launch_bounds__(224, 1)
       bool ok = true;
       const uint64_t q_desc0 = sw128_desc(sQ, 16, 1024), k_desc0 = sw128_desc(sK, 16, 1024),
                      v_desc0 = sw128_desc(sV, BN * 128, 1024);
-      // O += P_j V_j for the tile whose S/P buffer use counter is gp.
-      auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+      // O += P_j V_j for the tile whose S/P buffer use counter is gp (nsteps
+      // k-steps: those with keys below the sequence's end).
+      auto issue_pv = [&](uint32_t gp, bool first, int nsteps) -> bool {
         const uint32_t pb = gp & 1u;
         if (!mbar_wait_warp(bar(Tr::B_P_FULL + pb), (gp >> 1) & 1u, w, kSitePFull)) return false;
         const uint32_t vs = vc % VST;
         if (!mbar_wait_warp(bar(Tr::B_V_FULL + vs), (vc / VST) & 1u, w, kSiteVFull)) return false;
         tc_fence_after();
         const uint64_t vd = desc_advance(v_desc0, vs * Tr::KV_BYTES);
+        constexpr int kSteps = BN * Tr::EB / 32;
+        if (nsteps >= kSteps) {
 #pragma unroll
-        for (int kk = 0; kk < BN * Tr::EB / 32; ++kk)
-          mma_ts<T>(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
-                  desc_advance(vd, kk * (32 / Tr::EB) * 128),
-                  kIdescPV, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kSteps; ++kk)
+            mma_ts<T>(leader, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
+                      desc_advance(vd, kk * (32 / Tr::EB) * 128),
+                      kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kSteps; ++kk)
+            mma_ts<T>(leader && kk < nsteps, tmem + Tr::TM_O, tmem + pb * BN + kk * 8,
+                      desc_advance(vd, kk * (32 / Tr::EB) * 128),
+                      kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        }
         umma_commit(leader, bar(Tr::B_V_EMPTY + vs));
         umma_commit(leader, bar(Tr::B_O_DONE));
         ++vc;
@@ -1052,11 +1145,13 @@ __global__ void __launch_bounds__(224, 1)
           umma_commit(leader, bar(Tr::B_S_FULL + sb));
           if (i == n - 1) umma_commit(leader, bar(Tr::B_Q_EMPTY));
           ++kc;
-          if (i > 0 && !(ok = issue_pv(g - 1, i == 1))) break;
+          if (i > 0 &&
+              !(ok = issue_pv(g - 1, i == 1, pv_steps<BN, Tr::EB>(un.len, un.t0 + i - 1))))
+            break;
           ++g;
         }
         if (!ok) break;
-        if (!(ok = issue_pv(g - 1, n == 1))) break;
+        if (!(ok = issue_pv(g - 1, n == 1, pv_steps<BN, Tr::EB>(un.len, un.t1 - 1)))) break;
         ++uc;
       }
       // Every issued MMA must finish before tensor memory is released.
@@ -1075,32 +1170,38 @@ __global__ void __launch_bounds__(224, 1)
     for (Unit un; ok && it.next(p, un);) {
       float m = -INFINITY, l = 0.f;
       const int n = un.t1 - un.t0;
+      // a warp whose rows all lie past the sequence's end skips the softmax
+      // (its O rows are never stored) but takes every barrier step
+      const bool live = __any_sync(0xffffffffu, un.qt * Tr::BM + row < un.len);
       for (int i = 0; i < n; ++i, ++g) {
         const uint32_t sb = g & 1u;
         ok = mbar_wait(bar(Tr::B_S_FULL + sb), (g >> 1) & 1u, w, kSiteSFull);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
         const uint32_t scol = tl + sb * BN;
-        uint32_t r[BN / 32][32];
+        float alpha = 1.f;
+        if (live) {
+          uint32_t r[BN / 32][32];
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q) tmem_ld32(scol + q * 32, r[q]);
-        tmem_wait_ld();
+          for (int q = 0; q < BN / 32; ++q) tmem_ld32(scol + q * 32, r[q]);
+          tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
-        uint32_t pk[BN / 2];
-        const int t = un.t0 + i;
-        int valid = un.len - t * BN;
-        if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
-        const float alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
-        store_p<T, BN>(scol, pk);
-        tmem_wait_st();
+          for (int q = 0; q < BN / 32; ++q) reg_fence(r[q]);
+          uint32_t pk[BN / 2];
+          const int t = un.t0 + i;
+          int valid = un.len - t * BN;
+          if (p.causal) valid = imin(valid, un.qt * Tr::BM + row - t * BN + 1);
+          alpha = softmax_step<T, BN>(r, valid, c, m, l, pk);
+          store_p<T, BN>(scol, pk);
+          tmem_wait_st();
+        }
         if (i > 0) {
           // O holds P_{<j} V_{<j}: once the previous P.V has landed, rescale it
           // (if a row's reference max moved) before this tile's P.V is issued.
           ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteODone);
           if (!(ok = __all_sync(0xffffffffu, ok))) break;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(tl + Tr::TM_O, alpha);
+          if (live && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(tl + Tr::TM_O, alpha);
         }
         tc_fence_before();
         mbar_arrive(bar(Tr::B_P_FULL + sb));
