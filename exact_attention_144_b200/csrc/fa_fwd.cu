@@ -206,6 +206,9 @@ enum { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteP
 // Growth of the running max (base 2) tolerated before O is rescaled.
 constexpr float kRescaleThreshold = 8.0f;
 
+// Longest sequence whose forward epilogue goes through the staging tiles.
+constexpr int kStagedMaxN = 1024;
+
 // k-steps of a P.V product over K/V tile t that hold keys below the
 // sequence's length len (16 keys a step for 16-bit P, 32 for 8-bit P): the
 // ragged last tile needs only those, as P and V are zero past the end.
@@ -527,6 +530,58 @@ __device__ __forceinline__ bool store_row(const FwdParams& p, const Unit& un, ui
   return true;
 }
 
+// Epilogue of a whole unit's row in direct mode (O rounded to 16 bits, LSE
+// natural log) through a per-warp staging tile in shared memory: each thread
+// writes its row's 16-byte chunks there (chunk u of row r at position
+// u ^ (r & 7): conflict-free), then the warp writes the tile back row by row,
+// each store instruction covering RPI whole rows (one 16-byte chunk a lane),
+// instead of every store touching 32 rows.  stg: the warp's 32 x D x 2-byte
+// tile.  Collective over the warp.
+template <class T, int D>
+__device__ __forceinline__ void store_row_staged(const FwdParams& p, const Unit& un, uint32_t taddr,
+                                                 int q_row, float m, float l, uint8_t* stg) {
+  constexpr int CPR = D * 2 / 16;  // 16-byte chunks a row
+  constexpr int RPI = 32 / CPR;    // rows a warp store instruction covers
+  const int lane = threadIdx.x & 31;
+  const float inv_l = p.o_scale / l;
+  const float lse2 = m + lg2(l);
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(taddr + c * 32, o);
+    tmem_wait_ld();
+    reg_fence(o);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint4 v;
+      v.x = Elem<T>::pack(__uint_as_float(o[8 * u]) * inv_l, __uint_as_float(o[8 * u + 1]) * inv_l);
+      v.y = Elem<T>::pack(__uint_as_float(o[8 * u + 2]) * inv_l,
+                          __uint_as_float(o[8 * u + 3]) * inv_l);
+      v.z = Elem<T>::pack(__uint_as_float(o[8 * u + 4]) * inv_l,
+                          __uint_as_float(o[8 * u + 5]) * inv_l);
+      v.w = Elem<T>::pack(__uint_as_float(o[8 * u + 6]) * inv_l,
+                          __uint_as_float(o[8 * u + 7]) * inv_l);
+      const int chunk = c * 4 + u;
+      *reinterpret_cast<uint4*>(stg + lane * (CPR * 16) + ((chunk ^ (lane & 7)) * 16)) = v;
+    }
+  }
+  const int row0 = q_row - lane;  // the warp's first row (q_row = row0 + lane)
+  if (q_row < un.len)
+    p.lse[((size_t)un.tb * p.H + un.h) * p.total + un.tok0 + q_row] = lse2 * kLn2;
+  __syncwarp();
+  const int sub = lane / CPR, chunk = lane % CPR;
+#pragma unroll
+  for (int it = 0; it < 32 / RPI; ++it) {
+    const int r = it * RPI + sub;
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + r * (CPR * 16) + ((chunk ^ (r & 7)) * 16));
+    if (row0 + r < un.len) {
+      const size_t tok = (size_t)un.tb * p.total + un.tok0 + row0 + r;
+      reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.o) + (tok * p.H + un.h) * D)[chunk] = v;
+    }
+  }
+  __syncwarp();  // the tile is rewritten by the next unit's epilogue
+}
+
 // ===========================================================================
 // fa_fwd_pp_kernel: two Q tiles per unit
 // ===========================================================================
@@ -548,7 +603,10 @@ struct FwdPPTraits {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  // d = 64: the epilogue's per-warp O staging tiles (8 warps x 32 rows)
+  static constexpr int STG_BYTES = (D == 64 && EB == 2) ? 8 * 32 * D * 2 : 0;
+  static constexpr int OFF_STG = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
                        B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
                        B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
@@ -575,6 +633,7 @@ struct FwdPPTraits {
   // bound by the tensor-core issue rate, keep their plain loops (with the
   // measures, [1,8192,8,128] took 284.6 us against 272.9 us).
   static constexpr bool SHORT = SEP_P;
+  static_assert(!SHORT || STG_BYTES > 0, "the short-sequence kernel stages its epilogue");
   static constexpr int NISSUE = DUAL ? 2 : 1;
   // exponentials on the FMA pipe per 8 column pairs (see softmax_step): the
   // d = 128 warpgroups take turns, the d = 64 ones run together.  Measured on
@@ -932,7 +991,15 @@ __global__ void __launch_bounds__(384, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE + wg), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      ok = store_row<typename Elem<T>::Out, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l, w);
+      // staged for short sequences, where the epilogue is a large share of a
+      // unit (B200 [32,400,4,64]: 29.5 -> 27.7 us); long ones keep the direct
+      // stores (staged, [4,4096,8,64] measured 212.4 -> 214.9 us)
+      if (Tr::SHORT && p.N <= kStagedMaxN && un.kind == kStoreWhole && p.o_part == nullptr)
+        store_row_staged<typename Elem<T>::Out, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m,
+                                                   l, gbase + Tr::OFF_STG + warp * (32 * D * 2));
+      else
+        ok = store_row<typename Elem<T>::Out, D>(p, un, o_col, (2 * un.qt + wg) * BM + row, m, l,
+                                                 w);
     }
   }
 
