@@ -55,16 +55,22 @@ ORACLE_BUDGET_GFLOP = 40.0
 # while the kernel sources' code (comments excluded) hashes to the recorded
 # value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.760768e6 + 22.263552e6,
-                                                    "src": "212dbf11be8bd47c"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.544896e6 + 2.624768e6,
-                                                       "src": "212dbf11be8bd47c"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.674176e6 + 3.452160e6,
-                                                    "src": "212dbf11be8bd47c"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.681152e6 + 114.389504e6,
-                                                     "src": "212dbf11be8bd47c"},
-    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.275904e6 + 0.216832e6,
-                                                        "src": "212dbf11be8bd47c"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.762048e6 + 25.734656e6,
+                                                    "src": "bcf1af2045ebf704"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.488576e6 + 1.955840e6,
+                                                       "src": "bcf1af2045ebf704"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 50.873088e6 + 4.357376e6,
+                                                    "src": "bcf1af2045ebf704"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 103.645952e6 + 115.715328e6,
+                                                     "src": "bcf1af2045ebf704"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.273088e6 + 0.469248e6,
+                                                        "src": "bcf1af2045ebf704"},
+    ("fa_fwd_pp_kernel", "c2_detector_deep_b32_n400_h4_d64"): {"bytes": 19.759616e6,
+                                                               "src": "bcf1af2045ebf704"},
+    ("fa_fwd_kernel", "c3_detector_neck_n6400_h1_d256"): {"bytes": 9.939712e6,
+                                                          "src": "bcf1af2045ebf704"},
+    ("fa_bwd_tq_kernel", "c3_train_n6400_h1_d256"): {"bytes": 20.033024e6 + 6.752e6,
+                                                     "src": "bcf1af2045ebf704"},
 }
 
 
@@ -383,12 +389,16 @@ def time_config(fa, w: attn_inputs.Workload, dev, flush, runs: int, local: int, 
     fwd_name, bwd_name = main_kernel_names(fa, w, props)
     peak, peak_sus, _ = tensor_peak(pk, w)
 
+    src_hash = kernel_source_hash()
+
     def part(kern_ms, call_ms, flop, nbytes, name):
         k_mean, k_med = _stats(kern_ms)
         c_mean, c_med = _stats(call_ms)
         tf = flop / (k_mean * 1e-3) / 1e12
         gbs = nbytes / (k_mean * 1e-3) / 1e9
+        tr = TRAFFIC.get((name.split(" ")[0], w.name))
         return {"kernel": name, "kernel_us": 1e3 * k_mean, "kernel_us_median": 1e3 * k_med,
+                "traffic": tr["bytes"] if tr and tr["src"] == src_hash else None,
                 "call_us": 1e3 * c_mean, "call_us_median": 1e3 * c_med,
                 "kernel_cycles": (1e3 * k_mean * mhz) if mhz else None,
                 "tflops": tf, "pct_peak": 100.0 * tf / peak,
