@@ -75,7 +75,11 @@ struct BwdTraits64 {
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int ACC_BOX_ROWS = 32;  // dQ reduce box: 32 d columns x 32 queries (one warp's)
-  static constexpr int EMU = 0;  // exponentials on the FMA pipe per 8 column pairs of P^T
+  // exponentials on the FMA pipe per 8 column pairs of P^T: the compute
+  // warps' exponentials are MUFU-bound (16 a clock per SM).  Measured on
+  // B200, [4,4096,8,64] backward kernel: 0: 453.3, 1: 447.2, 2: 436.5,
+  // 3: 439.4 us
+  static constexpr int EMU = 2;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
