@@ -1383,7 +1383,7 @@ int plan_fwd(int B, int H, int N, int d, unsigned flags, int sm_count, FwdSchedu
   // accumulator leaves tensor memory room for only one Q tile).
   x.pair = (N > 128 && d <= 128) ? 1 : 0;
   x.unit_rows = x.pair ? 256 : 128;
-  x.bn = d == 256 ? 64 : 128;
+  x.bn = 128;
   x.n_qt = (N + x.unit_rows - 1) / x.unit_rows;
   x.n_kvt = (N + x.bn - 1) / x.bn;
   const long long base_units = (long long)B * H * x.n_qt;
@@ -1577,8 +1577,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse,
                       : run_single<T, FwdTraits<128, 128, 3, 2>>(s, q, k, v, o, lse, scale,
                                                                   o_scale, tok_in, stream);
       case 256:
-        return run_single<T, FwdTraits<256, 64, 2, 2>>(s, q, k, v, o, lse, scale, o_scale,
-                                                        tok_in, stream);
+        return run_single<T, FwdTraits<256, 128, 1, 1>>(s, q, k, v, o, lse, scale, o_scale,
+                                                          tok_in, stream);
       default:
         return FA_ERR_HEADDIM;
     }

@@ -248,7 +248,7 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
 typedef struct fa_fwd_plan {
     int kernel;          /* 1: two 128-row Q tiles a unit, 0: one tile a unit   */
     int unit_rows;       /* query rows per unit (256 or 128)                    */
-    int kv_tile_rows;    /* rows per K/V tile (128, or 64 at d = 256)           */
+    int kv_tile_rows;    /* rows per K/V tile (128)                              */
     int n_units;         /* B * H * ceil(N / unit_rows) * n_split               */
     int n_kv_tiles;      /* ceil(N / kv_tile_rows)                              */
     int n_split;         /* K/V shares per unit                                 */

@@ -104,7 +104,7 @@ def test_workload_plans():
     # the neck workload (one head, d = 256): 50 Q tiles, K/V range split in two
     plan = fa.fa_fwd_plan(1, 1, 6400, 256, 148)
     assert (plan["kernel"], plan["n_split"], plan["n_units"], plan["balanced"]) == (0, 2, 100, 0)
-    assert plan["kv_tile_rows"] == 64
+    assert plan["kv_tile_rows"] == 128
     # the detector deep stage: short units (4 K/V tiles) stay round-robin
     plan = fa.fa_fwd_plan(32, 4, 400, 64, 148)
     assert (plan["kernel"], plan["n_units"], plan["balanced"], plan["n_split"]) == (1, 256, 0, 1)
