@@ -582,6 +582,79 @@ __device__ __forceinline__ void store_row_staged(const FwdParams& p, const Unit&
   __syncwarp();  // the tile is rewritten by the next unit's epilogue
 }
 
+// Epilogue of one row in direct or split mode, through the warp's 4 KB
+// staging tile, 32 columns at a time: each thread writes its row's 32 output
+// values there (16-byte unit u of row r at unit position u ^ (r % units a
+// row)), then each warp store instruction covers whole 128-byte row pieces
+// (4 rows of fp32 partials, or 8 rows of 16-bit O) instead of 16 bytes of 32
+// rows.  PART: normalised fp32 partial rows and base-2 LSE of a K/V split;
+// otherwise O rounded to T and the natural-log LSE.  Collective over the warp.
+template <class T, int D, bool PART>
+__device__ __forceinline__ void store_row_chunked(const FwdParams& p, const Unit& un,
+                                                  uint32_t taddr, int q_row, float m, float l,
+                                                  uint8_t* stg) {
+  constexpr int EBO = PART ? 4 : 2;  // bytes an output element
+  constexpr int RB = 32 * EBO;       // bytes of a row's 32-column piece
+  constexpr int UPR = RB / 16;       // 16-byte units a piece: 8 or 4
+  constexpr int RPI = 32 / UPR;      // rows a warp store instruction covers
+  const int lane = threadIdx.x & 31;
+  const float inv_l = p.o_scale / l;
+  const float lse2 = m + lg2(l);
+  const int row0 = q_row - lane;  // the warp's first row
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(taddr + c * 32, o);
+    tmem_wait_ld();
+    reg_fence(o);
+#pragma unroll
+    for (int u = 0; u < UPR; ++u) {
+      uint4 v;
+      if constexpr (PART) {
+        v = make_uint4(__float_as_uint(__uint_as_float(o[4 * u]) * inv_l),
+                       __float_as_uint(__uint_as_float(o[4 * u + 1]) * inv_l),
+                       __float_as_uint(__uint_as_float(o[4 * u + 2]) * inv_l),
+                       __float_as_uint(__uint_as_float(o[4 * u + 3]) * inv_l));
+      } else {
+        v.x = Elem<T>::pack(__uint_as_float(o[8 * u]) * inv_l, __uint_as_float(o[8 * u + 1]) * inv_l);
+        v.y = Elem<T>::pack(__uint_as_float(o[8 * u + 2]) * inv_l,
+                            __uint_as_float(o[8 * u + 3]) * inv_l);
+        v.z = Elem<T>::pack(__uint_as_float(o[8 * u + 4]) * inv_l,
+                            __uint_as_float(o[8 * u + 5]) * inv_l);
+        v.w = Elem<T>::pack(__uint_as_float(o[8 * u + 6]) * inv_l,
+                            __uint_as_float(o[8 * u + 7]) * inv_l);
+      }
+      *reinterpret_cast<uint4*>(stg + lane * RB + ((u ^ (lane & (UPR - 1))) * 16)) = v;
+    }
+    __syncwarp();
+    const int u = lane % UPR;
+#pragma unroll
+    for (int it = 0; it < 32 / RPI; ++it) {
+      const int r = it * RPI + lane / UPR;
+      const uint4 v = *reinterpret_cast<const uint4*>(stg + r * RB + ((u ^ (r & (UPR - 1))) * 16));
+      const int row = row0 + r;
+      if (row < un.len) {
+        if constexpr (PART) {
+          float* orow =
+              p.o_part + ((((size_t)un.sp * p.B + un.b) * p.N + row) * p.H + un.h) * D + c * 32;
+          reinterpret_cast<uint4*>(orow)[u] = v;
+        } else {
+          const size_t tok = (size_t)un.tb * p.total + un.tok0 + row;
+          T* orow = reinterpret_cast<T*>(p.o) + (tok * p.H + un.h) * D + c * 32;
+          reinterpret_cast<uint4*>(orow)[u] = v;
+        }
+      }
+    }
+    __syncwarp();  // the tile is rewritten by the next piece
+  }
+  if (q_row < un.len) {
+    if constexpr (PART)
+      p.lse_part[(((size_t)un.sp * p.B + un.b) * p.H + un.h) * p.N + q_row] = lse2;
+    else
+      p.lse[((size_t)un.tb * p.H + un.h) * p.total + un.tok0 + q_row] = lse2 * kLn2;
+  }
+}
+
 // ===========================================================================
 // fa_fwd_pp_kernel: two Q tiles per unit
 // ===========================================================================
@@ -1029,7 +1102,8 @@ struct FwdTraits {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_STG = OFF_V + VST * KV_BYTES;  // 4 softmax warps x 4 KB (epilogue)
+  static constexpr int OFF_BAR = OFF_STG + 4 * 4096;
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST,
                        B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST,
                        B_S_FULL = B_V_EMPTY + VST, B_P_FULL = B_S_FULL + 2,
@@ -1277,8 +1351,15 @@ __global__ void __launch_bounds__(224, 1)
       ok = mbar_wait(bar(Tr::B_O_DONE), (g - 1) & 1u, w, kSiteEpi);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      ok = store_row<typename Elem<T>::Out, D>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l,
-                                               w);
+      // through the warp's staging tile: one thread a row would make every
+      // warp store touch 32 rows ([1,6400,1,256] split mode: the epilogue took
+      // a seventh of the kernel)
+      uint8_t* stg = gbase + Tr::OFF_STG + warp * 4096;
+      if (p.o_part != nullptr)
+        store_row_chunked<float, D, true>(p, un, tl + Tr::TM_O, un.qt * Tr::BM + row, m, l, stg);
+      else
+        store_row_chunked<typename Elem<T>::Out, D, false>(p, un, tl + Tr::TM_O,
+                                                            un.qt * Tr::BM + row, m, l, stg);
     }
   }
 
