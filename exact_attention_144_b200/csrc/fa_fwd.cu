@@ -22,9 +22,11 @@
 //   and both Q tiles share every K/V tile loaded into shared memory.
 //
 // fa_fwd_kernel (any d, used for d = 256 and short sequences; 224 threads) --
-//   one 128-row Q tile per unit, S double buffered in TMEM
-//   warps 0-3 softmax + epilogue, warp 4 Q/K producer, warp 5 V producer,
-//   warp 6 TMEM allocator + MMA issuer.
+//   one 128-row Q tile per unit, S double buffered in TMEM, 128-key K/V
+//   tiles (at d = 256: 2 x 128 S columns + 256 O columns = all of TMEM, and
+//   one K and one V stage of 64 KB)
+//   warps 0-3 softmax + epilogue (through per-warp staging tiles), warp 4
+//   Q/K producer, warp 5 V producer, warp 6 TMEM allocator + MMA issuer.
 //
 // Shared-memory tiles are rows of 64-element (128-byte, swizzled) chunks.  A
 // d = 96 head uses two chunks a row: the second TMA box reaches past the
