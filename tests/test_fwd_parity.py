@@ -57,6 +57,19 @@ def test_ragged_lengths_d64_bf16(fa, N):
     check_full(fa, 2, N, 3, 64, "bf16", 100 + N)
 
 
+@pytest.mark.parametrize("B,N,H,dtype", [(1, 3000, 1, "fp16"), (1, 2500, 1, "bf16"),
+                                         (1, 2000, 3, "bf16"), (1, 1537, 2, "fp16")])
+def test_d256_key_splits_with_ragged_last_tile(fa, B, N, H, dtype):
+    # d = 256 walks 128-key tiles with one K and one V stage.  These shapes cut
+    # the K/V range into 3, 2, 2 and 1 shares whose last tile is ragged (56,
+    # 68, 80 and 1 keys); split shares leave as fp32 partial rows through the
+    # per-warp staging tiles and are merged afterwards
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = fa.fa_fwd_plan(B, H, N, 256, sms)
+    assert plan["kernel"] == 0 and plan["kv_tile_rows"] == 128, plan
+    check_full(fa, B, N, H, 256, dtype, 3300 + N, std=0.5)
+
+
 @pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("N", [1, 65, 129, 300])
