@@ -168,6 +168,37 @@ def test_large_scale_is_stable(fa):
     assert err_stats(lse.cpu().double().numpy(), lse_ref)["max"] <= 1e-3 * 64
 
 
+@pytest.mark.parametrize("N,d,sign", [(128, 64, 1), (256, 64, 1), (256, 64, -1), (256, 128, 1),
+                                      (128, 256, 1), (256, 256, -1)])
+def test_row_max_in_last_column_group(fa, N, d, sign):
+    # Every row's dominant key sits in the last 8 columns of a 128-key tile,
+    # 200 above the other scores (2^288 in base 2): a row max that left those
+    # columns out would overflow the exponentials.  Rows of tile t's group use
+    # the directions 8 t .. 8 t + 7, so no two dominant keys tie.  N = 128 runs
+    # the single-tile kernel, N = 256 (d <= 128) the pair kernel; sign -1 takes
+    # the min branch (negative scale).
+    g = torch.Generator().manual_seed(77 + N + d)
+    n_t = N // 128
+    k = 0.01 * torch.randn(N, d, generator=g)
+    q = torch.zeros(N, d)
+    for t in range(n_t):
+        for j in range(8):
+            k[t * 128 + 120 + j] = 0.0
+            k[t * 128 + 120 + j, 8 * t + j] = 1.0
+    for i in range(N):
+        c = i % (8 * n_t)
+        q[i, c] = float(sign)
+    to_dev = lambda x: x.view(1, N, 1, d).to(torch.bfloat16).cuda()  # noqa: E731
+    q, k = to_dev(q), to_dev(k)
+    _, _, v = attn_inputs.draw(1, N, 1, d, "bf16", 406 + N + d, 3, device="cuda")
+    scale = 200.0 * sign
+    o, lse = run(fa, q, k, v, scale)
+    o_ref, lse_ref = oracle.attn_fwd(to64(q), to64(k), to64(v), scale)
+    assert np.all(np.isfinite(to64(o))) and np.all(np.isfinite(lse.cpu().numpy()))
+    assert err_stats(to64(o), o_ref)["max"] <= O_MAX
+    assert err_stats(lse.cpu().double().numpy(), lse_ref)["max"] <= LSE_MAX
+
+
 def test_deterministic(fa):
     w = attn_inputs.WORKLOADS["c3"]
     q, k, v = attn_inputs.draw_workload(w, count=3, device="cuda")
