@@ -235,13 +235,9 @@ __host__ __device__ __forceinline__ int pv_steps(int len, int t) {
 // time saved (225 -> 241 us), so there it is 0.
 // SKIP: partial tiles skip the 32-column chunks that hold no valid column of
 // any row of the warp (warp votes; all 32 lanes must call together).
-// PRE: `pre` holds the max of s*c's raw scores over columns [0, BN/2) (the
-// min when c < 0), taken by the caller while the other half was loading; a
-// full tile then scans only the second half (partial tiles scan everything).
-template <class T, int BN, int EMU = 0, bool SKIP = true, bool PRE = false>
+template <class T, int BN, int EMU = 0, bool SKIP = true>
 __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], int valid, float c,
-                                              float& m, float& l, uint32_t (&pk)[BN / 2],
-                                              float pre = 0.f) {
+                                              float& m, float& l, uint32_t (&pk)[BN / 2]) {
   auto S = [&](int j) { return __uint_as_float(r[j / 32][j % 32]); };
   // full: every column of the row is valid.  With SKIP it is decided for the
   // whole warp: the partial path then takes warp votes, and a causal
@@ -253,39 +249,36 @@ __device__ __forceinline__ float softmax_step(const uint32_t (&r)[BN / 32][32], 
   // columns per three-input max
   float mx;
   if (full) {
-    // the 8-column groups of [J0, BN): group 0 starts the chains, the rest
+    // the 8-column groups of the row: group 0 starts the chains, the rest
     // are taken two at a time, and an odd last group alone
-    constexpr int J0 = PRE ? BN / 2 : 0;  // first column scanned here
-    constexpr int NG = (BN - J0) / 8;
+    constexpr int NG = BN / 8;
     float part[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) part[q] = S(J0 + q);
+    for (int q = 0; q < 8; ++q) part[q] = S(q);
     if (!neg) {
 #pragma unroll
       for (int gi = 1; gi + 1 < NG; gi += 2)
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          part[q] = max3f(part[q], S(J0 + 8 * gi + q), S(J0 + 8 * gi + 8 + q));
+          part[q] = max3f(part[q], S(8 * gi + q), S(8 * gi + 8 + q));
       if constexpr ((NG - 1) % 2 == 1) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) part[q] = fmaxf(part[q], S(BN - 8 + q));
       }
       mx = max3f(max3f(part[0], part[1], part[2]), max3f(part[3], part[4], part[5]),
                  fmaxf(part[6], part[7]));
-      if (PRE) mx = fmaxf(mx, pre);
     } else {
 #pragma unroll
       for (int gi = 1; gi + 1 < NG; gi += 2)
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          part[q] = min3f(part[q], S(J0 + 8 * gi + q), S(J0 + 8 * gi + 8 + q));
+          part[q] = min3f(part[q], S(8 * gi + q), S(8 * gi + 8 + q));
       if constexpr ((NG - 1) % 2 == 1) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) part[q] = fminf(part[q], S(BN - 8 + q));
       }
       mx = min3f(min3f(part[0], part[1], part[2]), min3f(part[3], part[4], part[5]),
                  fminf(part[6], part[7]));
-      if (PRE) mx = fminf(mx, pre);
     }
   } else {
     // a partial tile (the ragged end of the keys, or the causal diagonal):
