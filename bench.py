@@ -55,22 +55,22 @@ ORACLE_BUDGET_GFLOP = 40.0
 # while the kernel sources' code (comments excluded) hashes to the recorded
 # value.
 TRAFFIC = {
-    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.761280e6 + 22.419456e6,
-                                                    "src": "cec083903dbc7875"},
-    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.456832e6 + 1.842176e6,
-                                                       "src": "cec083903dbc7875"},
-    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 51.304448e6 + 5.188352e6,
-                                                    "src": "cec083903dbc7875"},
-    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 101.656576e6 + 114.932480e6,
-                                                     "src": "cec083903dbc7875"},
-    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.282560e6 + 0.557568e6,
-                                                        "src": "cec083903dbc7875"},
-    ("fa_fwd_pp_kernel", "c2_detector_deep_b32_n400_h4_d64"): {"bytes": 19.759872e6,
-                                                               "src": "cec083903dbc7875"},
-    ("fa_fwd_kernel", "c3_detector_neck_n6400_h1_d256"): {"bytes": 9.940224e6,
-                                                          "src": "cec083903dbc7875"},
-    ("fa_bwd_tq_kernel", "c3_train_n6400_h1_d256"): {"bytes": 20.038144e6 + 7.941888e6,
-                                                     "src": "cec083903dbc7875"},
+    ("fa_bwd_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 101.761536e6 + 23.452672e6,
+                                                    "src": "83d013b47bf940ef"},
+    ("fa_fwd_pp_kernel", "c5_train_b4_n4096_h8_d64"): {"bytes": 50.483200e6 + 2.427392e6,
+                                                       "src": "83d013b47bf940ef"},
+    ("fa_fwd_pp_kernel", "c4_long_n8192_h8_d128"): {"bytes": 51.347456e6 + 4.947456e6,
+                                                    "src": "83d013b47bf940ef"},
+    ("fa_bwd_tq_kernel", "c4_train_n8192_h8_d128"): {"bytes": 102.718976e6 + 117.569280e6,
+                                                     "src": "83d013b47bf940ef"},
+    ("fa_fwd_pp_kernel", "c4_long_fp8_n8192_h8_d128"): {"bytes": 25.291776e6 + 0.559360e6,
+                                                        "src": "83d013b47bf940ef"},
+    ("fa_fwd_pp_kernel", "c2_detector_deep_b32_n400_h4_d64"): {"bytes": 19.760128e6,
+                                                               "src": "83d013b47bf940ef"},
+    ("fa_fwd_kernel", "c3_detector_neck_n6400_h1_d256"): {"bytes": 9.939200e6,
+                                                          "src": "83d013b47bf940ef"},
+    ("fa_bwd_tq_kernel", "c3_train_n6400_h1_d256"): {"bytes": 20.036864e6 + 6.463488e6,
+                                                     "src": "83d013b47bf940ef"},
 }
 
 
